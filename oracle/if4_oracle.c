@@ -1,0 +1,289 @@
+/*
+ * IF4 / NVFP4 CPU ORACLE -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, scalar C statement of what the IF4 quantizer and dequantizer
+ * compute, written from the pages on "Adaptive Block-Scaled Data Types"
+ * (Cook et al., arXiv 2603.28765).  Only the test suite, the smoke check and
+ * the CPU-baseline leg of the benchmark may load it.  It shares no code, table
+ * or header with the CUDA library, and the CUDA library never calls it.
+ *
+ * Arithmetic: IEEE binary32 for every value the format defines (compile with
+ * -O2 -ffp-contract=off, no fast-math, no flush-to-zero), binary64 for the
+ * per-group squared-error sums that decide FP4 vs INT4.
+ *
+ * Sources, by page and section:
+ *   [ABS]   the arXiv abstract (reprinted on shd-paper.top and fugumt.com):
+ *           groups of 16 values, an E4M3 scale per group "as is done with
+ *           NVFP4", the selected type kept in the scale's sign bit.
+ *   [FRAME] shd-paper.top, "Adaptive Block-Scaled Data Types", method details,
+ *           technical framework, steps 1-5: split into 16-blocks, evaluate the
+ *           FP4 and INT4 error, keep the lower, scale by E4M3, record the type
+ *           in the sign bit.
+ *   [SEL]   gist.science (pt), same title, section 2 "Metodologia",
+ *           "Mecanismo de Seleção": quantize to both, compute both MSEs, keep
+ *           the smaller.
+ *   [BIT]   gist.science section 2, "Codificação Eficiente": sign bit 0 = FP4,
+ *           1 = scaled INT4; and the episode companion "Adaptive Block-Scaled
+ *           Data Types for FP4 Training", "The Free Bit: Scale Factor Sign".
+ *   [67]    gist.science section 2, "Método 6/7": INT4 values are multiplied
+ *           by 7/6 before rounding and by 6/7 when used, so the largest value
+ *           is 6, as for FP4; companion, "One Group, Two Candidate Encodings".
+ *   [E2M1]  gist.science section 1 "O Problema": NVFP4 elements are E2M1.
+ *   [E4M3]  fugumt.com related entry "FP8 Formats for Deep Learning": E4M3
+ *           has no infinities and a single NaN mantissa pattern.
+ *
+ * Readings where the pages are silent (each listed in the design notes):
+ *   tensor scale ts = amax/(6*448), 1 for an all-zero tensor, and never
+ *   below 2^-117 so that every nonzero decoded block scale is a normal float;
+ *   block scale = (amax_g/6)/ts rounded to E4M3 by round-to-nearest-even with
+ *   saturation to 448 and subnormals kept; v = x * fl(1/eff); E2M1 and the
+ *   INT4 integer are round-to-nearest-even; FP4 zero keeps the sign of v;
+ *   INT4 codes are two's complement in [-7, 7]; the choice is INT4 only when
+ *   its error is strictly lower; a group whose block scale rounds to zero is
+ *   stored as all-zero FP4; the even element of a pair goes in the low nibble.
+ *
+ * Parity pins: every function here is checked by the non-GPU tests against
+ * brute force over the grids, a library float8 cast, closed-form values and
+ * hand-worked groups; none is "parity unpinned".
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* E2M1 magnitudes indexed by the 3-bit code [E2M1]. */
+static const float kE2M1Mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+/* ---------------------------------------------------------------- E4M3 ---- */
+
+/* Value of an E4M3 byte with bit 7 ignored: 4 exponent bits (bias 7), 3
+ * mantissa bits, exponent field 0 = subnormal (m * 2^-9), 0x7F = NaN. */
+float orc_e4m3_value(uint8_t b)
+{
+    int code = b & 0x7F;
+    int e = code >> 3, m = code & 7;
+    if (code == 0x7F) return NAN;
+    if (e == 0) return (float)ldexp((double)m, -9);
+    return (float)ldexp((double)(8 + m), e - 10);
+}
+
+/* Nearest E4M3 code to a non-negative float, ties to the even code,
+ * saturating at 448 (0x7E); never returns the NaN code for finite input. */
+uint8_t orc_e4m3_encode(float f)
+{
+    if (f != f) return 0x7F;
+    if (f <= 0.0f) return 0x00;
+    if (f >= 448.0f) return 0x7E;
+    int e2;
+    (void)frexp((double)f, &e2);         /* f in [2^(e2-1), 2^e2) */
+    int E = e2 - 1;
+    if (E < -6) E = -6;                  /* subnormal range: step 2^-9 */
+    /* f in units of 2^(E-3): exact power-of-two scaling, then RNE. */
+    double q = rint(ldexp((double)f, 3 - E));
+    /* normal: q in [8,16]; q == 16 carries into the next binade, which the
+     * additive code form below produces by itself.  subnormal: q in [0,8]. */
+    return (uint8_t)(((E + 7) << 3) + ((int)q - 8));
+}
+
+/* ---------------------------------------------------------------- E2M1 ---- */
+
+/* 4-bit FP4 nibble of v: bit 3 = sign of v (so a negative v that rounds to
+ * zero gives 0x8), bits 0-2 = magnitude code, round to nearest, ties to the
+ * even code, saturating at 6. */
+uint8_t orc_e2m1_nibble(float v)
+{
+    uint8_t sign = signbit(v) ? 8 : 0;
+    double a = fabs((double)v);
+    int c;
+    if (!(a <= 6.0)) {
+        c = 7;                           /* above 6 (or NaN): saturate */
+    } else if (a < 2.0) {
+        c = (int)rint(a * 2.0);          /* grid step 0.5, codes 0..4 */
+    } else if (a < 4.0) {
+        c = (int)rint(a) + 2;            /* grid step 1, codes 4..6 */
+    } else {
+        c = (int)rint(a * 0.5) + 4;      /* grid step 2, codes 6..7 */
+        if (c > 7) c = 7;
+    }
+    return (uint8_t)(sign | c);
+}
+
+float orc_e2m1_value(uint8_t nib)
+{
+    float m = kE2M1Mag[nib & 7];
+    return (nib & 8) ? -m : m;
+}
+
+/* ------------------------------------------------------ scaled INT4 ------- */
+
+/* t = fl(v * fl(7/6)) [67]; k = round-to-nearest-even(t) clamped to [-7, 7];
+ * the nibble is k in 4-bit two's complement (0x8 is never produced). */
+uint8_t orc_int4_nibble(float v)
+{
+    const float c76 = 7.0f / 6.0f;
+    float t = v * c76;
+    double k = rint((double)t);
+    if (!(k >= -7.0)) k = -7.0;          /* also maps NaN to -7 */
+    if (k > 7.0) k = 7.0;
+    return (uint8_t)(((int)k) & 0xF);
+}
+
+/* Decoded INT4 value fl(6k/7), k the sign-extended nibble [67]. */
+float orc_int4_value(uint8_t nib)
+{
+    int k = (nib & 8) ? (int)(nib & 0xF) - 16 : (int)(nib & 0xF);
+    return (float)(6 * k) / 7.0f;
+}
+
+/* ----------------------------------------------- tensor scale (A1, A2) ---- */
+
+float orc_tensor_amax(const float *x, int64_t rows, int64_t cols, int64_t ld)
+{
+    float amax = 0.0f;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            float a = fabsf(x[r * ld + c]);
+            if (a > amax || a != a) amax = a;
+        }
+    return amax;
+}
+
+/* ts = amax/(6*448) as an FP32 decode scale, as for NVFP4 [ABS]. */
+float orc_tensor_scale(float amax)
+{
+    const float floor_ts = 0x1p-117f;
+    if (amax == 0.0f) return 1.0f;
+    float ts = amax / 2688.0f;
+    return ts < floor_ts ? floor_ts : ts;
+}
+
+/* ------------------------------------------------- quantize (A3 - A6) ----- */
+
+enum { ORC_MODE_IF4 = 0, ORC_MODE_NVFP4 = 1 };
+
+/* Quantize one group of 16 floats.  Writes 8 code bytes and returns the
+ * scale byte.  e_fp / e_int receive the binary64 squared errors of the two
+ * candidates in the scaled domain; *near receives 1 when they differ by at
+ * most 1e-6 relative (or both are zero). */
+static uint8_t quantize_group(const float *x, float ts, int mode, uint8_t *codes,
+                              double *e_fp_out, double *e_int_out, uint8_t *near_out)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    float sb_f = (amax / 6.0f) / ts;
+    uint8_t sb = orc_e4m3_encode(sb_f);
+    if (sb == 0) {
+        memset(codes, 0, 8);
+        *e_fp_out = 0.0;
+        *e_int_out = 0.0;
+        *near_out = 1;
+        return 0x00;
+    }
+    float eff = orc_e4m3_value(sb) * ts;
+    float inv = 1.0f / eff;
+
+    uint8_t nf[16], ni[16];
+    double e_fp = 0.0, e_int = 0.0;
+    for (int i = 0; i < 16; ++i) {
+        float v = x[i] * inv;
+        nf[i] = orc_e2m1_nibble(v);
+        ni[i] = orc_int4_nibble(v);
+        double df = (double)v - (double)orc_e2m1_value(nf[i]);
+        double di = (double)v - (double)orc_int4_value(ni[i]);
+        e_fp = e_fp + df * df;
+        e_int = e_int + di * di;
+    }
+    int use_int4 = (mode == ORC_MODE_IF4) && (e_int < e_fp);
+    const uint8_t *n = use_int4 ? ni : nf;
+    for (int j = 0; j < 8; ++j)
+        codes[j] = (uint8_t)(n[2 * j] | (n[2 * j + 1] << 4));
+    double hi = e_fp > e_int ? e_fp : e_int;
+    *e_fp_out = e_fp;
+    *e_int_out = e_int;
+    *near_out = (uint8_t)(fabs(e_fp - e_int) <= 1e-6 * hi);
+    return (uint8_t)(sb | (use_int4 ? 0x80 : 0x00));
+}
+
+/* x: float [rows, ld] row-major, cols % 16 == 0.  codes: [rows, cols/2],
+ * scales: [rows, cols/16].  e_fp, e_int, near: [rows, cols/16] or NULL. */
+void orc_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld, float ts,
+                  int mode, uint8_t *codes, uint8_t *scales, double *e_fp,
+                  double *e_int, uint8_t *near, int nthreads)
+{
+    int64_t gpr = cols / 16;
+#ifdef _OPENMP
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+#endif
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < gpr; ++g) {
+            double ef, ei;
+            uint8_t nt;
+            int64_t gi = r * gpr + g;
+            scales[gi] = quantize_group(x + r * ld + g * 16, ts, mode,
+                                        codes + r * (cols / 2) + g * 8, &ef, &ei, &nt);
+            if (e_fp) e_fp[gi] = ef;
+            if (e_int) e_int[gi] = ei;
+            if (near) near[gi] = nt;
+        }
+    }
+    (void)nthreads;
+}
+
+/* ------------------------------------------------------ dequantize (A7) --- */
+
+/* y[r, c] = fl(q * fl(E4(sb) * ts)), q decoded as FP4 or INT4 by bit 7. */
+void orc_dequantize(const uint8_t *codes, const uint8_t *scales, float ts, int64_t rows,
+                    int64_t cols, float *y, int nthreads)
+{
+    int64_t gpr = cols / 16;
+#ifdef _OPENMP
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+#endif
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < gpr; ++g) {
+            uint8_t sb = scales[r * gpr + g];
+            float eff = orc_e4m3_value(sb) * ts;
+            for (int i = 0; i < 16; ++i) {
+                uint8_t byte = codes[r * (cols / 2) + g * 8 + i / 2];
+                uint8_t nib = (i & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+                float q = (sb & 0x80) ? orc_int4_value(nib) : orc_e2m1_value(nib);
+                y[r * cols + g * 16 + i] = q * eff;
+            }
+        }
+    }
+    (void)nthreads;
+}
+
+int orc_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------- element functions over arrays ----- */
+/* Used by the tests to sweep large value sets through the scalar functions. */
+
+void orc_e4m3_encode_array(const float *f, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_encode(f[i]);
+}
+
+void orc_e2m1_nibble_array(const float *v, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_e2m1_nibble(v[i]);
+}
+
+void orc_int4_nibble_array(const float *v, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_int4_nibble(v[i]);
+}
