@@ -1,0 +1,190 @@
+// Device helpers for the IF4 kernels (sm_100a).  Thin wrappers over PTX
+// instructions; no IF4 policy lives here.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+
+namespace if4dev {
+
+// ------------------------------------------------------------ memory ----
+
+// 256-bit read-only load, not kept in L1 (every byte is read once).
+__device__ __forceinline__ void ld_nc_v8(const void *p, uint32_t (&r)[8])
+{
+    asm("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]),
+          "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+        : "l"(p));
+}
+
+__device__ __forceinline__ void ld_nc_v4(const void *p, uint32_t &a, uint32_t &b,
+                                         uint32_t &c, uint32_t &d)
+{
+    asm("ld.global.nc.L1::no_allocate.v4.b32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "l"(p));
+}
+
+__device__ __forceinline__ void ld_nc_v2(const void *p, uint32_t &a, uint32_t &b)
+{
+    asm("ld.global.nc.L1::no_allocate.v2.b32 {%0,%1}, [%2];" : "=r"(a), "=r"(b) : "l"(p));
+}
+
+__device__ __forceinline__ uint32_t ld_nc_u8(const void *p)
+{
+    uint16_t v;
+    asm("ld.global.nc.L1::no_allocate.u8 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_v8(void *p, const uint32_t (&r)[8])
+{
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 :: "l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]),
+                    "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]) : "memory");
+}
+
+__device__ __forceinline__ void st_v4(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};"
+                 :: "l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ void st_v2(void *p, uint32_t a, uint32_t b)
+{
+    asm volatile("st.global.v2.b32 [%0], {%1,%2};" :: "l"(p), "r"(a), "r"(b) : "memory");
+}
+
+__device__ __forceinline__ void st_u8(void *p, uint32_t v)
+{
+    asm volatile("st.global.u8 [%0], %1;" :: "l"(p), "h"((uint16_t)v) : "memory");
+}
+
+// ----------------------------------------------------- packed fp32 pairs --
+// sm_100 executes these as one instruction on a 64-bit register pair.
+
+typedef unsigned long long f2_t;
+
+__device__ __forceinline__ f2_t f2_pack(float lo, float hi)
+{
+    f2_t r;
+    asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(f2_t v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ f2_t f2_mul(f2_t a, f2_t b)
+{
+    f2_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ f2_t f2_add(f2_t a, f2_t b)
+{
+    f2_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ f2_t f2_sub(f2_t a, f2_t b)
+{
+    f2_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ f2_t f2_fma(f2_t a, f2_t b, f2_t c)
+{
+    f2_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// ------------------------------------------------------- conversions ----
+
+// Two floats -> one byte of two E2M1 codes (lo -> bits 0-3, hi -> bits 4-7),
+// round-to-nearest-even, saturating to +-6.
+__device__ __forceinline__ uint32_t e2m1x2_from_f32(float lo, float hi)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+        "cvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+// One byte of two E2M1 codes -> f16x2 (bits 0-3 -> low half).
+__device__ __forceinline__ uint32_t f16x2_from_e2m1x2(uint32_t byte)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.u8.u32 t, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(r) : "r"(byte));
+    return r;
+}
+
+// float -> E4M3 code, round-to-nearest-even, saturating to 448 (0x7E).
+__device__ __forceinline__ uint32_t e4m3_from_f32(float f)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(f));
+    return r & 0xFFu;
+}
+
+// E4M3 code (bits 0-6) -> float, exact (every E4M3 value is an f16 value).
+__device__ __forceinline__ float f32_from_e4m3(uint32_t code)
+{
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)(code & 0x7Fu)));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+__device__ __forceinline__ float f16lo_to_f32(uint32_t h2)
+{
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+__device__ __forceinline__ float f16hi_to_f32(uint32_t h2)
+{
+    return __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+}
+
+// two floats -> bf16x2 / f16x2, round-to-nearest-even (lo in bits 0-15)
+__device__ __forceinline__ uint32_t bf16x2_from_f32(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t f16x2_from_f32(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+// ----------------------------------------------------------- integers ----
+
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+}  // namespace if4dev

@@ -1,0 +1,158 @@
+/*
+ * if4.h -- C ABI of libif4.so: the IF4 (Int/Float 4) adaptive block-scaled
+ * 4-bit format on NVIDIA B200 (sm_100a).
+ *
+ * The format ("Adaptive Block-Scaled Data Types", Cook et al., arXiv
+ * 2603.28765; abstract, and gist.science section 2 "Metodologia"): a tensor
+ * is cut into groups of 16 consecutive values along its contiguous (last)
+ * dimension.  Each group shares one 8-bit E4M3 block scale, as in NVFP4, and
+ * stores its 16 values as 4-bit codes, either as E2M1 FP4 or as INT4 scaled
+ * by 7/6 (integers -7..7 that decode to k*6/7, so both grids end at 6; "Metodo
+ * 6/7").  The quantizer forms both candidates and keeps the one with the
+ * lower squared error ("Mecanismo de Selecao"; shd-paper.top, technical
+ * framework steps 1-5).  The choice lives in the scale byte's sign bit, which
+ * NVFP4 leaves unused: 0 = FP4, 1 = INT4 ("Codificacao Eficiente"; companion
+ * page "The Free Bit: Scale Factor Sign").  Storage is NVFP4's, 4.5 bits per
+ * value.  A per-tensor FP32 decode scale ts = amax/(6*448) sits above the
+ * block scales, as in NVFP4.
+ *
+ * Arithmetic contract (every step IEEE binary32, round-to-nearest-even):
+ *   ts    = amax_T / 2688  (1 if amax_T == 0; never below 2^-117)
+ *   sb    = E4M3_RNE_satfinite((amax_g / 6) / ts), subnormals kept
+ *   eff   = E4M3(sb) * ts,  inv = 1 / eff,  v_i = x_i * inv
+ *   FP4   : nibble = sign(v) | RNE_E2M1(|v|) saturating at 6 (a negative v
+ *           that rounds to zero keeps its sign: nibble 0x8)
+ *   INT4  : k = clamp(RNE(v * fl(7/6)), -7, 7), nibble = k & 0xF,
+ *           value fl(6k/7)
+ *   choice: INT4 iff sum (v - q_int)^2 < sum (v - q_fp)^2, the sums taken in
+ *           binary64 in element order; equal sums keep FP4.  (The kernels
+ *           decide in binary32 and redo the binary64 sums for any group
+ *           whose binary32 margin is within its rounding bound, so the
+ *           result equals the binary64 rule everywhere.)
+ *   sb == 0 (the block scale underflows): all nibbles 0, scale byte 0x00.
+ *   dequantize: y = fl(q * fl(E4M3(sb & 0x7F) * ts)), then rounded to the
+ *           output type.
+ *
+ * Layouts (all row-major, groups along the last dimension):
+ *   x      [rows, cols], row stride ld_x elements, cols % 16 == 0
+ *   codes  uint8 [rows, cols/2]  dense; byte j of a group holds element 2j in
+ *          its low nibble and element 2j+1 in its high nibble
+ *   scales uint8 [rows, cols/16] dense; bit 7 = type, bits 0-6 = E4M3 code
+ *   ts     one float in device memory
+ * NVFP4 output is valid IF4 with every bit 7 clear, so if4_dequantize also
+ * decodes NVFP4.
+ *
+ * Ownership and ordering: the caller allocates every buffer (device memory
+ * for all tensor and scalar arguments) and keeps it alive until the stream
+ * work completes.  Entry points validate arguments on the host, enqueue
+ * kernels on `stream` (a cudaStream_t; NULL = the legacy default stream) and
+ * return without synchronising.  They allocate no memory, keep no state
+ * between calls and may be called from several host threads.
+ *
+ * Errors: a nonzero if4_status is returned before anything is enqueued when
+ * an argument is invalid; IF4_ERR_CUDA reports a launch failure.  Problems
+ * only the device can see are OR-ed into *err_flag (a device int the caller
+ * zeroes; may be NULL where stated) as IF4_DEV_* bits and never trap.
+ */
+#ifndef IF4_H
+#define IF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    IF4_OK = 0,
+    IF4_ERR_NULL = 1,        /* a required pointer is NULL                      */
+    IF4_ERR_SHAPE = 2,       /* rows/cols < 0, cols % 16 != 0, ld too small, or
+                                a size beyond the stated maximum               */
+    IF4_ERR_DTYPE = 3,       /* unknown dtype code                              */
+    IF4_ERR_ALIGN = 4,       /* pointer or leading dimension misaligned         */
+    IF4_ERR_MODE = 5,        /* unknown ts_mode                                 */
+    IF4_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than required         */
+    IF4_ERR_CUDA = 7,        /* a CUDA call or kernel launch failed             */
+    IF4_ERR_DEVICE = 8       /* the current device is not sm_100 (B200)        */
+} if4_status;
+
+/* element types of dense tensors */
+typedef enum { IF4_F32 = 0, IF4_BF16 = 1, IF4_F16 = 2 } if4_dtype;
+
+/* tensor-scale modes of the quantizers */
+enum {
+    IF4_TS_COMPUTE = 0,      /* compute amax over x, write ts = amax/2688 to *ts */
+    IF4_TS_GIVEN = 1         /* read the caller's ts from *ts                   */
+};
+
+/* device-side error bits OR-ed into *err_flag */
+enum {
+    IF4_DEV_NONFINITE = 1,   /* an input element is Inf or NaN: outputs unspecified */
+    IF4_DEV_BAD_SCALE = 2,   /* a given ts is not finite or outside [2^-117, 2^117] */
+    IF4_DEV_TIMEOUT = 4      /* a pipeline wait in the linear ran out of its bound  */
+};
+
+/* Largest supported tensor: rows * cols / 16 < 2^31 groups. */
+
+/*
+ * A1: amax = max |x| over x[rows, cols] (device float).  x_dtype is IF4_F32,
+ * IF4_BF16 or IF4_F16; x 16-byte aligned, ld_x*elem_size % 16 == 0.
+ * err_flag may be NULL; otherwise IF4_DEV_NONFINITE is set for Inf/NaN.
+ * (The tensor scale of NVFP4-style formats; arXiv abstract.)
+ */
+int if4_tensor_amax(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                    float *amax, int *err_flag, void *stream);
+
+/* A2: ts = amax / 2688 (1 if amax == 0, floored at 2^-117), device to device. */
+int if4_tensor_scale(const float *amax, float *ts, void *stream);
+
+/*
+ * A1-A6: IF4 quantize.  Per group of 16: the E4M3 block scale, the FP4 and
+ * the 7/6-scaled INT4 candidates, the lower-error choice in bit 7 of the
+ * scale byte (gist.science section 2; shd-paper.top framework steps 1-5).
+ * ts_mode IF4_TS_COMPUTE runs A1/A2 first and writes *ts; IF4_TS_GIVEN reads
+ * it.  codes must be 16-byte aligned.  err_flag may be NULL.
+ */
+int if4_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                 uint8_t *codes, uint8_t *scales, float *ts, int ts_mode,
+                 int *err_flag, void *stream);
+
+/*
+ * A9: NVFP4 quantize, the comparator: the FP4 candidate of if4_quantize for
+ * every group, bit 7 of every scale byte 0.  Same arguments and rules.
+ */
+int nvfp4_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                   uint8_t *codes, uint8_t *scales, float *ts, int ts_mode,
+                   int *err_flag, void *stream);
+
+/*
+ * A7: dequantize IF4 (or NVFP4) to y[rows, cols] of y_dtype (IF4_F32,
+ * IF4_BF16 or IF4_F16), row stride ld_y elements: fl(q * fl(E4M3 * ts)),
+ * then RNE to the output type.  codes 16-byte aligned; y 16-byte aligned and
+ * ld_y*elem_size % 16 == 0.  (gist.science section 2, "Metodo 6/7";
+ * companion, "MAC Unit: Decoding Two Formats from One Sign Bit".)
+ */
+int if4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts,
+                   int64_t rows, int64_t cols, void *y, int y_dtype, int64_t ld_y,
+                   void *stream);
+
+/*
+ * First stage of the linear: y = fp16_RNE(fl(q * E4M3(sb))) [rows, cols],
+ * dense, i.e. the dequantized value with the tensor scale left out (exact for
+ * FP4 groups, rounded to 11 bits for INT4 groups).  y 16-byte aligned.
+ */
+int if4_decode_f16(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
+                   void *y, void *stream);
+
+/* Static description of a status code. */
+const char *if4_status_str(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int if4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IF4_H */

@@ -1,0 +1,131 @@
+"""The C ABI on a host without a GPU: libif4.so builds for sm_100a, loads,
+exports every function include/*.h declares, and rejects invalid arguments
+with the documented status before touching the device.  No kernel runs and
+no pointer passed here is dereferenced."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from adaptive_block_scaled_b200 import build
+    path = build.build()
+    L = ctypes.CDLL(path)
+    vp, i64, i = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    L.if4_quantize.argtypes = [vp, i, i64, i64, i64, vp, vp, vp, i, vp, vp]
+    L.nvfp4_quantize.argtypes = L.if4_quantize.argtypes
+    L.if4_dequantize.argtypes = [vp, vp, vp, i64, i64, vp, i, i64, vp]
+    L.if4_tensor_amax.argtypes = [vp, i, i64, i64, i64, vp, vp, vp]
+    L.if4_tensor_scale.argtypes = [vp, vp, vp]
+    L.if4_decode_f16.argtypes = [vp, vp, i64, i64, vp, vp]
+    L.if4_status_str.restype = ctypes.c_char_p
+    return L
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(",
+                             text, flags=re.M):
+            if not m.group(0).lstrip().startswith(("typedef", "enum", "struct", "#")):
+                names.append(m.group(1))
+    return sorted(set(names))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for n in ("if4_quantize", "nvfp4_quantize", "if4_dequantize", "if4_tensor_amax",
+              "if4_tensor_scale", "if4_decode_f16", "if4_status_str", "if4_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from adaptive_block_scaled_b200 import build
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in declared_functions():
+        assert n in exported, n
+        assert hasattr(lib, n)
+    # nothing but the C ABI leaks out (the static CUDA runtime stays local)
+    assert all(n.startswith(("if4_", "nvfp4_")) for n in exported), sorted(exported)[:10]
+
+
+def test_status_strings(lib):
+    assert lib.if4_version() >= 100
+    for s in range(9):
+        assert lib.if4_status_str(s)
+    assert b"unknown" in lib.if4_status_str(99)
+
+
+A = 0x100000          # a 256-byte aligned address; never dereferenced here
+
+
+@pytest.mark.parametrize("fn", ["if4_quantize", "nvfp4_quantize"])
+def test_quantize_host_validation(lib, fn):
+    f = getattr(lib, fn)
+    # null input, codes, ts
+    assert f(None, 1, 4, 32, 32, A, A, A, 0, None, None) == 1
+    assert f(A, 1, 4, 32, 32, None, A, A, 0, None, None) == 1
+    assert f(A, 1, 4, 32, 32, A, A, None, 0, None, None) == 1
+    # shapes: cols % 16, negative sizes, ld < cols, too many groups
+    assert f(A, 1, 4, 24, 24, A, A, A, 0, None, None) == 2
+    assert f(A, 1, -1, 32, 32, A, A, A, 0, None, None) == 2
+    assert f(A, 1, 4, 32, 16, A, A, A, 0, None, None) == 2
+    assert f(A, 1, 1 << 31, 32, 32, A, A, A, 0, None, None) == 2
+    # dtype, mode
+    assert f(A, 7, 4, 32, 32, A, A, A, 0, None, None) == 3
+    assert f(A, 1, 4, 32, 32, A, A, A, 9, None, None) == 5
+    # alignment: x, ld, codes, ts
+    assert f(A + 8, 1, 4, 32, 32, A, A, A, 0, None, None) == 4
+    assert f(A, 1, 4, 32, 36, A, A, A, 0, None, None) == 4
+    assert f(A, 1, 4, 32, 32, A + 8, A, A, 0, None, None) == 4
+    assert f(A, 1, 4, 32, 32, A, A, A + 2, 0, None, None) == 4
+
+
+def test_dequantize_and_decode_host_validation(lib):
+    f = lib.if4_dequantize
+    assert f(None, A, A, 4, 32, A, 1, 32, None) == 1
+    assert f(A, A, None, 4, 32, A, 1, 32, None) == 1
+    assert f(A, A, A, 4, 40, A, 1, 40, None) == 2
+    assert f(A, A, A, 4, 32, A, 5, 32, None) == 3
+    assert f(A, A, A, 4, 32, A + 4, 1, 32, None) == 4
+    assert f(A + 1, A, A, 4, 32, A, 1, 32, None) == 4
+    g = lib.if4_decode_f16
+    assert g(None, A, 4, 32, A, None) == 1
+    assert g(A, A, 4, 33, A, None) == 2
+    assert g(A, A, 4, 32, A + 2, None) == 4
+
+
+def test_amax_and_scale_host_validation(lib):
+    assert lib.if4_tensor_amax(A, 1, 4, 32, 32, None, None, None) == 1
+    assert lib.if4_tensor_amax(A, 3, 4, 32, 32, A, None, None) == 3
+    assert lib.if4_tensor_amax(A, 0, 4, 32, 30, A, None, None) == 2
+    assert lib.if4_tensor_scale(None, A, None) == 1
+    assert lib.if4_tensor_scale(A + 1, A, None) == 4
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    """The Python binding has no fallback: a missing library is an error."""
+    import importlib
+    import sys
+    import adaptive_block_scaled_b200.build as b
+    saved = sys.modules.pop("adaptive_block_scaled_b200.binding", None)
+    monkeypatch.setattr(b, "LIB", str(tmp_path / "missing.so"))
+    try:
+        with pytest.raises(RuntimeError, match="not built"):
+            importlib.import_module("adaptive_block_scaled_b200.binding")
+    finally:
+        monkeypatch.undo()
+        sys.modules.pop("adaptive_block_scaled_b200.binding", None)
+        if saved is not None:
+            sys.modules["adaptive_block_scaled_b200.binding"] = saved
