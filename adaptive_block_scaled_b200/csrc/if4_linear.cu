@@ -1,0 +1,492 @@
+// IF4 x IF4 linear for B200 (sm_100a): decode both IF4 operands to fp16 with
+// the tensor scales factored out, then one dense tcgen05 GEMM with fp32
+// accumulation in tensor memory and the two tensor scales applied in the
+// epilogue.
+//
+// The pages' IF4 MAC routes every operand pair by its group's sign bit into
+// an FP4 or a 6/7-scaled INT4 decoder before multiplying (episode companion
+// "Adaptive Block-Scaled Data Types for FP4 Training", section "MAC Unit:
+// Decoding Two Formats from One Sign Bit").  B200 tensor cores have no IF4
+// type, so both decoders run once per operand element ahead of the GEMM: the
+// decoded value q * E4M3(scale) is exact in fp16 for FP4 groups and rounded
+// to 11 bits for INT4 groups, and the per-tensor scales (one float each)
+// factor out of the whole sum.
+//
+// GEMM structure (one CTA per SM, persistent over 128 x 256 output tiles):
+//   warp 0      TMA producer: 128B-swizzled 64-wide K slabs of A and B into a
+//               4-stage shared-memory ring (no multicast)
+//   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 accumulators)
+//               and one thread issues tcgen05.mma (M=128, N=256, K=16)
+//   warps 2-5   epilogue: tcgen05.ld of the finished accumulator, scale,
+//               bf16 RNE, global stores; the next tile's MMAs run meanwhile
+// Every mbarrier wait is bounded by a wall-clock limit; on expiry the kernel
+// sets IF4_DEV_TIMEOUT in the error word, stops issuing work, drains what is
+// in flight (bounded), frees its tensor memory and returns.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/if4.h"
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;                       // fp16: one 128-byte swizzle row
+constexpr int UMMA_K = 16;
+constexpr int STAGES = 4;
+constexpr int A_STAGE_BYTES = BM * BK * 2;   // 16 KB
+constexpr int B_STAGE_BYTES = BN * BK * 2;   // 32 KB
+constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+constexpr int TMEM_COLS = 2 * BN;            // two accumulators
+constexpr int NUM_THREADS = 192;             // 6 warps
+constexpr int EPI_WARP0 = 2;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;   // 1 s per wait
+
+// instruction descriptor, kind::f16: D f32, A f16, B f16, both K-major,
+// N = 256, M = 128
+constexpr uint32_t IDESC = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                           ((uint32_t)(BM >> 4) << 24);
+
+// ------------------------------------------------------------ PTX glue ----
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase of `parity` to complete.  Returns false (and
+// raises the CTA's abort flag) when the wall-clock limit runs out or another
+// role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 0u) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t bar)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3}], [%4];"
+                 :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map)
+{
+    asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row core-matrix groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((addr & 0x3FFFFu) >> 4);          // start address
+    d |= (uint64_t)1u << 16;                          // leading byte offset (unused)
+    d |= (uint64_t)(1024u >> 4) << 32;                // stride byte offset
+    d |= (uint64_t)1u << 46;                          // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                          // SWIZZLE_128B
+    return d;
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32"
+                 " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+                   "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]),
+                   "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+                   "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+                   "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void st_v4(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" :: "l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+// ------------------------------------------------------------- kernel ----
+
+struct TileIter {
+    int m_blocks, n_blocks, tiles;
+    __device__ void coords(int t, int &m0, int &n0) const
+    {
+        // consecutive tiles walk down M inside one column of N tiles, so the
+        // CTAs resident at one time share B slabs in L2
+        m0 = (t % m_blocks) * BM;
+        n0 = (t / m_blocks) * BN;
+    }
+};
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_f16_tcgen05(const __grid_constant__ CUtensorMap tmap_a,
+                 const __grid_constant__ CUtensorMap tmap_b,
+                 const float *__restrict__ a_ts, const float *__restrict__ b_ts,
+                 __nv_bfloat16 *__restrict__ c, int M, int N, int K, int *err)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem_a = smem;
+    uint8_t *smem_b = smem + STAGES * A_STAGE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    uint64_t *full = bars;                    // [STAGES]
+    uint64_t *empty = bars + STAGES;          // [STAGES]
+    uint64_t *acc_full = bars + 2 * STAGES;   // [2]
+    uint64_t *acc_empty = acc_full + 2;       // [2]
+    uint64_t *drain = acc_empty + 2;          // [1]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const TileIter it{(M + BM - 1) / BM, (N + BN - 1) / BN,
+                      ((M + BM - 1) / BM) * ((N + BN - 1) / BN)};
+    const int k_blocks = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&acc_full[b]), 1);
+            mbar_init(smem_u32(&acc_empty[b]), 4 * 32);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        prefetch_tmap(&tmap_a);
+        prefetch_tmap(&tmap_b);
+    }
+    if (warp == 1) {
+        __syncwarp();
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(tmem_slot)), "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0 && lane == 0) {
+        // ---------------------------------------------------- TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        int issued = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < it.tiles && ok; t += gridDim.x) {
+            int m0, n0;
+            it.coords(t, m0, n0);
+            for (int kb = 0; kb < k_blocks; ++kb) {
+                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) { ok = false; break; }
+                const uint32_t fb = smem_u32(&full[stage]);
+                mbar_expect_tx(fb, STAGE_BYTES);
+                tma_load_2d(smem_u32(smem_a + stage * A_STAGE_BYTES), &tmap_a, kb * BK, m0, fb);
+                tma_load_2d(smem_u32(smem_b + stage * B_STAGE_BYTES), &tmap_b, kb * BK, n0, fb);
+                ++issued;
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+        // every copy this thread issued must land before the CTA can exit:
+        // wait (bounded) for the last min(issued, STAGES) stages to fill
+        const int pending = issued < STAGES ? issued : STAGES;
+        for (int i = 0; i < pending; ++i) {
+            if (--stage < 0) { stage = STAGES - 1; phase ^= 1u; }
+            const unsigned long long t0 = globaltimer();
+            while (!mbar_try_wait(smem_u32(&full[stage]), phase))
+                if (globaltimer() - t0 > WAIT_LIMIT_NS) break;
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------------ MMA issuer
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < it.tiles && ok; t += gridDim.x) {
+            if (!mbar_wait(smem_u32(&acc_empty[acc]), acc_phase ^ 1u, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+            for (int kb = 0; kb < k_blocks; ++kb) {
+                if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(smem_a + stage * A_STAGE_BYTES);
+                const uint32_t b0 = smem_u32(smem_b + stage * B_STAGE_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                    umma_f16(d_tmem, smem_desc_sw128(a0 + kk * UMMA_K * 2),
+                             smem_desc_sw128(b0 + kk * UMMA_K * 2), (kb | kk) != 0 ? 1u : 0u);
+                }
+                umma_commit(smem_u32(&empty[stage]));
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            umma_commit(smem_u32(&acc_full[acc]));
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+        // all MMAs this thread issued complete before tensor memory is freed
+        umma_commit(smem_u32(drain));
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(smem_u32(drain), 0))
+            if (globaltimer() - t0 > WAIT_LIMIT_NS) break;
+    } else if (warp >= EPI_WARP0) {
+        // -------------------------------------------------------- epilogue
+        const int quarter = warp & 3;                 // TMEM lanes this warp may read
+        const int row_in_tile = quarter * 32 + lane;
+        const float scale = __fmul_rn(*a_ts, *b_ts);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < it.tiles; t += gridDim.x) {
+            int m0, n0;
+            it.coords(t, m0, n0);
+            // tcgen05.ld is warp-collective: every lane must take the same path
+            const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&acc_full[acc]), acc_phase,
+                                                              abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const int row = m0 + row_in_tile;
+            __nv_bfloat16 *crow = c + (int64_t)row * N;
+#pragma unroll 1
+            for (int chunk = 0; chunk < BN / 32; ++chunk) {
+                uint32_t r[32];
+                tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                              (uint32_t)(acc * BN + chunk * 32), r);
+                const int col0 = n0 + chunk * 32;
+                if (row < M) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int col = col0 + q * 8;
+                        if (col < N) {
+                            uint32_t p[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                p[e] = bf16x2(__fmul_rn(__uint_as_float(r[q * 8 + 2 * e]), scale),
+                                              __fmul_rn(__uint_as_float(r[q * 8 + 2 * e + 1]), scale));
+                            st_v4(crow + col, p[0], p[1], p[2], p[3]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&acc_empty[acc]));
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag && err) atomicOr(err, IF4_DEV_TIMEOUT);
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                     :: "r"(tmem_base), "r"(TMEM_COLS));
+    }
+}
+
+// ------------------------------------------------------------ host side ----
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// K-major fp16 matrix [rows, K] -> tensor map with a (64 x box_rows) box.
+bool make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count_checked(int &sms)
+{
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return IF4_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return IF4_ERR_CUDA;
+    if (major != 10) return IF4_ERR_DEVICE;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return IF4_ERR_CUDA;
+    return IF4_OK;
+}
+
+int check_gemm_args(const void *a, const void *b, const float *a_ts, const float *b_ts,
+                    int64_t M, int64_t N, int64_t K, const void *c, const int *err)
+{
+    if (!a || !b || !a_ts || !b_ts || !c || !err) return IF4_ERR_NULL;
+    if (M < 1 || N < 1 || K < 16 || K % 16 != 0 || N % 8 != 0) return IF4_ERR_SHAPE;
+    if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return IF4_ERR_SHAPE;
+    for (const void *p : {a, b, c})
+        if (reinterpret_cast<uintptr_t>(p) % 16 != 0) return IF4_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(a_ts) % 4 || reinterpret_cast<uintptr_t>(b_ts) % 4 ||
+        reinterpret_cast<uintptr_t>(err) % 4)
+        return IF4_ERR_ALIGN;
+    return IF4_OK;
+}
+
+int launch_gemm(const void *a, const void *b, const float *a_ts, const float *b_ts, int64_t M,
+                int64_t N, int64_t K, void *c, int *err, cudaStream_t st)
+{
+    int sms = 0;
+    int rc = sm_count_checked(sms);
+    if (rc != IF4_OK) return rc;
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, a, M, K, BM) || !make_map(&mb, b, N, K, BN)) return IF4_ERR_CUDA;
+    static std::once_flag attr_once;
+    static cudaError_t attr_rc = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_rc = cudaFuncSetAttribute(gemm_f16_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       SMEM_BYTES);
+    });
+    if (attr_rc != cudaSuccess) return IF4_ERR_CUDA;
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    gemm_f16_tcgen05<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(
+        ma, mb, a_ts, b_ts, static_cast<__nv_bfloat16 *>(c), (int)M, (int)N, (int)K, err);
+    return cudaGetLastError() == cudaSuccess ? IF4_OK : IF4_ERR_CUDA;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+int if4_gemm_f16(const void *a, const void *b, const float *a_ts, const float *b_ts, int64_t M,
+                 int64_t N, int64_t K, void *c, int *err_flag, void *stream)
+{
+    int rc = check_gemm_args(a, b, a_ts, b_ts, M, N, K, c, err_flag);
+    if (rc != IF4_OK) return rc;
+    return launch_gemm(a, b, a_ts, b_ts, M, N, K, c, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+size_t if4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 1 || N < 1 || K < 16 || K % 16 != 0) return 0;
+    return align_up((size_t)M * (size_t)K * 2, 256) + (size_t)N * (size_t)K * 2;
+}
+
+int if4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_ts,
+               const uint8_t *b_codes, const uint8_t *b_scales, const float *b_ts, int64_t M,
+               int64_t N, int64_t K, void *workspace, size_t ws_bytes, void *c, int *err_flag,
+               void *stream)
+{
+    if (!a_codes || !a_scales || !b_codes || !b_scales) return IF4_ERR_NULL;
+    int rc = check_gemm_args(a_codes, b_codes, a_ts, b_ts, M, N, K, c, err_flag);
+    if (rc != IF4_OK) return rc;
+    const size_t need = if4_linear_workspace_bytes(M, N, K);
+    if (workspace == nullptr || ws_bytes < need) return IF4_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return IF4_ERR_ALIGN;
+    uint8_t *wa = static_cast<uint8_t *>(workspace);
+    uint8_t *wb = wa + align_up((size_t)M * (size_t)K * 2, 256);
+    rc = if4_decode_f16(a_codes, a_scales, M, K, wa, stream);
+    if (rc != IF4_OK) return rc;
+    rc = if4_decode_f16(b_codes, b_scales, N, K, wb, stream);
+    if (rc != IF4_OK) return rc;
+    return launch_gemm(wa, wb, a_ts, b_ts, M, N, K, c, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

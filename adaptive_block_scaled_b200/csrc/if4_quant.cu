@@ -115,22 +115,26 @@ __device__ __forceinline__ float unpack_group(const Raw<DT> &r, f2_t (&x)[8], bo
 
 // ------------------------------------------------------- the quantizer ----
 
-// Candidates of one element pair.  fp4: byte of two E2M1 nibbles; r: the
-// INT4 integers as magic-biased floats (bits 0-3 = nibble); ef / ei: running
-// squared-error sums of the two candidates, one per lane.
-template <bool CLAMP>
-__device__ __forceinline__ void pair_candidates(f2_t v, uint32_t &fp4, f2_t &r,
-                                                f2_t &qf, f2_t &qi)
+// FP4 candidate of an element pair: the byte of two E2M1 nibbles (element
+// 2j low) and the two decoded values.
+__device__ __forceinline__ void fp4_pair(f2_t v, uint32_t &byte, f2_t &qf)
 {
     float v0, v1;
     f2_unpack(v, v0, v1);
-    fp4 = e2m1x2_from_f32(v0, v1);
-    uint32_t h = f16x2_from_e2m1x2(fp4);
+    byte = e2m1x2_from_f32(v0, v1);
+    const uint32_t h = f16x2_from_e2m1x2(byte);
     qf = f2_pack(f16lo_to_f32(h), f16hi_to_f32(h));
+}
 
+// INT4 candidate of an element pair: r = 1.5*2^23 + RNE(v * fl(7/6)), one
+// fused multiply-add, so the integer is the exact product rounded once (bits
+// 0-3 of r are the nibble); qi = fl(k * fl(6/7)) = fl(6k/7) for |k| <= 7.
+template <bool CLAMP>
+__device__ __forceinline__ void int4_pair(f2_t v, f2_t &r, f2_t &qi)
+{
     const f2_t C76 = f2_pack(c76(), c76());
     const f2_t M = f2_pack(kMagic, kMagic);
-    r = f2_add(f2_mul(v, C76), M);
+    r = f2_fma(v, C76, M);
     if constexpr (CLAMP) {
         float r0, r1;
         f2_unpack(r, r0, r1);
@@ -182,7 +186,7 @@ __device__ __noinline__ bool int4_wins_exact(const char *p, float inv)
         const float v = __fmul_rn(x, inv);
         const uint32_t h = f16x2_from_e2m1x2(e2m1x2_from_f32(v, 0.0f));
         const float qf = f16lo_to_f32(h);
-        float r = __fadd_rn(__fmul_rn(v, c76()), kMagic);
+        float r = __fmaf_rn(v, c76(), kMagic);
         r = fminf(fmaxf(r, kMagic - 7.0f), kMagic + 7.0f);
         const float qi = __fmul_rn(__fsub_rn(r, kMagic), c67());
         const double df = __dsub_rn((double)v, (double)qf);
@@ -198,19 +202,37 @@ struct GroupCode {
     uint32_t scale;    // scale byte
 };
 
+// Encode one group from its 16 inputs x (pairs), the block scale byte sb, the
+// reciprocal inv of the decoded scale and vmax = fl(amax * inv).
+//
+// Decision, fast path: each squared error is accumulated in binary32 from
+// d = fma(x, -inv, q), an explicit single rounding of q - x*inv (the square
+// does not see the sign).  Against the rule's d = v - q with v = fl(x*inv),
+// every d is off by at most half an ulp of v plus one rounding, and each sum
+// by at most 9 roundings; with Cauchy-Schwarz and vmax*sqrt(S) <= (vmax^2 +
+// S)/2 the difference of the two sums is off by less than 2^-20 S + 2^-21
+// vmax^2 + 2^-140.  Outside the band 2^-18 S + 2^-19 vmax^2 + 2^-126 the sign
+// of the binary32 difference is therefore the sign of the binary64 rule;
+// inside it the group is decided by the rule itself.
 template <int DT, bool IF4, bool CLAMP>
-__device__ __forceinline__ GroupCode encode_group(const f2_t (&v)[8], uint32_t sb,
-                                                const char *p, float inv)
+__device__ __forceinline__ GroupCode encode_group(const f2_t (&x)[8], uint32_t sb, float inv,
+                                                float vmax, const char *p)
 {
+    const f2_t INV = f2_pack(inv, inv);
+    const f2_t NINV = f2_pack(-inv, -inv);
     uint32_t fp4[8];
     f2_t r[8];
     f2_t ef = f2_pack(0.0f, 0.0f), ei = f2_pack(0.0f, 0.0f);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        f2_t qf, qi;
-        pair_candidates<CLAMP>(v[j], fp4[j], r[j], qf, qi);
+        const f2_t v = f2_mul(x[j], INV);
+        f2_t qf;
+        fp4_pair(v, fp4[j], qf);
         if constexpr (IF4) {
-            f2_t df = f2_sub(v[j], qf), di = f2_sub(v[j], qi);
+            f2_t qi;
+            int4_pair<CLAMP>(v, r[j], qi);
+            const f2_t df = f2_fma(x[j], NINV, qf);
+            const f2_t di = f2_fma(x[j], NINV, qi);
             ef = f2_fma(df, df, ef);
             ei = f2_fma(di, di, ei);
         }
@@ -225,11 +247,8 @@ __device__ __forceinline__ GroupCode encode_group(const f2_t (&v)[8], uint32_t s
         f2_unpack(ei, b0, b1);
         const float e_fp = __fadd_rn(a0, a1), e_int = __fadd_rn(b0, b1);
         const float d = __fsub_rn(e_fp, e_int);
-        // Each binary32 sum is within 9 roundings (+2 for a saturated
-        // difference) of the exact sum; 2^-18 relative plus 2^-126 absolute
-        // bounds the error of d with a wide margin, so outside that band the
-        // sign of d is the sign of the binary64 rule.
-        const float band = __fmaf_rn(__fadd_rn(e_fp, e_int), 0x1p-18f, 0x1p-126f);
+        const float band = __fmaf_rn(__fadd_rn(e_fp, e_int), 0x1p-18f,
+                                     __fmaf_rn(__fmul_rn(vmax, vmax), 0x1p-19f, 0x1p-126f));
         bool int4;
         if (fabsf(d) > band)
             int4 = d > 0.0f;
@@ -301,18 +320,14 @@ quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, uint
         } else {
             const float eff = __fmul_rn(f32_from_e4m3(sb), ts);
             const float inv = __frcp_rn(eff);
-            const f2_t INV = f2_pack(inv, inv);
-            f2_t v[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = f2_mul(xv[j], INV);
-            // INT4 rounding needs a clamp only if some |t| can reach 7.5;
-            // t is monotonic in |x|, so the group's amax decides.
-            const float tmax = __fmul_rn(__fmul_rn(amax, inv), c76());
+            const float vmax = __fmul_rn(amax, inv);
             const char *gp = group_ptr(x, g, contig, gpr, ld_bytes, GB);
-            if (tmax >= 7.5f)
-                out = encode_group<DT, IF4, true>(v, sb, gp, inv);
+            // The INT4 integer needs a clamp only if some |v| * fl(7/6) can
+            // reach 7.5; |v| is monotonic in |x|, so the group's max decides.
+            if (__fmul_rn(vmax, c76()) >= 7.5f)
+                out = encode_group<DT, IF4, true>(xv, sb, inv, vmax, gp);
             else
-                out = encode_group<DT, IF4, false>(v, sb, gp, inv);
+                out = encode_group<DT, IF4, false>(xv, sb, inv, vmax, gp);
         }
         st_v2(codes + (int64_t)g * 8, out.c0, out.c1);
         st_u8(scales + g, out.scale);

@@ -47,7 +47,7 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-linear", action="store_true")
     p.add_argument("--kernel-only", default=None,
-                   choices=["amax", "if4_quantize", "if4_dequantize", "nvfp4_quantize"],
+                   choices=["amax", "if4_quantize", "if4_dequantize", "nvfp4_quantize", "gemm"],
                    help="launch only this kernel, warmup+steps times (for ncu captures)")
     return p.parse_args()
 
@@ -360,8 +360,63 @@ def quality_report(x_cpu, step):
             "note": "IF4 MSE measured on the bf16 dequantized output; NVFP4 on fp32 dequant"}
 
 
-def linear_report(pk):
-    return None
+def linear_report(pk, steps=20, warmup=3):
+    """IF4 x IF4 linear on its own workload (A 8192x4096 activations, B
+    4096x4096 weights, both IF4 along K): decode A, decode B, tcgen05 GEMM,
+    each timed with CUDA events; cuBLAS fp16 on the same decoded operands is
+    timed beside it for context.  Inputs stay resident; the operands (100 MB
+    of fp16 after decode) are re-read from HBM/L2 every launch."""
+    from adaptive_block_scaled_b200 import binding as b
+    M, N, K = 8192, 4096, 4096
+    a, bw = make_input("linear_8192x4096x4096")
+    dev = torch.device("cuda")
+    aq = b.quantize(a.to(dev))
+    bq = b.quantize(bw.to(dev))
+    ws = torch.empty(b.if4_linear_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+    wa = ws[: M * K * 2].view(torch.float16).view(M, K)
+    off = ((M * K * 2 + 255) // 256) * 256
+    wb = ws[off: off + N * K * 2].view(torch.float16).view(N, K)
+    c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def run(ev=None):
+        if ev: ev[0].record()
+        b.if4_decode_f16(aq[0], aq[1], wa)
+        if ev: ev[1].record()
+        b.if4_decode_f16(bq[0], bq[1], wb)
+        if ev: ev[2].record()
+        b.if4_gemm_f16(wa, wb, aq[2], bq[2], c, err)
+        if ev: ev[3].record()
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        run(evs[i])
+    torch.cuda.synchronize()
+    t = [sum(e[k].elapsed_time(e[k + 1]) for e in evs) / steps for k in range(3)]
+    ref = torch.empty((M, N), dtype=torch.float16, device=dev)
+    for _ in range(warmup):
+        torch.matmul(wa, wb.t(), out=ref)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(steps):
+        torch.matmul(wa, wb.t(), out=ref)
+    e1.record()
+    torch.cuda.synchronize()
+    t_cublas = e0.elapsed_time(e1) / steps
+    flops = 2.0 * M * N * K
+    gemm_tf = flops / (t[2] * 1e-3) / 1e12
+    total = sum(t)
+    return {"workload": "linear_8192x4096x4096", "err": int(err.item()),
+            "decode_a_ms": t[0], "decode_b_ms": t[1], "gemm_ms": t[2], "linear_ms": total,
+            "gemm_tflops": gemm_tf, "linear_tflops": flops / (total * 1e-3) / 1e12,
+            "cublas_f16_ms": t_cublas, "cublas_f16_tflops": flops / (t_cublas * 1e-3) / 1e12,
+            "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": gemm_tf / pk["bf16_tflops"],
+                         "peak_source": f"{pk['source']} bf16_tflops (burst); fp16 dense rate = bf16"}}
 
 
 def run_ours(args):
@@ -458,6 +513,20 @@ def run_ours(args):
 def run_kernel_only(args):
     """Only the chosen kernel, on the chosen workload: the command ncu wraps."""
     from adaptive_block_scaled_b200 import binding as b
+    if args.kernel_only == "gemm":
+        M, N, K = 8192, 4096, 4096
+        a, bw = make_input("linear_8192x4096x4096")
+        dev = torch.device("cuda")
+        aq, bq = b.quantize(a.to(dev)), b.quantize(bw.to(dev))
+        wa, wb = b.decode_f16(aq[0], aq[1]), b.decode_f16(bq[0], bq[1])
+        c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        for _ in range(args.warmup + args.steps):
+            b.if4_gemm_f16(wa, wb, aq[2], bq[2], c, err)
+        torch.cuda.synchronize()
+        print(json.dumps({"kernel_only": "gemm", "launches": args.warmup + args.steps,
+                          "err": int(err.item())}))
+        return
     x_cpu = make_input(args.workload)
     step = Step(x_cpu, sets=1)
     s = step.sets[0]

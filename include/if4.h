@@ -145,6 +145,35 @@ int if4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts,
 int if4_decode_f16(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t cols,
                    void *y, void *stream);
 
+/*
+ * Second stage of the linear: C[M, N] = bf16_RNE(fl(a_ts * b_ts) * sum_k
+ * A[m, k] * B[n, k]) with A fp16 [M, K], B fp16 [N, K] dense and K-contiguous,
+ * products accumulated in fp32 by tcgen05 MMA.  a_ts, b_ts are device floats.
+ * M, N >= 1, K % 16 == 0, K >= 16; A, B, C 16-byte aligned, N % 8 == 0.
+ * err_flag must not be NULL (IF4_DEV_TIMEOUT).
+ */
+int if4_gemm_f16(const void *a, const void *b, const float *a_ts, const float *b_ts,
+                 int64_t M, int64_t N, int64_t K, void *c, int *err_flag, void *stream);
+
+/* Workspace the linear needs: two fp16 operand buffers, (M + N) * K * 2 bytes
+ * plus alignment padding; 0 for invalid sizes. */
+size_t if4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * A8: IF4 x IF4 linear.  C[M, N] (bf16, dense) = sum_k A_hat[m, k] *
+ * B_hat[n, k] where A (activations, [M, K]) and B (weights, [N, K], i.e. C =
+ * A B^T) are both IF4 along K.  Runs if4_decode_f16 on both operands into
+ * the caller's workspace, then if4_gemm_f16 with the two tensor scales in
+ * its epilogue.  The pages' MAC routes each operand pair by the sign bit
+ * into one of two decoders (companion, "MAC Unit: Decoding Two Formats from
+ * One Sign Bit"); here both decoders run ahead of a dense tensor-core GEMM.
+ * err_flag must not be NULL.
+ */
+int if4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_ts,
+               const uint8_t *b_codes, const uint8_t *b_scales, const float *b_ts,
+               int64_t M, int64_t N, int64_t K, void *workspace, size_t ws_bytes,
+               void *c, int *err_flag, void *stream);
+
 /* Static description of a status code. */
 const char *if4_status_str(int status);
 

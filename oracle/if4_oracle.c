@@ -36,8 +36,10 @@
  *   tensor scale ts = amax/(6*448), 1 for an all-zero tensor, and never
  *   below 2^-117 so that every nonzero decoded block scale is a normal float;
  *   block scale = (amax_g/6)/ts rounded to E4M3 by round-to-nearest-even with
- *   saturation to 448 and subnormals kept; v = x * fl(1/eff); E2M1 and the
- *   INT4 integer are round-to-nearest-even; FP4 zero keeps the sign of v;
+ *   saturation to 448 and subnormals kept; v = x * fl(1/eff); E2M1 is
+ *   round-to-nearest-even of v; the INT4 integer is round-to-nearest-even of
+ *   the exact product v * fl(7/6) (a single rounding); FP4 zero keeps the
+ *   sign of v;
  *   INT4 codes are two's complement in [-7, 7]; the choice is INT4 only when
  *   its error is strictly lower; a group whose block scale rounds to zero is
  *   stored as all-zero FP4; the even element of a pair goes in the low nibble.
@@ -118,13 +120,14 @@ float orc_e2m1_value(uint8_t nib)
 
 /* ------------------------------------------------------ scaled INT4 ------- */
 
-/* t = fl(v * fl(7/6)) [67]; k = round-to-nearest-even(t) clamped to [-7, 7];
- * the nibble is k in 4-bit two's complement (0x8 is never produced). */
+/* k = round-to-nearest-even(v * c) with c = fl(7/6), the product taken
+ * exactly (one rounding, to the integer) [67]; k is clamped to [-7, 7] and
+ * stored in 4-bit two's complement (0x8 is never produced).  Both factors
+ * are binary32, so their product is exact in binary64. */
 uint8_t orc_int4_nibble(float v)
 {
     const float c76 = 7.0f / 6.0f;
-    float t = v * c76;
-    double k = rint((double)t);
+    double k = rint((double)v * (double)c76);
     if (!(k >= -7.0)) k = -7.0;          /* also maps NaN to -7 */
     if (k > 7.0) k = 7.0;
     return (uint8_t)(((int)k) & 0xF);

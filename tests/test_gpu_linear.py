@@ -1,0 +1,140 @@
+"""GPU tests of the IF4 x IF4 linear, through the C ABI.
+
+The GEMM stage alone (if4_gemm_f16) is compared with a float64 product of
+its fp16 operands on small and ragged shapes.  The whole linear is compared
+with the oracle's float64 product of the dequantized IF4 operands:
+max |C - R| / max |R| <= 1e-2 (the stated tolerance), on sampled full rows
+and columns at 8192 x 4096 x 4096 and on every entry at 512 x 512 x 4096.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from adaptive_block_scaled_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def B():
+    from adaptive_block_scaled_b200 import binding
+    return binding
+
+
+def gemm(a, b, a_ts=1.0, b_ts=1.0):
+    bb = B()
+    M, N = a.shape[0], b.shape[0]
+    c = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ta = torch.tensor([a_ts], dtype=torch.float32, device="cuda")
+    tb = torch.tensor([b_ts], dtype=torch.float32, device="cuda")
+    bb.if4_gemm_f16(a, b, ta, tb, c, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    return c
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 264, 80), (1, 8, 16), (300, 520, 4096),
+                                   (1024, 1024, 4096), (129, 257 + 7, 1008), (2048, 4096, 512)])
+def test_gemm_f16_against_float64(M, N, K):
+    g = torch.Generator().manual_seed(M * 7 + N * 3 + K)
+    a = torch.randn((M, K), generator=g).to(torch.float16)
+    b = (torch.randn((N, K), generator=g) * 0.1).to(torch.float16)
+    s_a, s_b = 0.75, 1.25
+    c = gemm(a.cuda(), b.cuda(), s_a, s_b).float().cpu().numpy()
+    a64, b64 = a.double().numpy(), b.double().numpy()
+    ref = (a64 @ b64.T) * (np.float32(s_a) * np.float32(s_b))
+    mag = (np.abs(a64) @ np.abs(b64).T) * s_a * s_b
+    assert np.all(np.isfinite(c))
+    err = np.abs(c - ref)
+    tol = 2.0 ** -8 * np.abs(ref) + 1e-5 * mag + 1e-30
+    assert np.all(err <= tol), (float(err.max()), int((err > tol).sum()))
+
+
+def test_gemm_does_not_write_outside_c():
+    bb = B()
+    M, N, K = 130, 264, 96
+    a = torch.randn((M, K)).to(torch.float16).cuda()
+    b = torch.randn((N, K)).to(torch.float16).cuda()
+    big = torch.full((M + 2, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    c = big[1:M + 1]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    one = torch.ones(1, dtype=torch.float32, device="cuda")
+    bb.if4_gemm_f16(a, b, one, one, c, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.all(big[0] == 7.0) and torch.all(big[M + 1] == 7.0)
+
+
+def _quantized(x):
+    codes, scales, ts = B().quantize(x.cuda())
+    return codes, scales, ts
+
+
+def _linear(aq, bq, M, N, K):
+    bb = B()
+    ws = torch.empty(bb.if4_linear_workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
+    c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bb.if4_linear(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], ws, c, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    return c
+
+
+def _dequant_ref(q):
+    return oracle.dequantize(q[0].cpu().numpy(), q[1].cpu().numpy(), np.float32(q[2].item()))
+
+
+def _rel(c, ref):
+    return float(np.max(np.abs(c - ref)) / np.max(np.abs(ref)))
+
+
+def test_linear_full_check_512():
+    a, b = workloads.linear_operands(0, M=512, N=512, K=4096)
+    aq, bq = _quantized(a), _quantized(b)
+    c = _linear(aq, bq, 512, 512, 4096).float().cpu().numpy()
+    ref = oracle.linear(_dequant_ref(aq), _dequant_ref(bq))
+    rel = _rel(c, ref)
+    med = float(np.median(np.abs(c - ref) / np.maximum(np.abs(ref), 1e-30)))
+    print(f"[linear 512x512x4096] max|C-R|/max|R| = {rel:.3e}, median rel = {med:.3e}")
+    assert rel <= 1e-2
+
+
+def test_linear_workload_sampled_rows_and_columns():
+    M, N, K = 8192, 4096, 4096
+    a, b = workloads.linear_operands(0, M=M, N=N, K=K)
+    aq, bq = _quantized(a), _quantized(b)
+    c = _linear(aq, bq, M, N, K).float().cpu().numpy()
+    ah, bh = _dequant_ref(aq), _dequant_ref(bq)
+    rng = np.random.default_rng(11)
+    rows = np.sort(rng.choice(M, 128, replace=False))
+    cols = np.sort(rng.choice(N, 128, replace=False))
+    r_ref = oracle.linear(ah, bh, rows=rows)
+    c_ref = oracle.linear(ah, bh, cols=cols)
+    rel_r = _rel(c[rows], r_ref)
+    rel_c = _rel(c[:, cols], c_ref)
+    print(f"[linear 8192x4096x4096] rows {rel_r:.3e} cols {rel_c:.3e}")
+    assert rel_r <= 1e-2 and rel_c <= 1e-2
+
+
+def test_linear_ragged_shapes():
+    for (M, N, K) in [(100, 264, 48), (257, 136, 1040)]:
+        a, b = workloads.linear_operands(1, M=M, N=N, K=K)
+        aq, bq = _quantized(a), _quantized(b)
+        c = _linear(aq, bq, M, N, K).float().cpu().numpy()
+        ref = oracle.linear(_dequant_ref(aq), _dequant_ref(bq))
+        assert _rel(c, ref) <= 1e-2
+
+
+def test_linear_workspace_and_shape_errors():
+    bb = B()
+    assert bb.if4_linear_workspace_bytes(128, 256, 64) >= (128 + 256) * 64 * 2
+    assert bb.if4_linear_workspace_bytes(128, 256, 24) == 0
+    a, b = workloads.linear_operands(2, M=64, N=64, K=64)
+    aq, bq = _quantized(a), _quantized(b)
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    c = torch.empty((64, 64), dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(bb.IF4Error, match="workspace"):
+        bb.if4_linear(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], small, c, err)

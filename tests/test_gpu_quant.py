@@ -290,3 +290,39 @@ def test_repeated_calls_are_deterministic():
     torch.cuda.synchronize()
     for c, s, t in out[1:]:
         assert torch.equal(c, out[0][0]) and torch.equal(s, out[0][1]) and torch.equal(t, out[0][2])
+
+
+def _probe_groups(base15, probes):
+    """One group per probe value: 15 fixed values (max |x| = 6) and the probe
+    in the last slot, float32, ts = 1 so that v = x exactly."""
+    base = np.asarray(base15, np.float32)
+    x = np.empty((len(probes), 16), np.float32)
+    x[:, :15] = base
+    x[:, 15] = probes
+    return torch.from_numpy(x.reshape(-1, 256) if len(probes) % 16 == 0 else x)
+
+
+def _bf16_probe_values():
+    bits = (np.arange(65536, dtype=np.uint32) << 16).view(np.float32)
+    return bits[np.isfinite(bits) & (np.abs(bits) <= 6.0)]
+
+
+def test_int4_code_of_every_bf16_value():
+    """Groups where INT4 must win (15 values on the k*6/7 grid, off the FP4
+    grid), so the INT4 nibble of the probe is stored and compared."""
+    ks = [7, 6, 5, 4, 3, 2, 1, -1, -2, -3, -4, -5, -6, -7, 0]
+    base = [np.float32(6 * k) / np.float32(7) for k in ks]
+    probes = _bf16_probe_values()
+    x = _probe_groups(base, probes)
+    ref = check_quant(x, "int4 code of every bf16 value", ts=1.0)
+    assert (ref["scales"] & 0x80).all()
+
+
+def test_fp4_code_of_every_bf16_value():
+    """Groups where FP4 must win (15 values on the E2M1 grid), so the FP4
+    nibble of the probe is stored and compared."""
+    base = [6, 4, 3, 2, 1.5, 1, 0.5, -6, -4, -3, -2, -1.5, -1, -0.5, 0]
+    probes = _bf16_probe_values()
+    x = _probe_groups(base, probes)
+    ref = check_quant(x, "fp4 code of every bf16 value", ts=1.0)
+    assert not (ref["scales"] & 0x80).any()

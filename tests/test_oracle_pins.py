@@ -187,8 +187,10 @@ def test_int4_value_set():
 
 
 def brute_int4_nibble(v):
+    """Nearest integer in [-7, 7] to the exact product v * fl(7/6) (exact in
+    float64: 24-bit times 24-bit), ties to even."""
     v = np.asarray(v, np.float32)
-    t = (v * np.float32(np.float32(7.0) / np.float32(6.0))).astype(np.float64)
+    t = v.astype(np.float64) * np.float64(np.float32(7.0) / np.float32(6.0))
     t = np.clip(t, -1e4, 1e4)                             # see brute_e4m3_encode
     ks = np.arange(-7, 8, dtype=np.float64)
     dist = np.abs(t[:, None] - ks[None, :])
@@ -222,7 +224,10 @@ def test_int4_rounding_is_nearest_in_exact_arithmetic():
 
 
 def test_int4_named_cases():
-    assert oracle.int4_nibble(3.0) == 4          # t = 3.5 exactly -> 4 (even)
+    # 3 * fl(7/6) = 3.49999988..., just below the midpoint: k = 3 (the value
+    # 3 is equidistant from 18/7 and 24/7, so either k has the same error)
+    assert oracle.int4_nibble(3.0) == 3
+    assert oracle.int4_nibble(-3.0) == 0xD
     assert oracle.int4_nibble(6.0) == 7
     assert oracle.int4_nibble(-6.0) == 9         # -7
     assert oracle.int4_nibble(1e30) == 7 and oracle.int4_nibble(-1e30) == 9
