@@ -26,6 +26,7 @@ COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler",
 SOURCES = [
     ("if4_quant.cu", ["-fmad=false"]),
     ("if4_linear.cu", []),
+    ("if4_linear_noalloc.cu", []),
 ]
 HEADERS = ["if4_device.cuh", "exports.map"]
 

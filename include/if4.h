@@ -174,6 +174,30 @@ int if4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_t
                int64_t M, int64_t N, int64_t K, void *workspace, size_t ws_bytes,
                void *c, int *err_flag, void *stream);
 
+/* Size of the scratch array behind if4_linear_noalloc (32 MiB per device). */
+#define IF4_LINEAR_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
+
+/*
+ * if4_linear without a workspace argument, for callers that cannot provide
+ * device memory at the call: for example a plugin inside a framework that
+ * owns all device memory through its own pool, or a latency-critical path
+ * that must not risk the device synchronisation cudaMalloc can cause.  The
+ * pages have no counterpart; this is a deployment variant of A8.
+ * Same arguments and result as if4_linear.  The decoded operands live in a
+ * fixed scratch array in the library's device code (IF4_LINEAR_NOALLOC_MAX_BYTES
+ * per device, held from when the library's device code is loaded on that
+ * device until the process exits); it allocates nothing.  Problems whose
+ * if4_linear_workspace_bytes exceeds that size return IF4_ERR_WORKSPACE
+ * before anything is enqueued.  All calls on a device share the one array:
+ * calls whose work overlaps on the GPU race and corrupt each other, so order
+ * them (e.g. one stream).  The first call on each device looks up the
+ * array's address with that device current; make that first call before any
+ * stream capture.
+ */
+int if4_linear_noalloc(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_ts,
+                       const uint8_t *b_codes, const uint8_t *b_scales, const float *b_ts,
+                       int64_t M, int64_t N, int64_t K, void *c, int *err_flag, void *stream);
+
 /* Static description of a status code. */
 const char *if4_status_str(int status);
 
