@@ -25,6 +25,8 @@ _f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
 
 MODE_IF4 = 0
 MODE_NVFP4 = 1
+MODE_NVINT4 = 2
+MODE_4OVER6 = 3
 
 
 def lib():
@@ -61,6 +63,11 @@ def lib():
             fn = getattr(L, name)
             fn.argtypes = [_f32p, ctypes.c_int64, _u8p]
             fn.restype = None
+        L.orc_rht16.argtypes = [_f32p, ctypes.c_uint32, _f32p]
+        L.orc_rht16.restype = None
+        L.orc_rht.argtypes = [_f32p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                              ctypes.c_uint32, _f32p, ctypes.c_int]
+        L.orc_rht.restype = None
         L.orc_max_threads.argtypes = []
         L.orc_max_threads.restype = ctypes.c_int
         _LIB = L
@@ -140,7 +147,8 @@ def quantize(x, ts, mode: int = MODE_IF4, threads: int = 0):
 
     Returns dict(codes uint8 [rows, cols/2], scales uint8 [rows, cols/16],
     e_fp, e_int float64 [rows, cols/16] (scaled-domain squared errors of the
-    two candidates), near uint8 [rows, cols/16] (1 = the two errors are within
+    two candidates; for MODE_4OVER6 the x-domain errors of the /6 and the /4
+    candidates), near uint8 [rows, cols/16] (1 = the two errors are within
     1e-6 relative, or the group's block scale is zero)).
     """
     x = _as_f32_2d(x)
@@ -163,6 +171,21 @@ def quantize_tensor(x, mode: int = MODE_IF4, threads: int = 0):
     out = quantize(x, ts, mode, threads)
     out["amax"] = amax
     out["ts"] = ts
+    return out
+
+
+def rht(x, signs: int, threads: int = 0):
+    """y = H16 diag(s) x_g / 4 for every 16-group (see orc_rht16)."""
+    x = _as_f32_2d(x)
+    y = np.zeros_like(x)
+    lib().orc_rht(x, x.shape[0], x.shape[1], x.shape[1], int(signs) & 0xFFFF, y,
+                  int(threads) if threads else max_threads())
+    return y
+
+
+def quantize_tensor_rht(x, signs: int, mode: int = MODE_IF4, threads: int = 0):
+    """The transform, then A1-A6 on the transformed tensor."""
+    out = quantize_tensor(rht(x, signs, threads), mode, threads)
     return out
 
 

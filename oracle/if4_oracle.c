@@ -164,7 +164,14 @@ float orc_tensor_scale(float amax)
 
 /* ------------------------------------------------- quantize (A3 - A6) ----- */
 
-enum { ORC_MODE_IF4 = 0, ORC_MODE_NVFP4 = 1 };
+/* IF4: lower-error candidate per group.  NVFP4: FP4 always.  NVINT4: the
+ * 7/6-scaled INT4 candidate always, bit 7 set (the all-INT4 format the pages
+ * compare IF4 with: gist.science section 3, item 2; section 4, PTQ).
+ * 4/6 ("Four Over Six"): NVFP4 whose block scale maps the group maximum to 6
+ * or to 4, whichever reconstructs the group with the lower squared error in
+ * the x domain (gist.science section 1, third item: adapting the block
+ * maximum to 4 or 6); equal errors keep 6.  4/6 output is plain NVFP4. */
+enum { ORC_MODE_IF4 = 0, ORC_MODE_NVFP4 = 1, ORC_MODE_NVINT4 = 2, ORC_MODE_4OVER6 = 3 };
 
 /* Quantize one group of 16 floats.  Writes 8 code bytes and returns the
  * scale byte.  e_fp / e_int receive the binary64 squared errors of the two
@@ -201,7 +208,7 @@ static uint8_t quantize_group(const float *x, float ts, int mode, uint8_t *codes
         e_fp = e_fp + df * df;
         e_int = e_int + di * di;
     }
-    int use_int4 = (mode == ORC_MODE_IF4) && (e_int < e_fp);
+    int use_int4 = (mode == ORC_MODE_NVINT4) || ((mode == ORC_MODE_IF4) && (e_int < e_fp));
     const uint8_t *n = use_int4 ? ni : nf;
     for (int j = 0; j < 8; ++j)
         codes[j] = (uint8_t)(n[2 * j] | (n[2 * j + 1] << 4));
@@ -210,6 +217,48 @@ static uint8_t quantize_group(const float *x, float ts, int mode, uint8_t *codes
     *e_int_out = e_int;
     *near_out = (uint8_t)(fabs(e_fp - e_int) <= 1e-6 * hi);
     return (uint8_t)(sb | (use_int4 ? 0x80 : 0x00));
+}
+
+/* FP4 codes of a group under block scale byte sb; returns the binary64 sum
+ * of (x - xhat)^2 with xhat = fl(q * fl(E4(sb) * ts)), the dequantized value. */
+static double fp4_group_at_scale(const float *x, float ts, uint8_t sb, uint8_t *nib)
+{
+    float eff = orc_e4m3_value(sb) * ts;
+    float inv = sb ? 1.0f / eff : 0.0f;
+    double e = 0.0;
+    for (int i = 0; i < 16; ++i) {
+        float v = x[i] * inv;
+        nib[i] = sb ? orc_e2m1_nibble(v) : 0;
+        float xhat = orc_e2m1_value(nib[i]) * eff;
+        double d = (double)x[i] - (double)xhat;
+        e = e + d * d;
+    }
+    return e;
+}
+
+/* 4/6 for one group: candidates with block scales from amax/6 and amax/4. */
+static uint8_t quantize_group_4over6(const float *x, float ts, uint8_t *codes, double *e6_out,
+                                     double *e4_out, uint8_t *near_out)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    uint8_t sb6 = orc_e4m3_encode((amax / 6.0f) / ts);
+    uint8_t sb4 = orc_e4m3_encode((amax / 4.0f) / ts);
+    uint8_t n6[16], n4[16];
+    double e6 = fp4_group_at_scale(x, ts, sb6, n6);
+    double e4 = fp4_group_at_scale(x, ts, sb4, n4);
+    int use4 = e4 < e6;
+    const uint8_t *n = use4 ? n4 : n6;
+    for (int j = 0; j < 8; ++j)
+        codes[j] = (uint8_t)(n[2 * j] | (n[2 * j + 1] << 4));
+    double hi = e6 > e4 ? e6 : e4;
+    *e6_out = e6;
+    *e4_out = e4;
+    *near_out = (uint8_t)(fabs(e6 - e4) <= 1e-6 * hi);
+    return use4 ? sb4 : sb6;
 }
 
 /* x: float [rows, ld] row-major, cols % 16 == 0.  codes: [rows, cols/2],
@@ -228,13 +277,54 @@ void orc_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld, float 
             double ef, ei;
             uint8_t nt;
             int64_t gi = r * gpr + g;
-            scales[gi] = quantize_group(x + r * ld + g * 16, ts, mode,
-                                        codes + r * (cols / 2) + g * 8, &ef, &ei, &nt);
+            if (mode == ORC_MODE_4OVER6)
+                scales[gi] = quantize_group_4over6(x + r * ld + g * 16, ts,
+                                                   codes + r * (cols / 2) + g * 8, &ef, &ei, &nt);
+            else
+                scales[gi] = quantize_group(x + r * ld + g * 16, ts, mode,
+                                            codes + r * (cols / 2) + g * 8, &ef, &ei, &nt);
             if (e_fp) e_fp[gi] = ef;
             if (e_int) e_int[gi] = ei;
             if (near) near[gi] = nt;
         }
     }
+    (void)nthreads;
+}
+
+/* --------------------------------- random-sign Hadamard transform ------ */
+
+/* y = H16 diag(s) x / 4 for one group of 16, H16 the Sylvester Hadamard
+ * matrix (entry (i, j) = (-1)^popcount(i & j)) and s_j = -1 where bit j of
+ * `signs` is set: the orthonormal random-sign transform applied to weight
+ * gradients before quantization (gist.science section 1, second item;
+ * companion "Where the Gain Actually Comes From").  Evaluated as the fast
+ * Walsh-Hadamard transform in binary32: stages h = 1, 2, 4, 8, each replacing
+ * (y[i], y[i+h]) by (y[i] + y[i+h], y[i] - y[i+h]) for every i with bit h
+ * clear, then multiplied by 1/4 (exact). */
+void orc_rht16(const float *x, uint32_t signs, float *y)
+{
+    for (int j = 0; j < 16; ++j) y[j] = ((signs >> j) & 1u) ? -x[j] : x[j];
+    for (int h = 1; h < 16; h <<= 1)
+        for (int i = 0; i < 16; ++i)
+            if ((i & h) == 0) {
+                float a = y[i], b = y[i + h];
+                y[i] = a + b;
+                y[i + h] = a - b;
+            }
+    for (int j = 0; j < 16; ++j) y[j] = y[j] * 0.25f;
+}
+
+/* Apply orc_rht16 to every group of x [rows, ld] into y [rows, cols]. */
+void orc_rht(const float *x, int64_t rows, int64_t cols, int64_t ld, uint32_t signs, float *y,
+             int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+#endif
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t g = 0; g < cols / 16; ++g)
+            orc_rht16(x + r * ld + g * 16, signs, y + r * cols + g * 16);
     (void)nthreads;
 }
 
