@@ -46,7 +46,12 @@ def _load():
         "if4_tensor_scale": [_vp, _vp, _vp],
         "if4_quantize": [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _int, _vp, _vp],
         "nvfp4_quantize": [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _int, _vp, _vp],
+        "nvint4_quantize": [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _int, _vp, _vp],
+        "nvfp4_4over6_quantize": [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _int, _vp, _vp],
         "if4_dequantize": [_vp, _vp, _vp, _i64, _i64, _vp, _int, _i64, _vp],
+        "if4_tensor_amax_rht": [_vp, _int, _i64, _i64, _i64, ctypes.c_uint32, _vp, _vp, _vp],
+        "if4_quantize_rht": [_vp, _int, _i64, _i64, _i64, ctypes.c_uint32, _vp, _vp, _vp, _int,
+                             _vp, _vp],
         "if4_decode_f16": [_vp, _vp, _i64, _i64, _vp, _vp],
         "if4_gemm_f16": [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
         "if4_linear_workspace_bytes": [_i64, _i64, _i64],
@@ -135,6 +140,32 @@ def nvfp4_quantize(x, codes, scales, ts, ts_mode=TS_COMPUTE, err_flag=None, stre
                    stream)
 
 
+def if4_tensor_amax_rht(x, signs, amax, err_flag=None, stream=None):
+    rows, cols, ld = _matrix(x, "x")
+    _check(lib.if4_tensor_amax_rht(_ptr(x), _dtype(x, "x"), rows, cols, ld, int(signs) & 0xFFFF,
+                                   _ptr(amax), _ptr(err_flag), _stream(stream)),
+           "if4_tensor_amax_rht")
+
+
+def if4_quantize_rht(x, signs, codes, scales, ts, ts_mode=TS_COMPUTE, err_flag=None, stream=None):
+    rows, cols, ld = _matrix(x, "x")
+    _u8(codes, "codes", (rows, cols // 2))
+    _u8(scales, "scales", (rows, cols // 16))
+    _check(lib.if4_quantize_rht(_ptr(x), _dtype(x, "x"), rows, cols, ld, int(signs) & 0xFFFF,
+                                _ptr(codes), _ptr(scales), _ptr(ts), int(ts_mode), _ptr(err_flag),
+                                _stream(stream)), "if4_quantize_rht")
+
+
+def nvint4_quantize(x, codes, scales, ts, ts_mode=TS_COMPUTE, err_flag=None, stream=None):
+    _quantize_call(lib.nvint4_quantize, "nvint4_quantize", x, codes, scales, ts, ts_mode,
+                   err_flag, stream)
+
+
+def nvfp4_4over6_quantize(x, codes, scales, ts, ts_mode=TS_COMPUTE, err_flag=None, stream=None):
+    _quantize_call(lib.nvfp4_4over6_quantize, "nvfp4_4over6_quantize", x, codes, scales, ts,
+                   ts_mode, err_flag, stream)
+
+
 def if4_dequantize(codes, scales, ts, y, stream=None):
     rows, cols, ld = _matrix(y, "y")
     _u8(codes, "codes", (rows, cols // 2))
@@ -208,8 +239,9 @@ LINEAR_NOALLOC_MAX_BYTES = 32 * 1024 * 1024
 # ---------------------------------------------------- allocating helpers ---
 
 def quantize(x, mode="if4", ts=None, err_flag=None, stream=None):
-    """Quantize a 2-D tensor on its device.  Returns (codes, scales, ts).
-    ts=None computes the tensor scale; a float32 tensor is used as given."""
+    """Quantize a 2-D tensor on its device with mode "if4", "nvfp4", "nvint4"
+    or "4over6".  Returns (codes, scales, ts).  ts=None computes the tensor
+    scale; a float32 tensor is used as given."""
     rows, cols, _ = _matrix(x, "x")
     dev = x.device
     codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
@@ -218,8 +250,23 @@ def quantize(x, mode="if4", ts=None, err_flag=None, stream=None):
         ts_t, ts_mode = torch.empty(1, dtype=torch.float32, device=dev), TS_COMPUTE
     else:
         ts_t, ts_mode = ts, TS_GIVEN
-    fn = if4_quantize if mode == "if4" else nvfp4_quantize
+    fn = {"if4": if4_quantize, "nvfp4": nvfp4_quantize, "nvint4": nvint4_quantize,
+          "4over6": nvfp4_4over6_quantize}[mode]
     fn(x, codes, scales, ts_t, ts_mode, err_flag, stream)
+    return codes, scales, ts_t
+
+
+def quantize_rht(x, signs, ts=None, err_flag=None, stream=None):
+    """Random-sign Hadamard transform + IF4 quantize.  Returns (codes, scales, ts)."""
+    rows, cols, _ = _matrix(x, "x")
+    dev = x.device
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+    if ts is None:
+        ts_t, ts_mode = torch.empty(1, dtype=torch.float32, device=dev), TS_COMPUTE
+    else:
+        ts_t, ts_mode = ts, TS_GIVEN
+    if4_quantize_rht(x, signs, codes, scales, ts_t, ts_mode, err_flag, stream)
     return codes, scales, ts_t
 
 

@@ -30,6 +30,13 @@ __device__ __forceinline__ void ld_nc_v2(const void *p, uint32_t &a, uint32_t &b
     asm("ld.global.nc.L1::no_allocate.v2.b32 {%0,%1}, [%2];" : "=r"(a), "=r"(b) : "l"(p));
 }
 
+__device__ __forceinline__ uint32_t ld_nc_u32(const void *p)
+{
+    uint32_t v;
+    asm("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t ld_nc_u8(const void *p)
 {
     uint16_t v;
@@ -177,6 +184,22 @@ __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)
 {
     uint32_t r;
     asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// per 16-bit lane: max(|a|, |b|) with NaN propagated; the result's sign bit
+// is sign(a) ^ sign(b) and must be masked off by the caller
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t absmax_f16x2(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("max.NaN.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
     return r;
 }
 

@@ -36,12 +36,16 @@ namespace {
 __device__ __forceinline__ float c76() { return __uint_as_float(0x3F955555u); }
 __device__ __forceinline__ float c67() { return __uint_as_float(0x3F5B6DB7u); }
 constexpr float kMagic = 12582912.0f;
-constexpr uint32_t kMagicBits = 0x4B400000u;
 
 constexpr float kTsFloor = 0x1p-117f;
 constexpr float kTsCeil = 0x1p117f;
 
 enum { DT_F32 = IF4_F32, DT_BF16 = IF4_BF16, DT_F16 = IF4_F16 };
+
+// Quantizer modes: IF4 (lower-error candidate), NVFP4 (FP4 always), NVINT4
+// (7/6-scaled INT4 always), 4/6 (NVFP4 with the block maximum mapped to 6 or
+// to 4, lower x-domain error kept).
+enum { Q_IF4 = 0, Q_NVFP4 = 1, Q_NVINT4 = 2, Q_46 = 3 };
 
 // --------------------------------------------------------- group loads ----
 
@@ -92,17 +96,19 @@ __device__ __forceinline__ float unpack_group(const Raw<DT> &r, f2_t (&x)[8], bo
         nonfinite = m >= 0x7F800000u;
         return __uint_as_float(m);
     } else {
+        // max(|a|, |b|) per 16-bit lane in one instruction (the sign bit it
+        // leaves is ignored); NaN propagates, so Inf/NaN show up in the max
         uint32_t m = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            uint32_t w = r.w[j];
-            m = max_u16x2(m, w & 0x7FFF7FFFu);
+            const uint32_t w = r.w[j];
+            m = (DT == DT_BF16) ? absmax_bf16x2(m, w) : absmax_f16x2(m, w);
             if constexpr (DT == DT_BF16)
                 x[j] = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
             else
                 x[j] = f2_pack(f16lo_to_f32(w), f16hi_to_f32(w));
         }
-        uint32_t m16 = max(m & 0xFFFFu, m >> 16);
+        const uint32_t m16 = max(m & 0x7FFFu, (m >> 16) & 0x7FFFu);
         if constexpr (DT == DT_BF16) {
             nonfinite = m16 >= 0x7F80u;
             return __uint_as_float(m16 << 16);
@@ -113,24 +119,187 @@ __device__ __forceinline__ float unpack_group(const Raw<DT> &r, f2_t (&x)[8], bo
     }
 }
 
+// ------------------------------------- random-sign Hadamard transform ----
+//
+// y = H16 diag(s) x / 4 per group: the orthonormal random-sign transform the
+// pages apply to weight gradients before quantizing them (gist.science
+// section 1, second item; companion "Where the Gain Actually Comes From").
+// Evaluated in binary32 as the fast Walsh-Hadamard transform, stages h = 1,
+// 2, 4, 8 replacing (y[i], y[i+h]) by (y[i] + y[i+h], y[i] - y[i+h]) for i
+// with bit h clear, then times 1/4 (exact).
+
+// Sign flips as XOR masks on the raw words of a group: for 16-bit types word
+// j holds elements 2j and 2j+1 (bits 15 and 31), for f32 word i element i.
+struct SignMasks {
+    uint32_t w[16];
+};
+
+// The transform on the 8 element pairs of a group (pair j = elements 2j,
+// 2j+1): stage 1 inside each pair, stages 2, 4, 8 between pairs j and j + h/2.
+__device__ __forceinline__ void hadamard16(f2_t (&x)[8])
+{
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float a, b;
+        f2_unpack(x[j], a, b);
+        x[j] = f2_pack(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+#pragma unroll
+    for (int hp = 1; hp < 8; hp <<= 1) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if ((j & hp) == 0) {
+                const f2_t a = x[j], b = x[j + hp];
+                x[j] = f2_add(a, b);
+                x[j + hp] = f2_sub(a, b);
+            }
+        }
+    }
+    const f2_t Q = f2_pack(0.25f, 0.25f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = f2_mul(x[j], Q);
+}
+
+// The same transform on 16 scalars (the rare exact paths).
+__device__ __forceinline__ void hadamard16_scalar(float (&y)[16], uint32_t signs)
+{
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        if ((signs >> j) & 1u) y[j] = -y[j];
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if ((i & h) == 0) {
+                const float a = y[i], b = y[i + h];
+                y[i] = __fadd_rn(a, b);
+                y[i + h] = __fsub_rn(a, b);
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) y[j] = __fmul_rn(y[j], 0.25f);
+}
+
+// Unpack with the transform: sign masks on the raw bits, pairs as in
+// unpack_group, the transform, then max |y| over the transformed group.
+template <int DT>
+__device__ __forceinline__ float unpack_group_rht(const Raw<DT> &r, const SignMasks &sm,
+                                                  f2_t (&x)[8], bool &nonfinite)
+{
+    if constexpr (DT == DT_F32) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            x[j] = f2_pack(__uint_as_float(r.w[2 * j] ^ sm.w[2 * j]),
+                           __uint_as_float(r.w[2 * j + 1] ^ sm.w[2 * j + 1]));
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t w = r.w[j] ^ sm.w[j];
+            if constexpr (DT == DT_BF16)
+                x[j] = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+            else
+                x[j] = f2_pack(f16lo_to_f32(w), f16hi_to_f32(w));
+        }
+    }
+    hadamard16(x);
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float a, b;
+        f2_unpack(x[j], a, b);
+        m = max(m, max(__float_as_uint(a) & 0x7FFFFFFFu, __float_as_uint(b) & 0x7FFFFFFFu));
+    }
+    nonfinite = m >= 0x7F800000u;
+    return __uint_as_float(m);
+}
+
+// The 16 (transformed, when RHT) inputs of a group, re-read from memory.
+template <int DT, bool RHT>
+__device__ __forceinline__ void reload_group(const char *p, uint32_t signs, float (&y)[16])
+{
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        if constexpr (DT == DT_F32)
+            y[i] = __ldg(reinterpret_cast<const float *>(p) + i);
+        else if constexpr (DT == DT_BF16)
+            y[i] = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(p) + i) << 16);
+        else
+            y[i] = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short *>(p) + i)));
+    }
+    if constexpr (RHT) hadamard16_scalar(y, signs);
+}
+
 // ------------------------------------------------------- the quantizer ----
 
-// FP4 candidate of an element pair: the byte of two E2M1 nibbles (element
-// 2j low) and the two decoded values.
-__device__ __forceinline__ void fp4_pair(f2_t v, uint32_t &byte, f2_t &qf)
+// FP4 candidates of four element pairs (elements 0..7 of a word): one code
+// word (element 0 in bits 0-3) and, when ERR, the differences qf - v of all
+// eight elements as four pairs.  The E2M1 bytes stay in 8-bit registers, the
+// decoded values stay f16 (they are exact there) and each difference is one
+// mixed-precision subtract, i.e. one rounding of the exact qf - v.  Operands
+// are passed as 64-bit register pairs so no moves are needed around the
+// paired-float arithmetic.
+template <bool ERR>
+__device__ __forceinline__ uint32_t fp4_word(const f2_t (&v)[4], f2_t (&d)[4])
 {
-    float v0, v1;
-    f2_unpack(v, v0, v1);
-    byte = e2m1x2_from_f32(v0, v1);
-    const uint32_t h = f16x2_from_e2m1x2(byte);
-    qf = f2_pack(f16lo_to_f32(h), f16hi_to_f32(h));
+    uint32_t word;
+    if constexpr (ERR) {
+        asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 h0, h1, h2, h3;\n\t"
+            ".reg .b16 l0, l1, l2, l3, u0, u1, u2, u3;\n\t"
+            ".reg .f32 x<8>, e<8>;\n\t"
+            "mov.b64 {x0, x1}, %5;\n\t"
+            "mov.b64 {x2, x3}, %6;\n\t"
+            "mov.b64 {x4, x5}, %7;\n\t"
+            "mov.b64 {x6, x7}, %8;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 b0, x1, x0;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 b1, x3, x2;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 b2, x5, x4;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 b3, x7, x6;\n\t"
+            "mov.b32 %0, {b0, b1, b2, b3};\n\t"
+            "cvt.rn.f16x2.e2m1x2 h0, b0;\n\t"
+            "cvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
+            "cvt.rn.f16x2.e2m1x2 h2, b2;\n\t"
+            "cvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
+            "mov.b32 {l0, u0}, h0;\n\t"
+            "mov.b32 {l1, u1}, h1;\n\t"
+            "mov.b32 {l2, u2}, h2;\n\t"
+            "mov.b32 {l3, u3}, h3;\n\t"
+            "sub.rn.f32.f16 e0, l0, x0;\n\t"
+            "sub.rn.f32.f16 e1, u0, x1;\n\t"
+            "sub.rn.f32.f16 e2, l1, x2;\n\t"
+            "sub.rn.f32.f16 e3, u1, x3;\n\t"
+            "sub.rn.f32.f16 e4, l2, x4;\n\t"
+            "sub.rn.f32.f16 e5, u2, x5;\n\t"
+            "sub.rn.f32.f16 e6, l3, x6;\n\t"
+            "sub.rn.f32.f16 e7, u3, x7;\n\t"
+            "mov.b64 %1, {e0, e1};\n\t"
+            "mov.b64 %2, {e2, e3};\n\t"
+            "mov.b64 %3, {e4, e5};\n\t"
+            "mov.b64 %4, {e6, e7};\n\t}"
+            : "=r"(word), "=l"(d[0]), "=l"(d[1]), "=l"(d[2]), "=l"(d[3])
+            : "l"(v[0]), "l"(v[1]), "l"(v[2]), "l"(v[3]));
+    } else {
+        asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .f32 x<8>;\n\t"
+            "mov.b64 {x0, x1}, %1;\n\t"
+            "mov.b64 {x2, x3}, %2;\n\t"
+            "mov.b64 {x4, x5}, %3;\n\t"
+            "mov.b64 {x6, x7}, %4;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 b0, x1, x0;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 b1, x3, x2;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 b2, x5, x4;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 b3, x7, x6;\n\t"
+            "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+            : "=r"(word) : "l"(v[0]), "l"(v[1]), "l"(v[2]), "l"(v[3]));
+    }
+    return word;
 }
 
 // INT4 candidate of an element pair: r = 1.5*2^23 + RNE(v * fl(7/6)), one
 // fused multiply-add, so the integer is the exact product rounded once (bits
-// 0-3 of r are the nibble); qi = fl(k * fl(6/7)) = fl(6k/7) for |k| <= 7.
+// 0-3 of r are the nibble); d = v - k*fl(6/7) with one rounding (the rule's
+// value is fl(6k/7) = fl(k*fl(6/7)); the difference is at most 2^-22).
 template <bool CLAMP>
-__device__ __forceinline__ void int4_pair(f2_t v, f2_t &r, f2_t &qi)
+__device__ __forceinline__ void int4_pair(f2_t v, f2_t &r, f2_t &d)
 {
     const f2_t C76 = f2_pack(c76(), c76());
     const f2_t M = f2_pack(kMagic, kMagic);
@@ -142,8 +311,8 @@ __device__ __forceinline__ void int4_pair(f2_t v, f2_t &r, f2_t &qi)
         r1 = fminf(fmaxf(r1, kMagic - 7.0f), kMagic + 7.0f);
         r = f2_pack(r0, r1);
     }
-    const f2_t C67 = f2_pack(c67(), c67());
-    qi = f2_mul(f2_sub(r, M), C67);
+    const f2_t NC67 = f2_pack(-c67(), -c67());
+    d = f2_fma(f2_sub(r, M), NC67, v);
 }
 
 // Pack the low nibbles of 8 magic-biased floats (elements 0..7) into a word,
@@ -164,26 +333,38 @@ __device__ __forceinline__ uint32_t pack_int4_nibbles(const f2_t (&r)[4])
     return (E & 0x0F0F0F0Fu) | ((O << 4) & 0xF0F0F0F0u);
 }
 
+// True when every element's FP4 and INT4 candidates of one code word have
+// the same value.  The two grids share only 0 and +-6, so that means, per
+// nibble: the FP4 magnitude is 0 and k = 0, or the FP4 nibble is +6 (0x7) and
+// k = 7, or -6 (0xF) and k = -7 (0x9).  Then the two error sums add identical
+// terms in the same order, so they are equal in any precision and the rule
+// keeps FP4.  Evaluated on all eight nibbles at once.
+__device__ __forceinline__ bool candidates_coincide(uint32_t fp4, uint32_t int4)
+{
+    const uint32_t m = fp4 & 0x77777777u;                       // magnitudes
+    const uint32_t is6 = m & (m >> 1) & (m >> 2) & 0x11111111u;  // magnitude 7 (value 6)
+    const uint32_t nz = (m | (m >> 1) | (m >> 2)) & 0x11111111u; // magnitude != 0
+    const uint32_t sgn = (fp4 >> 3) & 0x11111111u;               // FP4 sign bits
+    // expected INT4 nibble: 0 for magnitude 0, 7 for +6, 9 for -6
+    const uint32_t want = (is6 * 0xFu) & (0x77777777u ^ (sgn * 0xEu));
+    return (nz & ~is6) == 0u && int4 == want;
+}
+
 // Binary64 squared-error sums of both candidates in element order: the
 // decision rule itself, used only when the binary32 margin of a group is too
 // small to trust.  It re-reads the group's 16 inputs (still in L2) and walks
 // them one by one, so the common path keeps no extra registers for it.  The
 // INT4 integer is always clamped here; the clamp is the identity whenever the
 // fast path skipped it.
-template <int DT>
-__device__ __noinline__ bool int4_wins_exact(const char *p, float inv)
+template <int DT, bool RHT>
+__device__ __noinline__ bool int4_wins_exact(const char *p, float inv, uint32_t signs)
 {
+    float xs[16];
+    reload_group<DT, RHT>(p, signs, xs);
     double ef = 0.0, ei = 0.0;
 #pragma unroll 1
     for (int i = 0; i < 16; ++i) {
-        float x;
-        if constexpr (DT == DT_F32)
-            x = __ldg(reinterpret_cast<const float *>(p) + i);
-        else if constexpr (DT == DT_BF16)
-            x = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(p) + i) << 16);
-        else
-            x = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short *>(p) + i)));
-        const float v = __fmul_rn(x, inv);
+        const float v = __fmul_rn(xs[i], inv);
         const uint32_t h = f16x2_from_e2m1x2(e2m1x2_from_f32(v, 0.0f));
         const float qf = f16lo_to_f32(h);
         float r = __fmaf_rn(v, c76(), kMagic);
@@ -197,72 +378,123 @@ __device__ __noinline__ bool int4_wins_exact(const char *p, float inv)
     return ei < ef;
 }
 
+// The IF4 choice for a group whose binary32 margin is within rounding: equal
+// candidates keep FP4, anything else is decided by the binary64 rule.
+template <int DT, bool RHT>
+__device__ __noinline__ bool int4_wins_rare(uint32_t f0, uint32_t f1, uint32_t i0, uint32_t i1,
+                                            const char *p, float inv, uint32_t signs)
+{
+    if (candidates_coincide(f0, i0) && candidates_coincide(f1, i1)) return false;
+    return int4_wins_exact<DT, RHT>(p, inv, signs);
+}
+
 struct GroupCode {
     uint32_t c0, c1;   // codes of elements 0..7 and 8..15
     uint32_t scale;    // scale byte
 };
 
-// Encode one group from its 16 inputs x (pairs), the block scale byte sb, the
-// reciprocal inv of the decoded scale and vmax = fl(amax * inv).
+// Encode one group from its 16 inputs x (pairs), the block scale byte sb and
+// the reciprocal inv of its decoded scale.
 //
-// Decision, fast path: each squared error is accumulated in binary32 from
-// d = fma(x, -inv, q), an explicit single rounding of q - x*inv (the square
-// does not see the sign).  Against the rule's d = v - q with v = fl(x*inv),
-// every d is off by at most half an ulp of v plus one rounding, and each sum
-// by at most 9 roundings; with Cauchy-Schwarz and vmax*sqrt(S) <= (vmax^2 +
-// S)/2 the difference of the two sums is off by less than 2^-20 S + 2^-21
-// vmax^2 + 2^-140.  Outside the band 2^-18 S + 2^-19 vmax^2 + 2^-126 the sign
-// of the binary32 difference is therefore the sign of the binary64 rule;
-// inside it the group is decided by the rule itself.
-template <int DT, bool IF4, bool CLAMP>
+// Decision, fast path: the two squared-error sums are accumulated in binary32
+// (two lanes of 8 terms each, then one add).  The FP4 differences qf - v are
+// exact (v and qf are within a factor of two of each other, or qf = 0); an
+// INT4 difference is off by at most 2^-22 (k*fl(6/7) is not rounded before
+// the subtraction) plus one rounding.  With Cauchy-Schwarz and sqrt(E) <=
+// (1 + E)/2, the binary32 difference of the sums is within (9u + 2^-20) S +
+// 2^-20 + 2^-40 of the binary64 rule (u = 2^-24, S = sum of both errors).
+// Outside the band 2^-18 (S + 1) its sign is the rule's; inside it the group
+// is decided by the rule itself.
+template <int DT, int MODE, bool CLAMP, bool RHT>
 __device__ __forceinline__ GroupCode encode_group(const f2_t (&x)[8], uint32_t sb, float inv,
-                                                float vmax, const char *p)
+                                                const char *p, uint32_t signs)
 {
     const f2_t INV = f2_pack(inv, inv);
-    const f2_t NINV = f2_pack(-inv, -inv);
-    uint32_t fp4[8];
-    f2_t r[8];
-    f2_t ef = f2_pack(0.0f, 0.0f), ei = f2_pack(0.0f, 0.0f);
+    f2_t v[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const f2_t v = f2_mul(x[j], INV);
-        f2_t qf;
-        fp4_pair(v, fp4[j], qf);
-        if constexpr (IF4) {
-            f2_t qi;
-            int4_pair<CLAMP>(v, r[j], qi);
-            const f2_t df = f2_fma(x[j], NINV, qf);
-            const f2_t di = f2_fma(x[j], NINV, qi);
-            ef = f2_fma(df, df, ef);
+    for (int j = 0; j < 8; ++j) v[j] = f2_mul(x[j], INV);
+    const f2_t lo[4] = {v[0], v[1], v[2], v[3]};
+    const f2_t hi[4] = {v[4], v[5], v[6], v[7]};
+    GroupCode out;
+    out.scale = sb;
+    if constexpr (MODE == Q_NVFP4) {
+        f2_t unused[4];
+        out.c0 = fp4_word<false>(lo, unused);
+        out.c1 = fp4_word<false>(hi, unused);
+        return out;
+    } else if constexpr (MODE == Q_NVINT4) {
+        f2_t r[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            f2_t unused;
+            int4_pair<CLAMP>(v[j], r[j], unused);
+        }
+        const f2_t rlo[4] = {r[0], r[1], r[2], r[3]};
+        const f2_t rhi[4] = {r[4], r[5], r[6], r[7]};
+        out.c0 = pack_int4_nibbles(rlo);
+        out.c1 = pack_int4_nibbles(rhi);
+        out.scale = sb | 0x80u;
+        return out;
+    } else {
+        f2_t df[8];
+        f2_t dlo[4], dhi[4];
+        out.c0 = fp4_word<true>(lo, dlo);
+        out.c1 = fp4_word<true>(hi, dhi);
+        f2_t ef = f2_pack(0.0f, 0.0f), ei = f2_pack(0.0f, 0.0f);
+        f2_t r[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { df[j] = dlo[j]; df[4 + j] = dhi[j]; }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            f2_t di;
+            int4_pair<CLAMP>(v[j], r[j], di);
+            ef = f2_fma(df[j], df[j], ef);
             ei = f2_fma(di, di, ei);
         }
-    }
-    GroupCode out;
-    out.c0 = fp4[0] | (fp4[1] << 8) | (fp4[2] << 16) | (fp4[3] << 24);
-    out.c1 = fp4[4] | (fp4[5] << 8) | (fp4[6] << 16) | (fp4[7] << 24);
-    out.scale = sb;
-    if constexpr (IF4) {
         float a0, a1, b0, b1;
         f2_unpack(ef, a0, a1);
         f2_unpack(ei, b0, b1);
         const float e_fp = __fadd_rn(a0, a1), e_int = __fadd_rn(b0, b1);
         const float d = __fsub_rn(e_fp, e_int);
-        const float band = __fmaf_rn(__fadd_rn(e_fp, e_int), 0x1p-18f,
-                                     __fmaf_rn(__fmul_rn(vmax, vmax), 0x1p-19f, 0x1p-126f));
-        bool int4;
-        if (fabsf(d) > band)
-            int4 = d > 0.0f;
-        else
-            int4 = int4_wins_exact<DT>(p, inv);
+        const float band = __fmul_rn(__fadd_rn(__fadd_rn(e_fp, e_int), 1.0f), 0x1p-18f);
+        const f2_t rlo[4] = {r[0], r[1], r[2], r[3]};
+        const f2_t rhi[4] = {r[4], r[5], r[6], r[7]};
+        const uint32_t i0 = pack_int4_nibbles(rlo), i1 = pack_int4_nibbles(rhi);
+        bool int4 = d > 0.0f;
+        if (!(fabsf(d) > band))      // rare: the binary32 margin is within rounding
+            int4 = int4_wins_rare<DT, RHT>(out.c0, out.c1, i0, i1, p, inv, signs);
         if (int4) {
-            const f2_t lo[4] = {r[0], r[1], r[2], r[3]};
-            const f2_t hi[4] = {r[4], r[5], r[6], r[7]};
-            out.c0 = pack_int4_nibbles(lo);
-            out.c1 = pack_int4_nibbles(hi);
+            out.c0 = i0;
+            out.c1 = i1;
             out.scale = sb | 0x80u;
         }
+        return out;
     }
-    return out;
+}
+
+// Block scale sb_f = fl(fl(amax / 6) / ts), each quotient by Markstein's
+// method: with y = RN(1/b), q = RN(a y), r = a - b q (exact by FMA), RN(q +
+// r y) is the correctly rounded a / b when no quotient over- or underflows.
+// Below amax = 2^-100 the IEEE division is used; a second quotient of 2^100 or
+// more is returned unrefined (any value that large saturates to 448, as the
+// exact one does); a second quotient below 2^-126 rounds to the E4M3 code 0
+// either way.
+__device__ __noinline__ float block_scale_ieee(float amax, float div, float ts)
+{
+    return __fdiv_rn(__fdiv_rn(amax, div), ts);
+}
+
+__device__ __forceinline__ float block_scale(float amax, float ts, float rts)
+{
+    const float r6 = __uint_as_float(0x3E2AAAABu);          // RN(1/6)
+    float q = __fmul_rn(amax, r6);
+    q = __fmaf_rn(__fmaf_rn(-q, 6.0f, amax), r6, q);
+    const float s = __fmul_rn(q, rts);
+    const float t = __fmaf_rn(__fmaf_rn(-s, ts, q), rts, s);
+    // rare: tiny amax (IEEE division), or a quotient beyond 2^100 (saturates)
+    if (!(amax >= 0x1p-100f && s < 0x1p100f))
+        return amax >= 0x1p-100f ? s : block_scale_ieee(amax, 6.0f, ts);
+    return t;
 }
 
 __device__ __forceinline__ bool ts_valid(float ts)
@@ -282,87 +514,303 @@ __device__ __forceinline__ const char *group_ptr(const char *x, uint32_t g, bool
     return x + (int64_t)row * ld_bytes + (int64_t)col * gbytes;
 }
 
-template <int DT, bool IF4, bool V8>
+// The encode with the INT4 clamp, for the rare groups whose scaled maximum
+// can round past 7 (a saturated or subnormal block scale).
+// It re-reads the group (still in L2) so that no registers of the common
+// path are passed to it.
+template <int DT, int MODE, bool RHT>
+__device__ __noinline__ GroupCode encode_group_clamped(uint32_t sb, float inv, const char *p,
+                                                       uint32_t signs)
+{
+    float y[16];
+    reload_group<DT, RHT>(p, signs, y);
+    f2_t x[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = f2_pack(y[2 * j], y[2 * j + 1]);
+    return encode_group<DT, MODE, true, RHT>(x, sb, inv, p, signs);
+}
+
+// fl(fl(amax / 4) / ts): amax / 4 is exact (a power of two) above 2^-124,
+// the quotient by ts is Markstein's, as in block_scale.
+__device__ __forceinline__ float block_scale4(float amax, float ts, float rts)
+{
+    const float q = __fmul_rn(amax, 0.25f);
+    const float s = __fmul_rn(q, rts);
+    const float t = __fmaf_rn(__fmaf_rn(-s, ts, q), rts, s);
+    if (!(amax >= 0x1p-100f && s < 0x1p100f))
+        return amax >= 0x1p-100f ? s : block_scale_ieee(amax, 4.0f, ts);
+    return t;
+}
+
+// FP4 code word of four element pairs and their decoded values as floats.
+__device__ __forceinline__ uint32_t fp4_word_values(const f2_t (&v)[4], f2_t (&q)[4])
+{
+    uint32_t word;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 h0, h1, h2, h3;\n\t"
+        ".reg .b16 l0, l1, l2, l3, u0, u1, u2, u3;\n\t"
+        ".reg .f32 x<8>, e<8>;\n\t"
+        "mov.b64 {x0, x1}, %5;\n\t"
+        "mov.b64 {x2, x3}, %6;\n\t"
+        "mov.b64 {x4, x5}, %7;\n\t"
+        "mov.b64 {x6, x7}, %8;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, x1, x0;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, x3, x2;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, x5, x4;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, x7, x6;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t"
+        "cvt.rn.f16x2.e2m1x2 h0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
+        "mov.b32 {l0, u0}, h0;\n\t"
+        "mov.b32 {l1, u1}, h1;\n\t"
+        "mov.b32 {l2, u2}, h2;\n\t"
+        "mov.b32 {l3, u3}, h3;\n\t"
+        "cvt.f32.f16 e0, l0;\n\t"
+        "cvt.f32.f16 e1, u0;\n\t"
+        "cvt.f32.f16 e2, l1;\n\t"
+        "cvt.f32.f16 e3, u1;\n\t"
+        "cvt.f32.f16 e4, l2;\n\t"
+        "cvt.f32.f16 e5, u2;\n\t"
+        "cvt.f32.f16 e6, l3;\n\t"
+        "cvt.f32.f16 e7, u3;\n\t"
+        "mov.b64 %1, {e0, e1};\n\t"
+        "mov.b64 %2, {e2, e3};\n\t"
+        "mov.b64 %3, {e4, e5};\n\t"
+        "mov.b64 %4, {e6, e7};\n\t}"
+        : "=r"(word), "=l"(q[0]), "=l"(q[1]), "=l"(q[2]), "=l"(q[3])
+        : "l"(v[0]), "l"(v[1]), "l"(v[2]), "l"(v[3]));
+    return word;
+}
+
+// Binary64 reconstruction errors of the two 4/6 candidates in element order
+// (the rule itself), for groups whose binary32 margin is within rounding.
+template <int DT>
+__device__ __noinline__ bool four_wins_exact(const char *p, float inv6, float eff6, float inv4,
+                                             float eff4)
+{
+    double e6 = 0.0, e4 = 0.0;
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i) {
+        float x;
+        if constexpr (DT == DT_F32)
+            x = __ldg(reinterpret_cast<const float *>(p) + i);
+        else if constexpr (DT == DT_BF16)
+            x = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(p) + i) << 16);
+        else
+            x = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short *>(p) + i)));
+        const float q6 = f16lo_to_f32(f16x2_from_e2m1x2(e2m1x2_from_f32(__fmul_rn(x, inv6), 0.0f)));
+        const float q4 = f16lo_to_f32(f16x2_from_e2m1x2(e2m1x2_from_f32(__fmul_rn(x, inv4), 0.0f)));
+        const double d6 = __dsub_rn((double)x, (double)__fmul_rn(q6, eff6));
+        const double d4 = __dsub_rn((double)x, (double)__fmul_rn(q4, eff4));
+        e6 = __dadd_rn(e6, __dmul_rn(d6, d6));
+        e4 = __dadd_rn(e4, __dmul_rn(d4, d4));
+    }
+    return e4 < e6;
+}
+
+// 4/6 encode of one group: FP4 under the block scale of amax/6 and under that
+// of amax/4, reconstruction errors sum (x - fl(q * eff))^2 compared, equal
+// errors keep /6.  Fast path: each difference is one explicit fma(q, -eff,
+// x), which differs from the rule's x - fl(q * eff) by at most 2^-24 * 6 eff,
+// and each sum by at most 9 roundings; the binary32 difference of the sums is
+// then within 2^-20 S + 2^-21 X^2 of the rule (X = 6 max(eff6, eff4)), so
+// outside the band 2^-18 S + 2^-19 X^2 + 2^-126 its sign is the rule's.
+template <int DT>
+__device__ __forceinline__ GroupCode encode_group_46(const f2_t (&x)[8], float amax, float ts,
+                                                   float rts, const float *inv_tab,
+                                                   const float *eff_tab, const char *p)
+{
+    const uint32_t sb6 = e4m3_from_f32(block_scale(amax, ts, rts)) & 0x7Fu;
+    const uint32_t sb4 = e4m3_from_f32(block_scale4(amax, ts, rts)) & 0x7Fu;
+    const float inv6 = inv_tab[sb6], eff6 = eff_tab[sb6];
+    const float inv4 = inv_tab[sb4], eff4 = eff_tab[sb4];
+    uint32_t w6[2], w4[2];
+    f2_t e6 = f2_pack(0.0f, 0.0f), e4 = f2_pack(0.0f, 0.0f);
+    const f2_t INV6 = f2_pack(inv6, inv6), INV4 = f2_pack(inv4, inv4);
+    const f2_t NEFF6 = f2_pack(-eff6, -eff6), NEFF4 = f2_pack(-eff4, -eff4);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        f2_t v6[4], v4[4], q6[4], q4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v6[j] = f2_mul(x[4 * h + j], INV6);
+            v4[j] = f2_mul(x[4 * h + j], INV4);
+        }
+        w6[h] = fp4_word_values(v6, q6);
+        w4[h] = fp4_word_values(v4, q4);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const f2_t d6 = f2_fma(q6[j], NEFF6, x[4 * h + j]);
+            const f2_t d4 = f2_fma(q4[j], NEFF4, x[4 * h + j]);
+            e6 = f2_fma(d6, d6, e6);
+            e4 = f2_fma(d4, d4, e4);
+        }
+    }
+    float a0, a1, b0, b1;
+    f2_unpack(e6, a0, a1);
+    f2_unpack(e4, b0, b1);
+    const float s6 = __fadd_rn(a0, a1), s4 = __fadd_rn(b0, b1);
+    const float d = __fsub_rn(s6, s4);
+    const float X = __fmul_rn(6.0f, fmaxf(eff6, eff4));
+    const float band = __fmaf_rn(__fadd_rn(s6, s4), 0x1p-18f,
+                                 __fmaf_rn(__fmul_rn(X, X), 0x1p-19f, 0x1p-126f));
+    bool four = d > 0.0f;
+    if (sb4 == sb6)
+        four = false;                 // identical candidates: a tie, keep /6
+    else if (!(fabsf(d) > band))
+        four = four_wins_exact<DT>(p, inv6, eff6, inv4, eff4);
+    GroupCode out;
+    const uint32_t sb = four ? sb4 : sb6;
+    out.c0 = four ? w4[0] : w6[0];
+    out.c1 = four ? w4[1] : w6[1];
+    out.scale = sb;
+    if (sb == 0) out.c0 = out.c1 = 0u;
+    return out;
+}
+
+// Encode group g from its raw bits r and store its codes and scale byte.
+// Returns true when an input element is Inf or NaN.
+template <int DT, int MODE, bool RHT>
+__device__ __forceinline__ bool quantize_one(const Raw<DT> &r, uint32_t g, const char *x,
+                                             int64_t ld_bytes, uint32_t gpr, int contig, float ts,
+                                             float rts, const float *inv_tab, const float *eff_tab,
+                                             uint8_t *codes, uint8_t *scales,
+                                             const SignMasks &sm, uint32_t signs)
+{
+    constexpr int GB = 16 * elem_bytes<DT>();
+    f2_t xv[8];
+    bool nonfinite;
+    float amax;
+    if constexpr (RHT)
+        amax = unpack_group_rht<DT>(r, sm, xv, nonfinite);
+    else
+        amax = unpack_group<DT>(r, xv, nonfinite);
+    if constexpr (MODE == Q_46) {
+        const GroupCode out = encode_group_46<DT>(xv, amax, ts, rts, inv_tab, eff_tab,
+                                                  group_ptr(x, g, contig, gpr, ld_bytes, GB));
+        st_v2(codes + (int64_t)g * 8, out.c0, out.c1);
+        st_u8(scales + g, out.scale);
+        return nonfinite;
+    }
+    // A3: block scale
+    const uint32_t sb = e4m3_from_f32(block_scale(amax, ts, rts)) & 0x7Fu;
+    // sb == 0: inv = 0 makes every candidate 0; the outputs are forced to
+    // all-zero FP4 below, without a branch around the arithmetic
+    const float inv = inv_tab[sb];
+    const char *gp = group_ptr(x, g, contig, gpr, ld_bytes, GB);
+    GroupCode out;
+    // The INT4 integer needs a clamp only if some |v| * fl(7/6) can reach
+    // 7.5; |v| is monotonic in |x|, so the group's max decides.
+    if (__fmul_rn(__fmul_rn(amax, inv), c76()) >= 7.5f)
+        out = encode_group_clamped<DT, MODE, RHT>(sb, inv, gp, signs);
+    else
+        out = encode_group<DT, MODE, false, RHT>(xv, sb, inv, gp, signs);
+    if (sb == 0) out.c0 = out.c1 = out.scale = 0u;
+    st_v2(codes + (int64_t)g * 8, out.c0, out.c1);
+    st_u8(scales + g, out.scale);
+    return nonfinite;
+}
+
+template <int DT, int MODE, bool V8, bool RHT>
 __global__ void __launch_bounds__(256)
 quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, uint32_t ngroups,
                 int contig, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
-                const float *__restrict__ ts_ptr, int *err, int check_ts)
+                const float *__restrict__ ts_ptr, int *err, int check_ts,
+                const __grid_constant__ SignMasks sm, uint32_t signs)
 {
     constexpr int GB = 16 * elem_bytes<DT>();
     const float ts = *ts_ptr;
     if (check_ts && blockIdx.x == 0 && threadIdx.x == 0 && !ts_valid(ts) && err)
         atomicOr(err, IF4_DEV_BAD_SCALE);
+    // inv_tab[c] = fl(1 / fl(E4M3(c) * ts)), the reciprocal of every block
+    // scale this tensor can use; inv_tab[0] = 0 (an underflowed block scale)
+    __shared__ float inv_tab[128];
+    __shared__ float eff_tab[MODE == Q_46 ? 128 : 1];
+    if (threadIdx.x < 128) {
+        const float eff = __fmul_rn(f32_from_e4m3(threadIdx.x), ts);
+        inv_tab[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __frcp_rn(eff);
+        if constexpr (MODE == Q_46) eff_tab[threadIdx.x] = eff;
+    }
+    const float rts = __frcp_rn(ts);
+    __syncthreads();
 
     const uint32_t stride = gridDim.x * blockDim.x;
     uint32_t g = blockIdx.x * blockDim.x + threadIdx.x;
-    if (g >= ngroups) return;
-    Raw<DT> cur;
-    load_group<DT, V8>(group_ptr(x, g, contig, gpr, ld_bytes, GB), cur);
     bool saw_nonfinite = false;
-    for (;;) {
-        const uint32_t gn = g + stride;
-        const bool more = gn < ngroups && gn > g;
-        Raw<DT> nxt;
-        if (more) load_group<DT, V8>(group_ptr(x, gn, contig, gpr, ld_bytes, GB), nxt);
-
-        f2_t xv[8];
-        bool nonfinite;
-        const float amax = unpack_group<DT>(cur, xv, nonfinite);
-        saw_nonfinite |= nonfinite;
-
-        // A3: block scale
-        const float sb_f = __fdiv_rn(__fdiv_rn(amax, 6.0f), ts);
-        const uint32_t sb = e4m3_from_f32(sb_f);
-        GroupCode out;
-        if (sb == 0) {
-            out.c0 = out.c1 = 0u;
-            out.scale = 0u;
-        } else {
-            const float eff = __fmul_rn(f32_from_e4m3(sb), ts);
-            const float inv = __frcp_rn(eff);
-            const float vmax = __fmul_rn(amax, inv);
-            const char *gp = group_ptr(x, g, contig, gpr, ld_bytes, GB);
-            // The INT4 integer needs a clamp only if some |v| * fl(7/6) can
-            // reach 7.5; |v| is monotonic in |x|, so the group's max decides.
-            if (__fmul_rn(vmax, c76()) >= 7.5f)
-                out = encode_group<DT, IF4, true>(xv, sb, inv, vmax, gp);
-            else
-                out = encode_group<DT, IF4, false>(xv, sb, inv, vmax, gp);
+    // Two register buffers, used in turn: the next group's load is in flight
+    // while the current one is encoded, with no copy between them.
+    Raw<DT> buf[2];
+    if (g < ngroups) load_group<DT, V8>(group_ptr(x, g, contig, gpr, ld_bytes, GB), buf[0]);
+    for (; g < ngroups;) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const uint32_t gn = g + stride;
+            const bool more = gn < ngroups && gn > g;
+            if (more) load_group<DT, V8>(group_ptr(x, gn, contig, gpr, ld_bytes, GB), buf[half ^ 1]);
+            saw_nonfinite |= quantize_one<DT, MODE, RHT>(buf[half], g, x, ld_bytes, gpr, contig,
+                                                          ts, rts, inv_tab, eff_tab, codes, scales,
+                                                          sm, signs);
+            g = more ? gn : ngroups;
+            if (!more) break;
         }
-        st_v2(codes + (int64_t)g * 8, out.c0, out.c1);
-        st_u8(scales + g, out.scale);
-
-        if (!more) break;
-        g = gn;
-        cur = nxt;
     }
     if (saw_nonfinite && err) atomicOr(err, IF4_DEV_NONFINITE);
 }
 
 // --------------------------------------------------------- A1 and A2 ----
 
-template <int DT, bool V8>
+// Float bits of max |x| over one group (NaN and Inf compare above every
+// finite value, so they survive the integer max below).
+template <int DT>
+__device__ __forceinline__ uint32_t group_absmax_bits(const Raw<DT> &r)
+{
+    if constexpr (DT == DT_F32) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = max(m, r.w[i] & 0x7FFFFFFFu);
+        return m;
+    } else {
+        uint32_t h = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            h = (DT == DT_BF16) ? absmax_bf16x2(h, r.w[i]) : absmax_f16x2(h, r.w[i]);
+        const uint32_t h16 = max(h & 0x7FFFu, (h >> 16) & 0x7FFFu);
+        return (DT == DT_BF16) ? (h16 << 16) : __float_as_uint(f16lo_to_f32(h16));
+    }
+}
+
+// A1: max |x| over the tensor, accumulated as float bits with atomicMax into
+// *amax_bits (zeroed by the caller's stream).  Each thread keeps four group
+// loads in flight.
+template <int DT, bool V8, bool RHT>
 __global__ void __launch_bounds__(256)
 amax_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, uint32_t ngroups,
-            int contig, unsigned int *amax_bits, int *err)
+            int contig, unsigned int *amax_bits, int *err, const __grid_constant__ SignMasks sm)
 {
     constexpr int GB = 16 * elem_bytes<DT>();
-    uint32_t m = 0;   // float bits of the running max |x|
+    constexpr int U = 4;
+    uint32_t m = 0;
     const uint32_t stride = gridDim.x * blockDim.x;
-    for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < ngroups; g += stride) {
-        Raw<DT> r;
-        load_group<DT, V8>(group_ptr(x, g, contig, gpr, ld_bytes, GB), r);
-        if constexpr (DT == DT_F32) {
+    for (uint64_t g0 = blockIdx.x * blockDim.x + threadIdx.x; g0 < ngroups;
+         g0 += (uint64_t)U * stride) {
+        Raw<DT> r[U];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) m = max(m, r.w[i] & 0x7FFFFFFFu);
-        } else {
-            uint32_t h = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) h = max_u16x2(h, r.w[i] & 0x7FFF7FFFu);
-            uint32_t h16 = max(h & 0xFFFFu, h >> 16);
-            uint32_t f = (DT == DT_BF16) ? (h16 << 16) : __float_as_uint(f16lo_to_f32(h16));
-            m = max(m, f);
+        for (int u = 0; u < U; ++u) {
+            const uint64_t g = g0 + (uint64_t)u * stride;
+            if (g < ngroups) load_group<DT, V8>(group_ptr(x, (uint32_t)g, contig, gpr, ld_bytes, GB), r[u]);
         }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (g0 + (uint64_t)u * stride < ngroups) {
+                if constexpr (RHT) {
+                    f2_t xv[8];
+                    bool nf;
+                    m = max(m, __float_as_uint(unpack_group_rht<DT>(r[u], sm, xv, nf)));
+                } else {
+                    m = max(m, group_absmax_bits<DT>(r[u]));
+                }
+            }
     }
     m = __reduce_max_sync(0xFFFFFFFFu, m);
     __shared__ uint32_t warp_max[8];
@@ -400,30 +848,90 @@ __device__ __forceinline__ uint32_t pack_out2(float a, float b)
     else return f16x2_from_f32(a, b);
 }
 
-// Decode 8 nibbles of one code word to 8 floats times eff.
-__device__ __forceinline__ void decode_word(uint32_t w, bool is_int, float eff, float (&y)[8])
+// Decoded value of every code: lut[n] is the FP4 value of nibble n,
+// lut[16 + n] the INT4 value fl(6k/7) of nibble n (k its sign extension).
+// 32 floats, one per shared-memory bank, so any pattern of lookups by a warp
+// is conflict-free.
+__device__ __forceinline__ float code_value(uint32_t i)
 {
-    if (is_int) {
-        // (nibble ^ 8) = k + 8 placed in the mantissa of 2^23 * 1.5: exact
-        const float bias = kMagic + 8.0f;
+    if (i < 16) {
+        const uint32_t h = f16x2_from_e2m1x2(i);      // nibble in bits 0-3
+        return f16lo_to_f32(h);
+    }
+    const float k = (float)((int)((i - 16) ^ 8u) - 8);
+    return __fmul_rn(k, c67());
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+// 8 decoded values (not yet scaled) of the 8 nibbles of w; base is the
+// shared address of lut or lut + 16 floats.
+__device__ __forceinline__ void decode_word(uint32_t w, uint32_t base, float (&q)[8])
+{
+    q[0] = lds_f32(base + ((w << 2) & 0x3Cu));
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t n = ((w >> (4 * i)) & 0xFu) ^ 0x8u;
-            const float k = __fsub_rn(__uint_as_float(kMagicBits | n), bias);
-            y[i] = __fmul_rn(__fmul_rn(k, c67()), eff);
+    for (int i = 1; i < 8; ++i) q[i] = lds_f32(base + ((w >> (4 * i - 2)) & 0x3Cu));
+}
+
+// Decode one group (code words w0, w1, scale byte sb) and store its 16
+// outputs at p.
+template <int ODT, bool UNIT_TS>
+__device__ __forceinline__ void dequant_group(uint32_t w0, uint32_t w1, uint32_t sb, float ts,
+                                              uint32_t lut_addr, char *p)
+{
+    const float e4 = f32_from_e4m3(sb);
+    const float eff = UNIT_TS ? e4 : __fmul_rn(e4, ts);
+    const uint32_t base = lut_addr + ((sb >> 1) & 0x40u);        // INT4 half for bit 7
+    float qa[8], qb[8];
+    decode_word(w0, base, qa);
+    decode_word(w1, base, qb);
+    const f2_t EFF = f2_pack(eff, eff);
+    f2_t ya[4], yb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        ya[j] = f2_mul(f2_pack(qa[2 * j], qa[2 * j + 1]), EFF);
+        yb[j] = f2_mul(f2_pack(qb[2 * j], qb[2 * j + 1]), EFF);
+    }
+    if constexpr (ODT == DT_F32) {
+        uint32_t a[8], b[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float lo, hi;
+            f2_unpack(ya[j], lo, hi);
+            a[2 * j] = __float_as_uint(lo);
+            a[2 * j + 1] = __float_as_uint(hi);
+            f2_unpack(yb[j], lo, hi);
+            b[2 * j] = __float_as_uint(lo);
+            b[2 * j + 1] = __float_as_uint(hi);
         }
+        st_v4(p, a[0], a[1], a[2], a[3]);
+        st_v4(p + 16, a[4], a[5], a[6], a[7]);
+        st_v4(p + 32, b[0], b[1], b[2], b[3]);
+        st_v4(p + 48, b[4], b[5], b[6], b[7]);
     } else {
+        uint32_t o[8];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const uint32_t h = f16x2_from_e2m1x2((w >> (8 * b)) & 0xFFu);
-            y[2 * b] = __fmul_rn(f16lo_to_f32(h), eff);
-            y[2 * b + 1] = __fmul_rn(f16hi_to_f32(h), eff);
+        for (int j = 0; j < 4; ++j) {
+            float lo, hi;
+            f2_unpack(ya[j], lo, hi);
+            o[j] = pack_out2<ODT>(lo, hi);
+            f2_unpack(yb[j], lo, hi);
+            o[4 + j] = pack_out2<ODT>(lo, hi);
         }
+        st_v4(p, o[0], o[1], o[2], o[3]);
+        st_v4(p + 16, o[4], o[5], o[6], o[7]);
     }
 }
 
 // ODT: output dtype.  UNIT_TS: leave the tensor scale out (the linear's
-// operand decode), else multiply by *ts.
+// operand decode), else multiply by *ts.  One thread per group (lanes of a
+// warp own consecutive groups, so loads and stores are contiguous spans); the
+// next group's codes and scale are loaded before the current one is decoded.
 template <int ODT, bool UNIT_TS>
 __global__ void __launch_bounds__(256)
 dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
@@ -431,33 +939,39 @@ dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__
                   char *__restrict__ y, int64_t ld_bytes, int contig)
 {
     constexpr int OB = ODT == DT_F32 ? 4 : 2;
+    __shared__ __align__(128) float lut[32];
+    if (threadIdx.x < 32) lut[threadIdx.x] = code_value(threadIdx.x);
     const float ts = UNIT_TS ? 1.0f : *ts_ptr;
+    const uint32_t lut_addr = (uint32_t)__cvta_generic_to_shared(lut);
+    __syncthreads();
     const uint32_t stride = gridDim.x * blockDim.x;
-    for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < ngroups; g += stride) {
-        uint32_t w0, w1;
-        ld_nc_v2(codes + (int64_t)g * 8, w0, w1);
-        const uint32_t sb = ld_nc_u8(scales + g);
-        const float e4 = f32_from_e4m3(sb);
-        const float eff = UNIT_TS ? e4 : __fmul_rn(e4, ts);
-        const bool is_int = (sb & 0x80u) != 0u;
-        float ya[8], yb[8];
-        decode_word(w0, is_int, eff, ya);
-        decode_word(w1, is_int, eff, yb);
-        char *p = const_cast<char *>(group_ptr(y, g, contig, gpr, ld_bytes, 16 * OB));
-        if constexpr (ODT == DT_F32) {
-            uint32_t a[8], b[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) { a[i] = __float_as_uint(ya[i]); b[i] = __float_as_uint(yb[i]); }
-            st_v4(p, a[0], a[1], a[2], a[3]);
-            st_v4(p + 16, a[4], a[5], a[6], a[7]);
-            st_v4(p + 32, b[0], b[1], b[2], b[3]);
-            st_v4(p + 48, b[4], b[5], b[6], b[7]);
-        } else {
-            st_v4(p, pack_out2<ODT>(ya[0], ya[1]), pack_out2<ODT>(ya[2], ya[3]),
-                  pack_out2<ODT>(ya[4], ya[5]), pack_out2<ODT>(ya[6], ya[7]));
-            st_v4(p + 16, pack_out2<ODT>(yb[0], yb[1]), pack_out2<ODT>(yb[2], yb[3]),
-                  pack_out2<ODT>(yb[4], yb[5]), pack_out2<ODT>(yb[6], yb[7]));
+    uint32_t g = blockIdx.x * blockDim.x + threadIdx.x;
+    uint32_t a0 = 0, a1 = 0, as = 0, b0 = 0, b1 = 0, bs = 0;
+    if (g < ngroups) {
+        ld_nc_v2(codes + (int64_t)g * 8, a0, a1);
+        as = ld_nc_u8(scales + g);
+    }
+    while (g < ngroups) {
+        uint32_t gn = g + stride;
+        bool more = gn < ngroups && gn > g;
+        if (more) {
+            ld_nc_v2(codes + (int64_t)gn * 8, b0, b1);
+            bs = ld_nc_u8(scales + gn);
         }
+        dequant_group<ODT, UNIT_TS>(a0, a1, as, ts, lut_addr,
+                                    const_cast<char *>(group_ptr(y, g, contig, gpr, ld_bytes, 16 * OB)));
+        if (!more) break;
+        g = gn;
+        gn = g + stride;
+        more = gn < ngroups && gn > g;
+        if (more) {
+            ld_nc_v2(codes + (int64_t)gn * 8, a0, a1);
+            as = ld_nc_u8(scales + gn);
+        }
+        dequant_group<ODT, UNIT_TS>(b0, b1, bs, ts, lut_addr,
+                                    const_cast<char *>(group_ptr(y, g, contig, gpr, ld_bytes, 16 * OB)));
+        if (!more) break;
+        g = gn;
     }
 }
 
@@ -544,74 +1058,121 @@ int launch_status()
     return cudaGetLastError() == cudaSuccess ? IF4_OK : IF4_ERR_CUDA;
 }
 
-template <typename K>
-uint32_t grid_for(K kernel, const DeviceInfo &d, uint32_t work_items, int threads)
+// Blocks to launch: enough for every work item, capped at one full wave of
+// resident blocks (the kernels are grid-stride loops).  `occ` is the number
+// of resident blocks per SM, queried once per kernel instantiation.
+uint32_t grid_for(int occ, const DeviceInfo &d, uint32_t work_items, int threads)
 {
-    static_assert(sizeof(K) > 0, "");
-    const int occ = resident_blocks(kernel, threads);
     const uint64_t want = ((uint64_t)work_items + threads - 1) / threads;
     const uint64_t cap = (uint64_t)d.sm_count * (uint64_t)occ;
     return (uint32_t)std::max<uint64_t>(1, std::min(want, cap));
 }
 
-template <int DT, bool V8>
+// Transform request of an entry point: off, or on with a 16-bit sign vector.
+struct Rht {
+    bool on = false;
+    uint32_t signs = 0;
+};
+
+SignMasks sign_masks(int dt, uint32_t signs)
+{
+    SignMasks m{};
+    for (int j = 0; j < 16; ++j) {
+        if (dt == IF4_F32) {
+            m.w[j] = ((signs >> j) & 1u) << 31;
+        } else if (j < 8) {
+            m.w[j] = (((signs >> (2 * j)) & 1u) << 15) | (((signs >> (2 * j + 1)) & 1u) << 31);
+        }
+    }
+    return m;
+}
+
+template <int DT, bool V8, bool RHT>
 int launch_amax(const Shape &s, const void *x, unsigned int *amax_bits, int *err,
-                cudaStream_t st, const DeviceInfo &d)
+                cudaStream_t st, const DeviceInfo &d, const SignMasks &sm)
 {
     if (s.ngroups == 0) return IF4_OK;
-    auto k = amax_kernel<DT, V8>;
-    const uint32_t grid = grid_for(k, d, s.ngroups, 256);
+    auto k = amax_kernel<DT, V8, RHT>;
+    static const int occ = resident_blocks(k, 256);
+    const uint32_t grid = grid_for(occ, d, s.ngroups, 256);
     k<<<grid, 256, 0, st>>>(static_cast<const char *>(x), s.ld_bytes, s.gpr, s.ngroups,
-                            s.contig ? 1 : 0, amax_bits, err);
+                            s.contig ? 1 : 0, amax_bits, err, sm);
     return launch_status();
+}
+
+template <int DT, bool RHT>
+int dispatch_amax_dt(const Shape &s, const void *x, unsigned int *amax_bits, int *err,
+                     cudaStream_t st, const DeviceInfo &d, const SignMasks &sm)
+{
+    return s.v8 ? launch_amax<DT, true, RHT>(s, x, amax_bits, err, st, d, sm)
+                : launch_amax<DT, false, RHT>(s, x, amax_bits, err, st, d, sm);
 }
 
 int dispatch_amax(int dt, const Shape &s, const void *x, unsigned int *amax_bits, int *err,
-                  cudaStream_t st, const DeviceInfo &d)
+                  cudaStream_t st, const DeviceInfo &d, Rht rht = Rht())
 {
+    const SignMasks sm = sign_masks(dt, rht.signs);
     switch (dt) {
-    case IF4_F32: return s.v8 ? launch_amax<DT_F32, true>(s, x, amax_bits, err, st, d)
-                              : launch_amax<DT_F32, false>(s, x, amax_bits, err, st, d);
-    case IF4_BF16: return s.v8 ? launch_amax<DT_BF16, true>(s, x, amax_bits, err, st, d)
-                               : launch_amax<DT_BF16, false>(s, x, amax_bits, err, st, d);
-    default: return s.v8 ? launch_amax<DT_F16, true>(s, x, amax_bits, err, st, d)
-                         : launch_amax<DT_F16, false>(s, x, amax_bits, err, st, d);
+    case IF4_F32:
+        return rht.on ? dispatch_amax_dt<DT_F32, true>(s, x, amax_bits, err, st, d, sm)
+                      : dispatch_amax_dt<DT_F32, false>(s, x, amax_bits, err, st, d, sm);
+    case IF4_BF16:
+        return rht.on ? dispatch_amax_dt<DT_BF16, true>(s, x, amax_bits, err, st, d, sm)
+                      : dispatch_amax_dt<DT_BF16, false>(s, x, amax_bits, err, st, d, sm);
+    default:
+        return rht.on ? dispatch_amax_dt<DT_F16, true>(s, x, amax_bits, err, st, d, sm)
+                      : dispatch_amax_dt<DT_F16, false>(s, x, amax_bits, err, st, d, sm);
     }
 }
 
-template <int DT, bool IF4, bool V8>
+template <int DT, int MODE, bool V8, bool RHT>
 int launch_quant(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
-                 const float *ts, int *err, int check_ts, cudaStream_t st, const DeviceInfo &d)
+                 const float *ts, int *err, int check_ts, cudaStream_t st, const DeviceInfo &d,
+                 const SignMasks &sm, uint32_t signs)
 {
     if (s.ngroups == 0) return IF4_OK;
-    auto k = quantize_kernel<DT, IF4, V8>;
-    const uint32_t grid = grid_for(k, d, s.ngroups, 256);
+    auto k = quantize_kernel<DT, MODE, V8, RHT>;
+    static const int occ = resident_blocks(k, 256);
+    const uint32_t grid = grid_for(occ, d, s.ngroups, 256);
     k<<<grid, 256, 0, st>>>(static_cast<const char *>(x), s.ld_bytes, s.gpr, s.ngroups,
-                            s.contig ? 1 : 0, codes, scales, ts, err, check_ts);
+                            s.contig ? 1 : 0, codes, scales, ts, err, check_ts, sm, signs);
     return launch_status();
 }
 
-template <bool IF4>
-int dispatch_quant(int dt, const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
-                   const float *ts, int *err, int check_ts, cudaStream_t st, const DeviceInfo &d)
+template <int DT, int MODE, bool RHT>
+int dispatch_quant_dt(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
+                      const float *ts, int *err, int check_ts, cudaStream_t st,
+                      const DeviceInfo &d, const SignMasks &sm, uint32_t signs)
 {
+    return s.v8 ? launch_quant<DT, MODE, true, RHT>(s, x, codes, scales, ts, err, check_ts, st, d,
+                                                    sm, signs)
+                : launch_quant<DT, MODE, false, RHT>(s, x, codes, scales, ts, err, check_ts, st,
+                                                     d, sm, signs);
+}
+
+template <int MODE, bool RHT>
+int dispatch_quant(int dt, const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
+                   const float *ts, int *err, int check_ts, cudaStream_t st, const DeviceInfo &d,
+                   uint32_t signs)
+{
+    const SignMasks sm = sign_masks(dt, signs);
     switch (dt) {
     case IF4_F32:
-        return s.v8 ? launch_quant<DT_F32, IF4, true>(s, x, codes, scales, ts, err, check_ts, st, d)
-                    : launch_quant<DT_F32, IF4, false>(s, x, codes, scales, ts, err, check_ts, st, d);
+        return dispatch_quant_dt<DT_F32, MODE, RHT>(s, x, codes, scales, ts, err, check_ts, st, d,
+                                                    sm, signs);
     case IF4_BF16:
-        return s.v8 ? launch_quant<DT_BF16, IF4, true>(s, x, codes, scales, ts, err, check_ts, st, d)
-                    : launch_quant<DT_BF16, IF4, false>(s, x, codes, scales, ts, err, check_ts, st, d);
+        return dispatch_quant_dt<DT_BF16, MODE, RHT>(s, x, codes, scales, ts, err, check_ts, st,
+                                                     d, sm, signs);
     default:
-        return s.v8 ? launch_quant<DT_F16, IF4, true>(s, x, codes, scales, ts, err, check_ts, st, d)
-                    : launch_quant<DT_F16, IF4, false>(s, x, codes, scales, ts, err, check_ts, st, d);
+        return dispatch_quant_dt<DT_F16, MODE, RHT>(s, x, codes, scales, ts, err, check_ts, st, d,
+                                                    sm, signs);
     }
 }
 
-template <bool IF4>
+template <int MODE, bool RHT = false>
 int quantize_entry(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
                    uint8_t *codes, uint8_t *scales, float *ts, int ts_mode, int *err_flag,
-                   void *stream)
+                   void *stream, uint32_t signs = 0)
 {
     Shape s;
     int rc = check_tensor(x, x_dtype, rows, cols, ld_x, s);
@@ -628,14 +1189,18 @@ int quantize_entry(const void *x, int x_dtype, int64_t rows, int64_t cols, int64
     if (ts_mode == IF4_TS_COMPUTE) {
         // A1 accumulates max |x| as float bits into *ts, A2 turns it into ts
         if (cudaMemsetAsync(ts, 0, sizeof(float), st) != cudaSuccess) return IF4_ERR_CUDA;
-        rc = dispatch_amax(x_dtype, s, x, reinterpret_cast<unsigned int *>(ts), err_flag, st, d);
+        Rht rht;
+        rht.on = RHT;
+        rht.signs = signs;
+        rc = dispatch_amax(x_dtype, s, x, reinterpret_cast<unsigned int *>(ts), err_flag, st, d,
+                           rht);
         if (rc != IF4_OK) return rc;
         tensor_scale_kernel<<<1, 1, 0, st>>>(ts, ts);
         rc = launch_status();
         if (rc != IF4_OK) return rc;
     }
-    return dispatch_quant<IF4>(x_dtype, s, x, codes, scales, ts, err_flag,
-                               ts_mode == IF4_TS_GIVEN ? 1 : 0, st, d);
+    return dispatch_quant<MODE, RHT>(x_dtype, s, x, codes, scales, ts, err_flag,
+                                     ts_mode == IF4_TS_GIVEN ? 1 : 0, st, d, signs);
 }
 
 template <int ODT, bool UNIT_TS>
@@ -644,7 +1209,8 @@ int launch_dequant(const Shape &s, const uint8_t *codes, const uint8_t *scales, 
 {
     if (s.ngroups == 0) return IF4_OK;
     auto k = dequantize_kernel<ODT, UNIT_TS>;
-    const uint32_t grid = grid_for(k, d, s.ngroups, 256);
+    static const int occ = resident_blocks(k, 256);
+    const uint32_t grid = grid_for(occ, d, s.ngroups, 256);
     k<<<grid, 256, 0, st>>>(codes, scales, ts, s.gpr, s.ngroups, static_cast<char *>(y),
                             s.ld_bytes, s.contig ? 1 : 0);
     return launch_status();
@@ -688,16 +1254,60 @@ int if4_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t
                  uint8_t *codes, uint8_t *scales, float *ts, int ts_mode, int *err_flag,
                  void *stream)
 {
-    return quantize_entry<true>(x, x_dtype, rows, cols, ld_x, codes, scales, ts, ts_mode,
-                                err_flag, stream);
+    return quantize_entry<Q_IF4>(x, x_dtype, rows, cols, ld_x, codes, scales, ts, ts_mode,
+                                 err_flag, stream);
 }
 
 int nvfp4_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
                    uint8_t *codes, uint8_t *scales, float *ts, int ts_mode, int *err_flag,
                    void *stream)
 {
-    return quantize_entry<false>(x, x_dtype, rows, cols, ld_x, codes, scales, ts, ts_mode,
-                                 err_flag, stream);
+    return quantize_entry<Q_NVFP4>(x, x_dtype, rows, cols, ld_x, codes, scales, ts, ts_mode,
+                                   err_flag, stream);
+}
+
+int nvint4_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                    uint8_t *codes, uint8_t *scales, float *ts, int ts_mode, int *err_flag,
+                    void *stream)
+{
+    return quantize_entry<Q_NVINT4>(x, x_dtype, rows, cols, ld_x, codes, scales, ts, ts_mode,
+                                    err_flag, stream);
+}
+
+int nvfp4_4over6_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                          uint8_t *codes, uint8_t *scales, float *ts, int ts_mode, int *err_flag,
+                          void *stream)
+{
+    return quantize_entry<Q_46>(x, x_dtype, rows, cols, ld_x, codes, scales, ts, ts_mode,
+                                err_flag, stream);
+}
+
+int if4_tensor_amax_rht(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                        uint32_t signs, float *amax, int *err_flag, void *stream)
+{
+    Shape s;
+    int rc = check_tensor(x, x_dtype, rows, cols, ld_x, s);
+    if (rc != IF4_OK) return rc;
+    if (amax == nullptr) return IF4_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(amax) % 4 != 0) return IF4_ERR_ALIGN;
+    DeviceInfo d;
+    rc = check_device(d);
+    if (rc != IF4_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(amax, 0, sizeof(float), st) != cudaSuccess) return IF4_ERR_CUDA;
+    Rht rht;
+    rht.on = true;
+    rht.signs = signs & 0xFFFFu;
+    return dispatch_amax(x_dtype, s, x, reinterpret_cast<unsigned int *>(amax), err_flag, st, d,
+                         rht);
+}
+
+int if4_quantize_rht(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                     uint32_t signs, uint8_t *codes, uint8_t *scales, float *ts, int ts_mode,
+                     int *err_flag, void *stream)
+{
+    return quantize_entry<Q_IF4, true>(x, x_dtype, rows, cols, ld_x, codes, scales, ts, ts_mode,
+                                       err_flag, stream, signs & 0xFFFFu);
 }
 
 int if4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts, int64_t rows,

@@ -127,6 +127,48 @@ int nvfp4_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64
                    int *err_flag, void *stream);
 
 /*
+ * Random-sign Hadamard transform fused into the quantizer, for weight
+ * gradients (gist.science section 1, second item: a Hadamard transform makes
+ * the data near-uniform, where INT4 does better; companion "Where the Gain
+ * Actually Comes From").  Every group of 16 is replaced by y = H16 diag(s)
+ * x_g / 4 before quantization: H16 the Sylvester Hadamard matrix, s_j = -1
+ * where bit j of `signs` is set (bits 16-31 ignored).  The transform is
+ * evaluated in binary32 as a fast Walsh-Hadamard transform with stages h = 1,
+ * 2, 4, 8 (each (y[i], y[i+h]) -> (y[i] + y[i+h], y[i] - y[i+h]) for i with
+ * bit h clear), then times 1/4.  The transformed tensor never reaches memory;
+ * the codes are those of if4_quantize applied to it, and if4_dequantize gives
+ * back the transformed values.
+ */
+int if4_tensor_amax_rht(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                        uint32_t signs, float *amax, int *err_flag, void *stream);
+int if4_quantize_rht(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                     uint32_t signs, uint8_t *codes, uint8_t *scales, float *ts, int ts_mode,
+                     int *err_flag, void *stream);
+
+/*
+ * Comparator, all-INT4 ("NVINT4"): the 7/6-scaled INT4 candidate of
+ * if4_quantize for every group, bit 7 set wherever the block scale is
+ * nonzero (gist.science section 3, item 2, and section 4: IF4 is compared with
+ * NVFP4 and NVINT4).  Same arguments and rules as if4_quantize; decoded by
+ * if4_dequantize.
+ */
+int nvint4_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                    uint8_t *codes, uint8_t *scales, float *ts, int ts_mode,
+                    int *err_flag, void *stream);
+
+/*
+ * Comparator, Four Over Six ("4/6"): NVFP4 whose block scale maps the group
+ * maximum either to 6 (sb from amax/6, as NVFP4) or to 4 (sb from amax/4),
+ * whichever reconstructs the group with the lower squared error
+ * sum (x - fl(q * fl(E4M3 * ts)))^2 (binary64 rule, equal errors keep 6);
+ * gist.science section 1, third item.  Output is plain NVFP4 (bit 7 clear),
+ * decoded by if4_dequantize.  Same arguments and rules as if4_quantize.
+ */
+int nvfp4_4over6_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                          uint8_t *codes, uint8_t *scales, float *ts, int ts_mode,
+                          int *err_flag, void *stream);
+
+/*
  * A7: dequantize IF4 (or NVFP4) to y[rows, cols] of y_dtype (IF4_F32,
  * IF4_BF16 or IF4_F16), row stride ld_y elements: fl(q * fl(E4M3 * ts)),
  * then RNE to the output type.  codes 16-byte aligned; y 16-byte aligned and

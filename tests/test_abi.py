@@ -57,7 +57,7 @@ def test_library_exports_every_declared_symbol(lib):
         assert n in exported, n
         assert hasattr(lib, n)
     # nothing but the C ABI leaks out (the static CUDA runtime stays local)
-    assert all(n.startswith(("if4_", "nvfp4_")) for n in exported), sorted(exported)[:10]
+    assert all(n.startswith(("if4_", "nvfp4_", "nvint4_")) for n in exported), sorted(exported)[:10]
 
 
 def test_status_strings(lib):

@@ -326,3 +326,126 @@ def test_fp4_code_of_every_bf16_value():
     x = _probe_groups(base, probes)
     ref = check_quant(x, "fp4 code of every bf16 value", ts=1.0)
     assert not (ref["scales"] & 0x80).any()
+
+
+# ------------------------------------------------------ comparator formats --
+
+_MODES = {"nvint4": oracle.MODE_NVINT4, "4over6": oracle.MODE_4OVER6}
+
+
+def check_mode(x_cpu, mode, label, ts=None):
+    x_np = x_cpu.float().numpy()
+    if ts is None:
+        ref = oracle.quantize_tensor(x_np, mode=_MODES[mode])
+        ts_ref = ref["ts"]
+    else:
+        ts_ref = np.float32(ts)
+        ref = oracle.quantize(x_np, ts_ref, mode=_MODES[mode])
+    codes, scales, ts_g, err = gpu_quant(x_cpu, mode, ts=ts)
+    assert err == 0
+    assert f32_bits(ts_g) == f32_bits(ts_ref)
+    bad_s = np.count_nonzero(scales != ref["scales"])
+    bad_c = np.count_nonzero(codes != ref["codes"])
+    assert bad_s == 0 and bad_c == 0, f"{label} {mode}: {bad_s} scale / {bad_c} code bytes differ"
+    y = B().dequantize(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(),
+                       torch.tensor([ts_ref], device="cuda"), dtype=torch.float32).cpu().numpy()
+    mse = oracle.mse(x_np, y)
+    print(f"[{label} {mode}] mse={mse:.6g} near_ties={int(ref['near'].sum())}")
+    return ref
+
+
+@pytest.mark.parametrize("mode", ["nvint4", "4over6"])
+def test_comparators_on_workloads(mode):
+    check_mode(workloads.small_fp32(0), mode, "small_fp32_256x1024")
+    check_mode(workloads.llm_weight(0), mode, "weight_bf16_4096x4096")
+    check_mode(workloads.activation_outliers(0), mode, "activation_bf16_8192x8192")
+    check_mode(workloads.hadamard_gradient(0), mode, "gradient_bf16_16384x4096")
+
+
+@pytest.mark.parametrize("mode", ["nvint4", "4over6"])
+def test_comparators_edge_cases(mode):
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((64, 256)).astype(np.float32)
+    x *= np.exp2(-rng.integers(0, 24, (64, 16))).repeat(16, axis=1).astype(np.float32)
+    x[0, 0] = 1000.0
+    x[1, :16] = -0.0
+    check_mode(torch.from_numpy(x), mode, "tiny groups")
+    check_mode(torch.zeros((3, 48)), mode, "zeros")
+    w = torch.from_numpy(rng.standard_normal((128, 512)).astype(np.float32)).to(torch.bfloat16)
+    amax = float(w.abs().max())
+    check_mode(w, mode, "saturating ts", ts=np.float32(amax / 2688.0 * 0.05))
+    for shape in [(1, 16), (3, 48), (33, 272)]:
+        for dt in (torch.float32, torch.bfloat16, torch.float16):
+            check_mode((torch.randn(shape) * 2).to(dt), mode, f"ragged {shape} {dt}")
+    bits = (np.arange(0x0001, 0x7F80, dtype=np.uint32) << 16).view(np.float32)
+    frac = rng.uniform(-1, 1, (bits.size, 15)).astype(np.float32)
+    sweep = np.concatenate([bits[:, None], bits[:, None] * frac], axis=1)
+    check_mode(torch.from_numpy(sweep).to(torch.bfloat16), mode, "block scale sweep", ts=1.0)
+
+
+def test_mse_ordering_on_workloads():
+    """Per-group IF4 error never exceeds NVFP4's or NVINT4's, and 4/6 never
+    exceeds NVFP4's (the formats' own guarantees, here on GPU outputs)."""
+    x = workloads.llm_weight(5, rows=512, cols=4096)
+    xd = x.float().numpy().astype(np.float64)
+    errs = {}
+    for mode in ("if4", "nvfp4", "nvint4", "4over6"):
+        c, s, ts = B().quantize(x.cuda(), mode)
+        y = B().dequantize(c, s, ts, dtype=torch.float32).cpu().numpy().astype(np.float64)
+        errs[mode] = ((xd - y) ** 2).reshape(x.shape[0], -1, 16).sum(-1)
+    slack = 1 + 1e-6
+    assert np.all(errs["if4"] <= errs["nvfp4"] * slack + 1e-30)
+    assert np.all(errs["4over6"] <= errs["nvfp4"] * slack + 1e-30)
+    tot = {k: float(v.sum()) for k, v in errs.items()}
+    print("[mse ordering] " + " ".join(f"{k}={v:.4g}" for k, v in tot.items()))
+    assert tot["if4"] < tot["nvfp4"] and tot["if4"] < tot["nvint4"]
+
+
+# -------------------------------------- random-sign Hadamard + quantize --
+
+def check_rht(x_cpu, signs, label, ts=None):
+    b = B()
+    x_np = x_cpu.float().numpy()
+    y = oracle.rht(x_np, signs)
+    if ts is None:
+        ref = oracle.quantize_tensor(y)
+        ts_ref = ref["ts"]
+    else:
+        ts_ref = np.float32(ts)
+        ref = oracle.quantize(y, ts_ref)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ts_t = None if ts is None else torch.tensor([ts], dtype=torch.float32, device="cuda")
+    codes, scales, ts_g = b.quantize_rht(x_cpu.cuda(), signs, ts=ts_t, err_flag=err)
+    amax = torch.empty(1, dtype=torch.float32, device="cuda")
+    b.if4_tensor_amax_rht(x_cpu.cuda(), signs, amax)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert amax.item() == oracle.tensor_amax(y)
+    assert f32_bits(np.float32(ts_g.item())) == f32_bits(ts_ref)
+    c, s = codes.cpu().numpy(), scales.cpu().numpy()
+    assert np.count_nonzero(s != ref["scales"]) == 0 and np.count_nonzero(c != ref["codes"]) == 0, label
+    nv = oracle.quantize(y, ts_ref, mode=oracle.MODE_NVFP4)
+    yd = y.astype(np.float64)
+    e_if4 = oracle.mse(yd, oracle.dequantize(c, s, ts_ref))
+    e_nv = oracle.mse(yd, oracle.dequantize(nv["codes"], nv["scales"], ts_ref))
+    print(f"[rht {label}] int4_frac={oracle.group_int4_fraction(s):.4f} "
+          f"mse if4={e_if4:.4g} nvfp4={e_nv:.4g} near_ties={int(ref['near'].sum())}")
+
+
+@pytest.mark.parametrize("signs", [0x0000, 0xFFFF, 0x6A3C])
+def test_rht_quantize_on_gradient_like_data(signs):
+    rng = np.random.default_rng(31)
+    x = (rng.standard_normal((2048, 1024)) * 1e-3).astype(np.float32)
+    check_rht(torch.from_numpy(x).to(torch.bfloat16), signs, f"normal {signs:#06x}")
+    t = (rng.standard_t(3, (1024, 1024)) * 1e-3).astype(np.float32)
+    check_rht(torch.from_numpy(t).to(torch.bfloat16), signs, f"student-t {signs:#06x}")
+
+
+def test_rht_quantize_dtypes_shapes_and_given_scale():
+    rng = np.random.default_rng(32)
+    for shape in [(1, 16), (7, 80), (33, 272)]:
+        for dt in (torch.float32, torch.bfloat16, torch.float16):
+            check_rht((torch.randn(shape) * 3).to(dt), 0x1357, f"{shape} {dt}")
+    w = torch.from_numpy(rng.standard_normal((256, 512)).astype(np.float32))
+    check_rht(w, 0xBEEF, "given ts", ts=np.float32(float(w.abs().max()) / 2688.0 * 0.1))
+    check_rht(torch.zeros((4, 64)), 0xFFFF, "zeros")
