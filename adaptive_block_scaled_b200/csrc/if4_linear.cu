@@ -12,7 +12,8 @@
 // to 11 bits for INT4 groups, and the per-tensor scales (one float each)
 // factor out of the whole sum.
 //
-// GEMM structure (one CTA per SM, persistent over 128 x 256 output tiles):
+// GEMM structure (one CTA per SM, persistent over 128 x 256 output tiles;
+// large problems use the CTA-pair kernel further down, 256 x 256 tiles):
 //   warp 0      TMA producer: 128B-swizzled 64-wide K slabs of A and B into a
 //               4-stage shared-memory ring (no multicast)
 //   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 accumulators)
@@ -93,15 +94,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// Same, with cluster-scope acquire: for barriers that threads of the peer CTA
+// arrive on with release.cluster.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase of `parity` to complete.  Returns false (and
 // raises the CTA's abort flag) when the wall-clock limit runs out or another
 // role already aborted.
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag)
 {
-    if (mbar_try_wait(bar, parity)) return true;
+    auto try_once = [&] {
+        return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+    };
+    if (try_once()) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (try_once()) return true;
         if ((i & 255u) == 0u) {
             if (*abort_flag) return false;
             if (globaltimer() - t0 > WAIT_LIMIT_NS) {
@@ -366,6 +383,257 @@ gemm_f16_tcgen05(const __grid_constant__ CUtensorMap tmap_a,
     }
 }
 
+// ------------------------------------------------ two-SM (CTA pair) GEMM ----
+//
+// A cluster of two CTAs on two SMs computes one 256 x 256 output tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256): CTA r loads rows r*128..+127
+// of the tile's A slab and of its B slab into its own shared memory, and the
+// even CTA (the leader) issues MMAs that read both CTAs' halves, so each SM
+// receives 32 KB per 64-wide K step instead of 48 KB.  The leader's full
+// barrier counts both CTAs' copies (cp.async.bulk.tensor.cta_group::2 lets a
+// copy complete on the peer's barrier); its tcgen05.commit is multicast to the
+// same barrier in both CTAs, which frees a stage in both rings and announces
+// a finished accumulator to both epilogues; each epilogue thread then arrives
+// on the leader's accumulator-free barrier.  No load uses multicast.
+
+namespace pair {
+
+constexpr int PBM = 128;                 // rows per CTA (256 per pair)
+constexpr int PBN = 256;                 // output columns per pair
+constexpr int PBNH = PBN / 2;             // B rows loaded per CTA
+constexpr int PSTAGES = 6;
+constexpr int PA_BYTES = PBM * BK * 2;    // 16 KB
+constexpr int PB_BYTES = PBNH * BK * 2;   // 16 KB
+constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;
+constexpr int PSMEM_BYTES = PSTAGES * PSTAGE_BYTES + 1024 + 256;
+constexpr uint32_t PIDESC = (1u << 4) | ((uint32_t)(PBN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cta_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// shared::cluster address of the same variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    __syncwarp();
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+                 ::: "memory");
+}
+
+__device__ __forceinline__ void arrive_remote(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+                 :: "r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                                 uint32_t bar_cluster)
+{
+    asm volatile("cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3}], [%4];"
+                 :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+                 : "memory");
+}
+
+__device__ __forceinline__ void umma_f16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(PIDESC), "r"(accumulate));
+}
+
+// arrive on barrier `bar` (same offset) in both CTAs when the MMAs complete
+__device__ __forceinline__ void umma_commit_both(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+                 " [%0], %1;" :: "r"(bar), "h"((uint16_t)0x3) : "memory");
+}
+
+}  // namespace pair
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_f16_tcgen05_2sm(const __grid_constant__ CUtensorMap tmap_a,
+                     const __grid_constant__ CUtensorMap tmap_b,
+                     const float *__restrict__ a_ts, const float *__restrict__ b_ts,
+                     __nv_bfloat16 *__restrict__ c, int M, int N, int K, int *err)
+{
+    using namespace pair;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem_a = smem;
+    uint8_t *smem_b = smem + PSTAGES * PA_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + PSTAGES * PSTAGE_BYTES);
+    uint64_t *full = bars;                    // [PSTAGES], used in the leader
+    uint64_t *empty = bars + PSTAGES;          // [PSTAGES], both CTAs
+    uint64_t *acc_full = bars + 2 * PSTAGES;   // [2], both CTAs
+    uint64_t *acc_empty = acc_full + 2;       // [2], used in the leader
+    uint64_t *drain = acc_empty + 2;          // [1], leader
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cta_rank();
+    const bool leader = rank == 0;
+    const int m_tiles = (M + 2 * PBM - 1) / (2 * PBM);
+    const int n_tiles = (N + PBN - 1) / PBN;
+    const int tiles = m_tiles * n_tiles;
+    const int pair_id = blockIdx.x >> 1;
+    const int num_pairs = gridDim.x >> 1;
+    const int k_blocks = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < PSTAGES; ++st) {
+            mbar_init(smem_u32(&full[st]), 1);
+            mbar_init(smem_u32(&empty[st]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&acc_full[b]), 1);
+            mbar_init(smem_u32(&acc_empty[b]), 2 * 4 * 32);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        prefetch_tmap(&tmap_a);
+        prefetch_tmap(&tmap_b);
+    }
+    if (warp == 1) {
+        __syncwarp();
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(tmem_slot)), "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                      // peer barriers initialised before any remote use
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0 && lane == 0) {
+        // ---------------------------------------------------- TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int t = pair_id; t < tiles && ok; t += num_pairs) {
+            const int m0 = (t % m_tiles) * 2 * PBM + (int)rank * PBM;
+            const int n0 = (t / m_tiles) * PBN + (int)rank * PBNH;
+            for (int kb = 0; kb < k_blocks; ++kb) {
+                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) { ok = false; break; }
+                const uint32_t fb = map_to(smem_u32(&full[stage]), 0);
+                if (leader) mbar_expect_tx(smem_u32(&full[stage]), 2 * PSTAGE_BYTES);
+                tma_load_2d_pair(smem_u32(smem_a + stage * PA_BYTES), &tmap_a, kb * BK, m0, fb);
+                tma_load_2d_pair(smem_u32(smem_b + stage * PB_BYTES), &tmap_b, kb * BK, n0, fb);
+                if (++stage == PSTAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+        // every copy issued here has been consumed by the leader's MMAs when
+        // the loops end normally; after an abort, give them a bounded time
+        const unsigned long long t0 = globaltimer();
+        if (*abort_flag)
+            while (globaltimer() - t0 < 2000000ull) { }
+    } else if (warp == 1 && lane == 0 && leader) {
+        // ------------------------------------------- MMA issuer (leader)
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int t = pair_id; t < tiles && ok; t += num_pairs) {
+            // both CTAs' epilogue threads arrive here, the peer's remotely
+            if (!mbar_wait<true>(smem_u32(&acc_empty[acc]), acc_phase ^ 1u, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * PBN);
+            for (int kb = 0; kb < k_blocks; ++kb) {
+                if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(smem_a + stage * PA_BYTES);
+                const uint32_t b0 = smem_u32(smem_b + stage * PB_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < BK / UMMA_K; ++kk)
+                    umma_f16_pair(d_tmem, smem_desc_sw128(a0 + kk * UMMA_K * 2),
+                                  smem_desc_sw128(b0 + kk * UMMA_K * 2), (kb | kk) != 0 ? 1u : 0u);
+                umma_commit_both(smem_u32(&empty[stage]));
+                if (++stage == PSTAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            umma_commit_both(smem_u32(&acc_full[acc]));
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                     :: "r"(smem_u32(drain)) : "memory");
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(smem_u32(drain), 0))
+            if (globaltimer() - t0 > WAIT_LIMIT_NS) break;
+    } else if (warp >= EPI_WARP0) {
+        // -------------------------------------------------------- epilogue
+        const int quarter = warp & 3;
+        const int row_in_cta = quarter * 32 + lane;
+        const float scale = __fmul_rn(*a_ts, *b_ts);
+        const uint32_t acc_empty_leader0 = map_to(smem_u32(&acc_empty[0]), 0);
+        const uint32_t acc_empty_leader1 = map_to(smem_u32(&acc_empty[1]), 0);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = pair_id; t < tiles; t += num_pairs) {
+            const int m0 = (t % m_tiles) * 2 * PBM + (int)rank * PBM;
+            const int n0 = (t / m_tiles) * PBN;
+            const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&acc_full[acc]), acc_phase,
+                                                              abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const int row = m0 + row_in_cta;
+            __nv_bfloat16 *crow = c + (int64_t)row * N;
+#pragma unroll 1
+            for (int chunk = 0; chunk < PBN / 32; ++chunk) {
+                uint32_t r[32];
+                tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                              (uint32_t)(acc * PBN + chunk * 32), r);
+                const int col0 = n0 + chunk * 32;
+                if (row < M) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int col = col0 + q * 8;
+                        if (col < N) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                pk[e] = bf16x2(__fmul_rn(__uint_as_float(r[q * 8 + 2 * e]), scale),
+                                               __fmul_rn(__uint_as_float(r[q * 8 + 2 * e + 1]), scale));
+                            st_v4(crow + col, pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            arrive_remote(acc ? acc_empty_leader1 : acc_empty_leader0);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                      // the peer's MMAs and copies are done
+    if (threadIdx.x == 0 && *abort_flag && err) atomicOr(err, IF4_DEV_TIMEOUT);
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;"
+                     :: "r"(tmem_base), "r"(TMEM_COLS));
+    }
+}
+
 // ------------------------------------------------------------ host side ----
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -433,7 +701,56 @@ int launch_gemm(const void *a, const void *b, const float *a_ts, const float *b_
     int sms = 0;
     int rc = sm_count_checked(sms);
     if (rc != IF4_OK) return rc;
+    // A CTA pair per 256 x 256 tile when both dimensions fill a pair tile,
+    // otherwise one CTA per 128 x 256 tile.
+    const bool use_pair = M >= 256 && N >= 256 && sms >= 2;
     CUtensorMap ma, mb;
+    if (use_pair) {
+        if (!make_map(&ma, a, M, K, pair::PBM) || !make_map(&mb, b, N, K, pair::PBNH))
+            return IF4_ERR_CUDA;
+        static std::once_flag attr2_once;
+        static cudaError_t attr2_rc = cudaSuccess;
+        std::call_once(attr2_once, [] {
+            attr2_rc = cudaFuncSetAttribute(gemm_f16_tcgen05_2sm,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            pair::PSMEM_BYTES);
+        });
+        if (attr2_rc != cudaSuccess) return IF4_ERR_CUDA;
+        const int64_t tiles = ((M + 2 * pair::PBM - 1) / (2 * pair::PBM)) *
+                              ((N + pair::PBN - 1) / pair::PBN);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(2 * (sms / 2)), 1, 1);
+        cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = pair::PSMEM_BYTES;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        // persistent: as many pairs as can be resident at once (SM pairs
+        // must share a GPC, so this can be below sms / 2)
+        static std::once_flag clusters_once;
+        static int resident_pairs = 0;
+        std::call_once(clusters_once, [&cfg] {
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, gemm_f16_tcgen05_2sm, &cfg) == cudaSuccess)
+                resident_pairs = n;
+            else
+                (void)cudaGetLastError();
+        });
+        int64_t pairs = resident_pairs > 0 ? resident_pairs : sms / 2;
+        if (pairs > sms / 2) pairs = sms / 2;
+        if (tiles < pairs) pairs = tiles;
+        cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+        if (cudaLaunchKernelEx(&cfg, gemm_f16_tcgen05_2sm, ma, mb, a_ts, b_ts,
+                               static_cast<__nv_bfloat16 *>(c), (int)M, (int)N, (int)K, err) !=
+            cudaSuccess)
+            return IF4_ERR_CUDA;
+        return cudaGetLastError() == cudaSuccess ? IF4_OK : IF4_ERR_CUDA;
+    }
     if (!make_map(&ma, a, M, K, BM) || !make_map(&mb, b, N, K, BN)) return IF4_ERR_CUDA;
     static std::once_flag attr_once;
     static cudaError_t attr_rc = cudaSuccess;

@@ -693,7 +693,7 @@ __device__ __forceinline__ bool quantize_one(const Raw<DT> &r, uint32_t g, const
         st_u8(scales + g, out.scale);
         return nonfinite;
     }
-    // A3: block scale
+    // block scale
     const uint32_t sb = e4m3_from_f32(block_scale(amax, ts, rts)) & 0x7Fu;
     // sb == 0: inv = 0 makes every candidate 0; the outputs are forced to
     // all-zero FP4 below, without a branch around the arithmetic
@@ -758,7 +758,7 @@ quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, uint
     if (saw_nonfinite && err) atomicOr(err, IF4_DEV_NONFINITE);
 }
 
-// --------------------------------------------------------- A1 and A2 ----
+// ------------------------------------------ tensor amax and tensor scale --
 
 // Float bits of max |x| over one group (NaN and Inf compare above every
 // finite value, so they survive the integer max below).
@@ -780,7 +780,7 @@ __device__ __forceinline__ uint32_t group_absmax_bits(const Raw<DT> &r)
     }
 }
 
-// A1: max |x| over the tensor, accumulated as float bits with atomicMax into
+// Tensor amax: max |x| over the tensor, accumulated as float bits with atomicMax into
 // *amax_bits (zeroed by the caller's stream).  Each thread keeps four group
 // loads in flight.
 template <int DT, bool V8, bool RHT>
@@ -839,7 +839,7 @@ __global__ void tensor_scale_kernel(const float *amax, float *ts)
     *ts = t;
 }
 
-// ------------------------------------------------------------ A7 / K4 ----
+// ------------------------------------------------ dequantize, fp16 decode --
 
 template <int ODT>
 __device__ __forceinline__ uint32_t pack_out2(float a, float b)
@@ -1187,7 +1187,8 @@ int quantize_entry(const void *x, int x_dtype, int64_t rows, int64_t cols, int64
     if (rc != IF4_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (ts_mode == IF4_TS_COMPUTE) {
-        // A1 accumulates max |x| as float bits into *ts, A2 turns it into ts
+        // the amax kernel accumulates max |x| as float bits into *ts, the
+        // scale kernel turns it into ts
         if (cudaMemsetAsync(ts, 0, sizeof(float), st) != cudaSuccess) return IF4_ERR_CUDA;
         Rht rht;
         rht.on = RHT;

@@ -3,8 +3,9 @@
 
 One step = one pass of the whole quantization path over one tensor that is
 already resident in HBM:
-    tensor amax (A1) -> tensor scale (A2) -> IF4 quantize (A3-A6)
-    -> IF4 dequantize to bf16 (A7) -> NVFP4 quantize with the same scale (A9)
+    tensor amax -> tensor scale -> IF4 quantize (block scale, FP4 and INT4
+    candidates, choice) -> IF4 dequantize to bf16 -> NVFP4 quantize with the
+    same tensor scale
 Default workload: the LLM weight matrix, bf16 4096 x 4096, Student-t(3)
 scaled to std 0.02, groups of 16 along K.  The IF4 x IF4 linear has its own
 workload and is reported under "linear" when its entry point is built.
@@ -34,6 +35,7 @@ METRIC = "IF4 quantize Gelem/s & HBM GB/s vs ~8 TB/s peak (1 B200); MSE vs NVFP4
 UNIT = "Gelem/s"
 WORKLOAD = "weight_bf16_4096x4096"
 L2_BYTES = 126e6
+RHT_SIGNS = 0x6A3C          # one fixed random-sign vector for the transform
 
 
 def parse():
@@ -46,8 +48,12 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-linear", action="store_true")
+    p.add_argument("--no-large", action="store_true",
+                   help="skip the per-kernel table of the two large workloads")
     p.add_argument("--kernel-only", default=None,
-                   choices=["amax", "if4_quantize", "if4_dequantize", "nvfp4_quantize", "gemm"],
+                   choices=["amax", "if4_quantize", "if4_dequantize", "nvfp4_quantize", "gemm",
+                            "nvint4_quantize", "nvfp4_4over6_quantize", "if4_quantize_rht",
+                            "if4_decode_f16"],
                    help="launch only this kernel, warmup+steps times (for ncu captures)")
     return p.parse_args()
 
@@ -278,7 +284,40 @@ class Step:
         s = self.sets[0]
         return sum(t.numel() * t.element_size() for t in s.values())
 
-    def run(self, i, events=None):
+    EXTRA = ["nvint4_quantize", "nvfp4_4over6_quantize", "if4_quantize_rht", "if4_decode_f16"]
+
+    def run_one(self, name, i):
+        b, s = self.b, self.sets[i % len(self.sets)]
+        if name == "nvint4_quantize":
+            b.nvint4_quantize(s["x"], s["ncodes"], s["nscales"], s["ts"], b.TS_GIVEN, self.err)
+            return
+        if name == "nvfp4_4over6_quantize":
+            b.nvfp4_4over6_quantize(s["x"], s["ncodes"], s["nscales"], s["ts"], b.TS_GIVEN, self.err)
+            return
+        if name == "if4_quantize_rht":
+            b.if4_quantize_rht(s["x"], RHT_SIGNS, s["ncodes"], s["nscales"], s["ts"], b.TS_GIVEN,
+                               self.err)
+            return
+        if name == "if4_decode_f16":
+            b.if4_decode_f16(s["codes"], s["scales"], s["y"].view(torch.float16))
+            return
+        if name == "amax":
+            b.if4_tensor_amax(s["x"], s["amax"], self.err)
+        elif name == "scale":
+            b.if4_tensor_scale(s["amax"], s["ts"])
+        elif name == "if4_quantize":
+            b.if4_quantize(s["x"], s["codes"], s["scales"], s["ts"], b.TS_GIVEN, self.err)
+        elif name == "if4_dequantize":
+            b.if4_dequantize(s["codes"], s["scales"], s["ts"], s["y"])
+        elif name == "nvfp4_quantize":
+            b.nvfp4_quantize(s["x"], s["ncodes"], s["nscales"], s["ts"], b.TS_GIVEN, self.err)
+        else:
+            raise ValueError(name)
+
+    def run(self, i, events=None, side=None):
+        """One step on buffer set i.  With a side stream, the NVFP4 quantizer
+        (which needs only ts) runs on it beside IF4 quantize -> dequantize:
+        the two quantizers read the same input at about the same time."""
         b, s = self.b, self.sets[i % len(self.sets)]
         ev = events if events is not None else [None] * 6
         if ev[0] is not None:
@@ -287,6 +326,10 @@ class Step:
         if ev[1] is not None:
             ev[1].record()
         b.if4_tensor_scale(s["amax"], s["ts"])
+        if side is not None:
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                b.nvfp4_quantize(s["x"], s["ncodes"], s["nscales"], s["ts"], b.TS_GIVEN, self.err)
         if ev[2] is not None:
             ev[2].record()
         b.if4_quantize(s["x"], s["codes"], s["scales"], s["ts"], b.TS_GIVEN, self.err)
@@ -295,15 +338,99 @@ class Step:
         b.if4_dequantize(s["codes"], s["scales"], s["ts"], s["y"])
         if ev[4] is not None:
             ev[4].record()
-        b.nvfp4_quantize(s["x"], s["ncodes"], s["nscales"], s["ts"], b.TS_GIVEN, self.err)
+        if side is None:
+            b.nvfp4_quantize(s["x"], s["ncodes"], s["nscales"], s["ts"], b.TS_GIVEN, self.err)
+        else:
+            torch.cuda.current_stream().wait_stream(side)
         if ev[5] is not None:
             ev[5].record()
 
 
+def kernel_times(step, names, reps):
+    """Per-kernel times: one CUDA graph per kernel launching it once on every
+    buffer set in turn, replayed `reps` times between two events on the
+    replay stream; mean time per launch (ms)."""
+    out = {}
+    sets = len(step.sets)
+    for name in names:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(sets):
+                step.run_one(name, i)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        out[name] = e0.elapsed_time(e1) / (reps * sets)
+        del g
+    return out
+
+
+def kernel_table(ms, n_elem, in_bytes, pk):
+    q_bytes = in_bytes + n_elem // 2 + n_elem // 16
+    dq_bytes = n_elem // 2 + n_elem // 16 + 2 * n_elem
+    nbytes = {"amax": in_bytes, "scale": 8, "if4_quantize": q_bytes, "if4_dequantize": dq_bytes,
+              "nvfp4_quantize": q_bytes, "nvint4_quantize": q_bytes,
+              "nvfp4_4over6_quantize": q_bytes, "if4_quantize_rht": q_bytes,
+              "if4_decode_f16": dq_bytes}
+    table = {}
+    for k, t in ms.items():
+        b = nbytes[k]
+        gbs = b / (t * 1e-3) / 1e9
+        table[k] = {"ms": t, "bytes": b, "gbs": gbs, "frac_of_measured_hbm": gbs / pk["hbm_gbs"],
+                    "frac_of_8tbs": gbs / 8000.0, "gelems": n_elem / (t * 1e-3) / 1e9}
+    return table
+
+
+def large_workloads(pk, names=("activation_bf16_8192x8192", "gradient_bf16_16384x4096")):
+    """Per-kernel times on the large workloads (more than L2 per launch)."""
+    out = {}
+    for wname in names:
+        x_cpu = make_input(wname)
+        n_elem, in_bytes = x_cpu.numel(), x_cpu.numel() * x_cpu.element_size()
+        step = Step(x_cpu, sets=3)
+        for i in range(3):
+            step.run(i)
+        torch.cuda.synchronize()
+        ms = kernel_times(step, step.kernels + Step.EXTRA, 10)
+        out[wname] = kernel_table(ms, n_elem, in_bytes, pk)
+        out[wname]["quality"] = quality_report(x_cpu, step)
+        del step
+        torch.cuda.empty_cache()
+    return out
+
+
+def quality_report(x_cpu, step):
+    """MSE against the input (x domain, float64 on the host) of IF4 and of
+    the comparators on the same tensor and tensor scale, from GPU outputs
+    (quantized and dequantized by the library, outside the timed region);
+    the IF4 INT4-group fraction."""
+    from adaptive_block_scaled_b200 import binding as b
+    s = step.sets[0]
+    x = x_cpu.float().numpy().astype(np.float64)
+    out = {}
+    for mode in ("if4", "nvfp4", "nvint4", "4over6"):
+        c, sc, _ = b.quantize(s["x"], mode, ts=s["ts"].clone())
+        y = b.dequantize(c, sc, s["ts"], dtype=torch.float32).cpu().numpy().astype(np.float64)
+        out["mse_" + mode] = float(np.mean((x - y) ** 2))
+        if mode == "if4":
+            out["int4_group_fraction"] = float(np.mean(sc.cpu().numpy() >> 7))
+    nv = out["mse_nvfp4"]
+    out["mse_reduction_vs_nvfp4_pct"] = 100.0 * (1.0 - out["mse_if4"] / nv) if nv > 0 else 0.0
+    return out
+
+
 def measure_e2e(x_cpu, steps, warmup):
-    """Same step through the C ABI from pinned host memory: H2D of the input,
-    the five kernels, D2H of every result (IF4 codes, scales, scale, bf16
-    dequantized tensor, NVFP4 codes and scales), inside the timed region."""
+    """The same step through the C ABI from pinned host memory: per step, the
+    H2D copy of the input, the five kernels, and the D2H copy of every result
+    (IF4 codes, scales and tensor scale, the bf16 dequantized tensor, NVFP4
+    codes and scales), all inside the timed region.  Consecutive steps
+    alternate between two streams with their own buffers, so one step's
+    upload overlaps the previous step's download (PCIe is full duplex)."""
     from adaptive_block_scaled_b200 import binding as b
     rows, cols = x_cpu.shape
     dev = torch.device("cuda")
@@ -311,53 +438,49 @@ def measure_e2e(x_cpu, steps, warmup):
     outs = dict(codes=((rows, cols // 2), torch.uint8), scales=((rows, cols // 16), torch.uint8),
                 ts=((1,), torch.float32), y=((rows, cols), torch.bfloat16),
                 ncodes=((rows, cols // 2), torch.uint8), nscales=((rows, cols // 16), torch.uint8))
-    d = {k: torch.empty(sh, dtype=dt, device=dev) for k, (sh, dt) in outs.items()}
-    h = {k: torch.empty(sh, dtype=dt, pin_memory=True) for k, (sh, dt) in outs.items()}
-    d_x = torch.empty_like(h_x, device=dev)
-    amax = torch.empty(1, dtype=torch.float32, device=dev)
+    lanes = []
+    for _ in range(2):
+        lanes.append(dict(
+            stream=torch.cuda.Stream(),
+            x=torch.empty_like(h_x, device=dev),
+            amax=torch.empty(1, dtype=torch.float32, device=dev),
+            d={k: torch.empty(sh, dtype=dt, device=dev) for k, (sh, dt) in outs.items()},
+            h={k: torch.empty(sh, dtype=dt, pin_memory=True) for k, (sh, dt) in outs.items()}))
     err = torch.zeros(1, dtype=torch.int32, device=dev)
 
-    def step():
-        d_x.copy_(h_x, non_blocking=True)
-        b.if4_tensor_amax(d_x, amax, err)
-        b.if4_tensor_scale(amax, d["ts"])
-        b.if4_quantize(d_x, d["codes"], d["scales"], d["ts"], b.TS_GIVEN, err)
-        b.if4_dequantize(d["codes"], d["scales"], d["ts"], d["y"])
-        b.nvfp4_quantize(d_x, d["ncodes"], d["nscales"], d["ts"], b.TS_GIVEN, err)
-        for k in h:
-            h[k].copy_(d[k], non_blocking=True)
+    def step(i):
+        L = lanes[i % 2]
+        with torch.cuda.stream(L["stream"]):
+            d = L["d"]
+            L["x"].copy_(h_x, non_blocking=True)
+            b.if4_tensor_amax(L["x"], L["amax"], err)
+            b.if4_tensor_scale(L["amax"], d["ts"])
+            b.if4_quantize(L["x"], d["codes"], d["scales"], d["ts"], b.TS_GIVEN, err)
+            b.if4_dequantize(d["codes"], d["scales"], d["ts"], d["y"])
+            b.nvfp4_quantize(L["x"], d["ncodes"], d["nscales"], d["ts"], b.TS_GIVEN, err)
+            for k in L["h"]:
+                L["h"][k].copy_(d[k], non_blocking=True)
 
-    for _ in range(warmup):
-        step()
+    cur = torch.cuda.current_stream()
+    for i in range(warmup):
+        step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        step()
-    e1.record()
+    e0.record(cur)
+    for L in lanes:
+        L["stream"].wait_stream(cur)
+    for i in range(steps):
+        step(i)
+    for L in lanes:
+        cur.wait_stream(L["stream"])
+    e1.record(cur)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     h2d = h_x.numel() * h_x.element_size()
-    d2h = sum(t.numel() * t.element_size() for t in h.values())
+    d2h = sum(t.numel() * t.element_size() for t in lanes[0]["h"].values())
     return {"value": rows * cols / (ms * 1e-3) / 1e9, "unit": UNIT, "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-
-
-def quality_report(x_cpu, step):
-    """MSE of IF4 and NVFP4 against the input (x domain, float64 on the host)
-    from the GPU outputs of set 0, and the INT4 group fraction."""
-    from adaptive_block_scaled_b200 import binding as b
-    s = step.sets[0]
-    y_if4 = s["y"].float().cpu().numpy().astype(np.float64)
-    y_nv = b.dequantize(s["ncodes"], s["nscales"], s["ts"], dtype=torch.float32).cpu().numpy()
-    x = x_cpu.float().numpy().astype(np.float64)
-    mse_if4 = float(np.mean((x - y_if4) ** 2))
-    mse_nv = float(np.mean((x - y_nv.astype(np.float64)) ** 2))
-    sc = s["scales"].cpu().numpy()
-    return {"mse_if4": mse_if4, "mse_nvfp4": mse_nv,
-            "mse_reduction_pct": 100.0 * (1.0 - mse_if4 / mse_nv) if mse_nv > 0 else 0.0,
-            "int4_group_fraction": float(np.mean(sc >> 7)),
-            "note": "IF4 MSE measured on the bf16 dequantized output; NVFP4 on fp32 dequant"}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "how": "C ABI calls from Python, two streams alternating steps"}
 
 
 def linear_report(pk, steps=20, warmup=3):
@@ -429,7 +552,9 @@ def run_ours(args):
 
     step = Step(x_cpu, sets=1)
     per_set = step.bytes_per_set()
-    sets = max(2, int(np.ceil(2 * L2_BYTES / per_set)) + 1)
+    # enough rotating sets that even the lightest kernel (amax: 2 B/element)
+    # cycles through more than three times the 126 MB L2 before reusing one
+    sets = max(4, int(np.ceil(3 * L2_BYTES / in_bytes)) + 1)
     step = Step(x_cpu, sets=sets)
 
     for i in range(args.warmup):
@@ -438,41 +563,46 @@ def run_ours(args):
     if int(step.err.item()) != 0:
         raise RuntimeError(f"device error flag {int(step.err.item())} during warm-up")
 
-    n_ev = 6
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    # One CUDA graph per buffer set holds a whole step (5 kernels and the
+    # memset that zeroes amax), so host launch overhead does not pace the GPU;
+    # the NVFP4 comparator is a parallel branch of the graph.
+    graphs = []
+    side = torch.cuda.Stream()
+    for i in range(sets):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step.run(i, side=side)
+        graphs.append(g)
+    for i in range(max(args.warmup, sets)):
+        graphs[i % sets].replay()
+    torch.cuda.synchronize()
+
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         start.record()
         for i in range(args.steps):
-            step.run(args.warmup + i, events[i])
+            graphs[i % sets].replay()
         stop.record()
         torch.cuda.synchronize()
     barrier(world)
     ms_local = start.elapsed_time(stop) / args.steps
     ms = max_over_ranks(ms_local, world)
-    kern_ms = {}
-    for k, name in enumerate(step.kernels):
-        kern_ms[name] = sum(events[i][k].elapsed_time(events[i][k + 1]) for i in range(args.steps)) / args.steps
+
+    kern_ms = kernel_times(step, step.kernels, max(2, args.steps // sets))
+    if int(step.err.item()) != 0:
+        raise RuntimeError(f"device error flag {int(step.err.item())}")
+    graphs_keep = graphs
 
     value = world * n_elem / (ms * 1e-3) / 1e9
     q_bytes = in_bytes + n_elem // 2 + n_elem // 16
-    kernels = {
-        "amax": {"ms": kern_ms["amax"], "bytes": in_bytes},
-        "scale": {"ms": kern_ms["scale"], "bytes": 8},
-        "if4_quantize": {"ms": kern_ms["if4_quantize"], "bytes": q_bytes},
-        "if4_dequantize": {"ms": kern_ms["if4_dequantize"], "bytes": n_elem // 2 + n_elem // 16 + 2 * n_elem},
-        "nvfp4_quantize": {"ms": kern_ms["nvfp4_quantize"], "bytes": q_bytes},
-    }
-    for k, v in kernels.items():
-        v["gbs"] = v["bytes"] / (v["ms"] * 1e-3) / 1e9
-        v["frac_of_measured_hbm"] = v["gbs"] / pk["hbm_gbs"]
-        v["frac_of_8tbs"] = v["gbs"] / 8000.0
-    kernels["if4_quantize"]["gelems"] = n_elem / (kern_ms["if4_quantize"] * 1e-3) / 1e9
+    kernels = kernel_table(kern_ms, n_elem, in_bytes, pk)
+    extra = kernel_table(kernel_times(step, Step.EXTRA, max(2, args.steps // sets)), n_elem,
+                         in_bytes, pk)
 
     top = kernels["if4_quantize"]
-    roofline = {"bound": "hbm", "kernel": "if4_quantize (A3-A6, ts given)",
+    roofline = {"bound": "hbm", "kernel": "if4_quantize (tensor scale given)",
                 "achieved": top["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": top["gbs"] / pk["hbm_gbs"],
                 "peak_source": f"{pk['source']} hbm_gbs (copy bandwidth, read+write)",
@@ -491,10 +621,14 @@ def run_ours(args):
             "config": {"workload": args.workload, "rows": int(x_cpu.shape[0]),
                        "cols": int(x_cpu.shape[1]), "input_dtype": str(x_cpu.dtype).replace("torch.", ""),
                        "group": 16, "parallelism": f"independent tensors x{world}",
-                       "l2": f"rotating {sets} buffer sets, {sets * per_set / 1e6:.0f} MB > 2x126 MB L2",
+                       "l2": f"rotating {sets} buffer sets, {sets * per_set / 1e6:.0f} MB "
+                             f"(inputs {sets * in_bytes / 1e6:.0f} MB > 3x126 MB L2)",
+                       "launch": "one CUDA graph per step (NVFP4 on a parallel branch after "
+                                 "the tensor scale); per-kernel times from one graph per "
+                                 "kernel over all sets",
                        "step": "amax, scale, IF4 quantize, IF4 dequantize (bf16), NVFP4 quantize"},
             "gpu_launches": step.launches_per_step * args.steps,
-            "kernels": kernels, "roofline": roofline}
+            "kernels": kernels, "kernels_outside_step": extra, "roofline": roofline}
     if rank == 0:
         line["clocks"] = clk.summary()
         line["quality"] = quality_report(x_cpu, step)
@@ -503,6 +637,10 @@ def run_ours(args):
             line["cpu_baseline"] = cpu_baseline(x_cpu, args.cpu_seconds)
         if not args.no_linear and hasattr(step.b.lib, "if4_linear"):
             line["linear"] = linear_report(pk)
+        if not args.no_large:
+            del step, graphs_keep
+            torch.cuda.empty_cache()
+            line["large_workloads"] = large_workloads(pk)
         print(json.dumps(line), flush=True)
     barrier(world)
     if world > 1:
@@ -526,6 +664,8 @@ def run_kernel_only(args):
         torch.cuda.synchronize()
         print(json.dumps({"kernel_only": "gemm", "launches": args.warmup + args.steps,
                           "err": int(err.item())}))
+        if int(err.item()) != 0:
+            sys.exit(1)
         return
     x_cpu = make_input(args.workload)
     step = Step(x_cpu, sets=1)
@@ -534,19 +674,22 @@ def run_kernel_only(args):
     b.if4_tensor_scale(s["amax"], s["ts"])
     b.if4_quantize(s["x"], s["codes"], s["scales"], s["ts"], b.TS_GIVEN, step.err)
     torch.cuda.synchronize()
-    calls = {
+    calls = {name: (lambda name=name: step.run_one(name, 0)) for name in Step.EXTRA}
+    calls.update({
         "amax": lambda: b.if4_tensor_amax(s["x"], s["amax"], step.err),
         "if4_quantize": lambda: b.if4_quantize(s["x"], s["codes"], s["scales"], s["ts"],
                                                b.TS_GIVEN, step.err),
         "if4_dequantize": lambda: b.if4_dequantize(s["codes"], s["scales"], s["ts"], s["y"]),
         "nvfp4_quantize": lambda: b.nvfp4_quantize(s["x"], s["ncodes"], s["nscales"], s["ts"],
                                                    b.TS_GIVEN, step.err),
-    }
+    })
     for _ in range(args.warmup + args.steps):
         calls[args.kernel_only]()
     torch.cuda.synchronize()
     print(json.dumps({"kernel_only": args.kernel_only, "workload": args.workload,
                       "launches": args.warmup + args.steps, "err": int(step.err.item())}))
+    if int(step.err.item()) != 0:
+        sys.exit(1)
 
 
 def main():

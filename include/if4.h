@@ -96,7 +96,7 @@ enum {
 /* Largest supported tensor: rows * cols / 16 < 2^31 groups. */
 
 /*
- * A1: amax = max |x| over x[rows, cols] (device float).  x_dtype is IF4_F32,
+ * Tensor amax: amax = max |x| over x[rows, cols] (device float).  x_dtype is IF4_F32,
  * IF4_BF16 or IF4_F16; x 16-byte aligned, ld_x*elem_size % 16 == 0.
  * err_flag may be NULL; otherwise IF4_DEV_NONFINITE is set for Inf/NaN.
  * (The tensor scale of NVFP4-style formats; arXiv abstract.)
@@ -104,14 +104,14 @@ enum {
 int if4_tensor_amax(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
                     float *amax, int *err_flag, void *stream);
 
-/* A2: ts = amax / 2688 (1 if amax == 0, floored at 2^-117), device to device. */
+/* Tensor scale: ts = amax / 2688 (1 if amax == 0, floored at 2^-117), device to device. */
 int if4_tensor_scale(const float *amax, float *ts, void *stream);
 
 /*
- * A1-A6: IF4 quantize.  Per group of 16: the E4M3 block scale, the FP4 and
+ * IF4 quantize.  Per group of 16: the E4M3 block scale, the FP4 and
  * the 7/6-scaled INT4 candidates, the lower-error choice in bit 7 of the
  * scale byte (gist.science section 2; shd-paper.top framework steps 1-5).
- * ts_mode IF4_TS_COMPUTE runs A1/A2 first and writes *ts; IF4_TS_GIVEN reads
+ * ts_mode IF4_TS_COMPUTE runs the amax and scale steps first and writes *ts; IF4_TS_GIVEN reads
  * it.  codes must be 16-byte aligned.  err_flag may be NULL.
  */
 int if4_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
@@ -119,7 +119,7 @@ int if4_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t
                  int *err_flag, void *stream);
 
 /*
- * A9: NVFP4 quantize, the comparator: the FP4 candidate of if4_quantize for
+ * NVFP4 quantize, the comparator: the FP4 candidate of if4_quantize for
  * every group, bit 7 of every scale byte 0.  Same arguments and rules.
  */
 int nvfp4_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
@@ -169,7 +169,7 @@ int nvfp4_4over6_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols
                           int *err_flag, void *stream);
 
 /*
- * A7: dequantize IF4 (or NVFP4) to y[rows, cols] of y_dtype (IF4_F32,
+ * Dequantize IF4 (or NVFP4) to y[rows, cols] of y_dtype (IF4_F32,
  * IF4_BF16 or IF4_F16), row stride ld_y elements: fl(q * fl(E4M3 * ts)),
  * then RNE to the output type.  codes 16-byte aligned; y 16-byte aligned and
  * ld_y*elem_size % 16 == 0.  (gist.science section 2, "Metodo 6/7";
@@ -202,7 +202,7 @@ int if4_gemm_f16(const void *a, const void *b, const float *a_ts, const float *b
 size_t if4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
- * A8: IF4 x IF4 linear.  C[M, N] (bf16, dense) = sum_k A_hat[m, k] *
+ * IF4 x IF4 linear.  C[M, N] (bf16, dense) = sum_k A_hat[m, k] *
  * B_hat[n, k] where A (activations, [M, K]) and B (weights, [N, K], i.e. C =
  * A B^T) are both IF4 along K.  Runs if4_decode_f16 on both operands into
  * the caller's workspace, then if4_gemm_f16 with the two tensor scales in
@@ -224,7 +224,7 @@ int if4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_t
  * device memory at the call: for example a plugin inside a framework that
  * owns all device memory through its own pool, or a latency-critical path
  * that must not risk the device synchronisation cudaMalloc can cause.  The
- * pages have no counterpart; this is a deployment variant of A8.
+ * pages have no counterpart; this is a deployment variant of if4_linear.
  * Same arguments and result as if4_linear.  The decoded operands live in a
  * fixed scratch array in the library's device code (IF4_LINEAR_NOALLOC_MAX_BYTES
  * per device, held from when the library's device code is loaded on that

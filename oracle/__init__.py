@@ -165,7 +165,7 @@ def quantize(x, ts, mode: int = MODE_IF4, threads: int = 0):
 
 
 def quantize_tensor(x, mode: int = MODE_IF4, threads: int = 0):
-    """A1-A6: tensor amax, tensor scale, then the per-group quantizer."""
+    """Tensor amax, tensor scale, then the per-group quantizer."""
     amax = tensor_amax(x)
     ts = tensor_scale(amax)
     out = quantize(x, ts, mode, threads)
@@ -184,13 +184,13 @@ def rht(x, signs: int, threads: int = 0):
 
 
 def quantize_tensor_rht(x, signs: int, mode: int = MODE_IF4, threads: int = 0):
-    """The transform, then A1-A6 on the transformed tensor."""
+    """The transform, then amax, tensor scale and quantizer on its output."""
     out = quantize_tensor(rht(x, signs, threads), mode, threads)
     return out
 
 
 def dequantize(codes, scales, ts, threads: int = 0):
-    """A7: float32 [rows, cols] = fl(q * fl(E4(scale) * ts))."""
+    """Dequantize: float32 [rows, cols] = fl(q * fl(E4(scale) * ts))."""
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.uint8)
     rows, cols = codes.shape[0], codes.shape[1] * 2

@@ -140,7 +140,7 @@ float orc_int4_value(uint8_t nib)
     return (float)(6 * k) / 7.0f;
 }
 
-/* ----------------------------------------------- tensor scale (A1, A2) ---- */
+/* --------------------------------------- tensor amax and tensor scale ---- */
 
 float orc_tensor_amax(const float *x, int64_t rows, int64_t cols, int64_t ld)
 {
@@ -162,7 +162,7 @@ float orc_tensor_scale(float amax)
     return ts < floor_ts ? floor_ts : ts;
 }
 
-/* ------------------------------------------------- quantize (A3 - A6) ----- */
+/* ------------------------------------------------------------ quantize ---- */
 
 /* IF4: lower-error candidate per group.  NVFP4: FP4 always.  NVINT4: the
  * 7/6-scaled INT4 candidate always, bit 7 set (the all-INT4 format the pages
@@ -328,7 +328,7 @@ void orc_rht(const float *x, int64_t rows, int64_t cols, int64_t ld, uint32_t si
     (void)nthreads;
 }
 
-/* ------------------------------------------------------ dequantize (A7) --- */
+/* ---------------------------------------------------------- dequantize ---- */
 
 /* y[r, c] = fl(q * fl(E4(sb) * ts)), q decoded as FP4 or INT4 by bit 7. */
 void orc_dequantize(const uint8_t *codes, const uint8_t *scales, float ts, int64_t rows,

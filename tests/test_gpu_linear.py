@@ -138,3 +138,16 @@ def test_linear_workspace_and_shape_errors():
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     with pytest.raises(bb.IF4Error, match="workspace"):
         bb.if4_linear(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], small, c, err)
+
+
+def test_pair_and_single_cta_paths_agree():
+    """M, N >= 256 runs the CTA-pair kernel; 128-row slices of the same A run
+    the one-CTA kernel.  Both accumulate each output over K in the same order
+    (16-wide MMA steps, 64-wide slabs), so the results are identical."""
+    M, N, K = 512, 768, 2048
+    g = torch.Generator().manual_seed(77)
+    a = torch.randn((M, K), generator=g).to(torch.float16).cuda()
+    b = (torch.randn((N, K), generator=g) * 0.05).to(torch.float16).cuda()
+    full = gemm(a, b, 0.5, 2.0)
+    parts = torch.cat([gemm(a[i:i + 128].contiguous(), b, 0.5, 2.0) for i in range(0, M, 128)])
+    assert torch.equal(full, parts)
