@@ -178,6 +178,14 @@ __device__ __forceinline__ uint32_t f16x2_from_f32(float lo, float hi)
     return r;
 }
 
+// The two bf16 halves of w as an exact float pair (low half first).
+__device__ __forceinline__ unsigned long long f2_from_bf16x2(uint32_t w)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+    return r;
+}
+
 // ----------------------------------------------------------- integers ----
 
 __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)

@@ -104,7 +104,7 @@ __device__ __forceinline__ float unpack_group(const Raw<DT> &r, f2_t (&x)[8], bo
             const uint32_t w = r.w[j];
             m = (DT == DT_BF16) ? absmax_bf16x2(m, w) : absmax_f16x2(m, w);
             if constexpr (DT == DT_BF16)
-                x[j] = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+                x[j] = f2_from_bf16x2(w);
             else
                 x[j] = f2_pack(f16lo_to_f32(w), f16hi_to_f32(w));
         }
@@ -197,7 +197,7 @@ __device__ __forceinline__ float unpack_group_rht(const Raw<DT> &r, const SignMa
         for (int j = 0; j < 8; ++j) {
             const uint32_t w = r.w[j] ^ sm.w[j];
             if constexpr (DT == DT_BF16)
-                x[j] = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+                x[j] = f2_from_bf16x2(w);
             else
                 x[j] = f2_pack(f16lo_to_f32(w), f16hi_to_f32(w));
         }
@@ -530,6 +530,16 @@ __device__ __noinline__ GroupCode encode_group_clamped(uint32_t sb, float inv, c
     return encode_group<DT, MODE, true, RHT>(x, sb, inv, p, signs);
 }
 
+// Address of group g of a [rows, gpr groups] tensor with row stride
+// ld_bytes (a contiguous tensor is passed as one row of every group).
+template <int GB>
+__device__ __forceinline__ const char *group_addr(const char *x, uint32_t g, uint32_t gpr,
+                                                  int64_t ld_bytes)
+{
+    const uint32_t row = g / gpr;
+    return x + (int64_t)row * ld_bytes + (int64_t)(g - row * gpr) * GB;
+}
+
 // fl(fl(amax / 4) / ts): amax / 4 is exact (a power of two) above 2^-124,
 // the quotient by ts is Markstein's, as in block_scale.
 __device__ __forceinline__ float block_scale4(float amax, float ts, float rts)
@@ -619,7 +629,8 @@ __device__ __noinline__ bool four_wins_exact(const char *p, float inv6, float ef
 template <int DT>
 __device__ __forceinline__ GroupCode encode_group_46(const f2_t (&x)[8], float amax, float ts,
                                                    float rts, const float *inv_tab,
-                                                   const float *eff_tab, const char *p)
+                                                   const float *eff_tab, const char *xbase,
+                                                   uint32_t g, uint32_t gpr, int64_t ld_bytes)
 {
     const uint32_t sb6 = e4m3_from_f32(block_scale(amax, ts, rts)) & 0x7Fu;
     const uint32_t sb4 = e4m3_from_f32(block_scale4(amax, ts, rts)) & 0x7Fu;
@@ -659,7 +670,8 @@ __device__ __forceinline__ GroupCode encode_group_46(const f2_t (&x)[8], float a
     if (sb4 == sb6)
         four = false;                 // identical candidates: a tie, keep /6
     else if (!(fabsf(d) > band))
-        four = four_wins_exact<DT>(p, inv6, eff6, inv4, eff4);
+        four = four_wins_exact<DT>(group_addr<16 * elem_bytes<DT>()>(xbase, g, gpr, ld_bytes), inv6,
+                                   eff6, inv4, eff4);
     GroupCode out;
     const uint32_t sb = four ? sb4 : sb6;
     out.c0 = four ? w4[0] : w6[0];
@@ -669,12 +681,136 @@ __device__ __forceinline__ GroupCode encode_group_46(const f2_t (&x)[8], float a
     return out;
 }
 
+// IF4 groups off the fast path (rare): a block scale that the quotients of
+// the fast path do not give exactly, or one under which the INT4 integer may
+// need its clamp.  The block scale with its exact fallbacks, then the encode
+// with the clamp, from the group re-read from memory.
+template <int DT, bool RHT>
+__device__ __noinline__ GroupCode if4_group_general(float amax, float ts, float rts,
+                                                    const float *inv_tab, const char *gp,
+                                                    uint32_t signs)
+{
+    const uint32_t sb = e4m3_from_f32(block_scale(amax, ts, rts)) & 0x7Fu;
+    float y[16];
+    reload_group<DT, RHT>(gp, signs, y);
+    f2_t x[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = f2_pack(y[2 * j], y[2 * j + 1]);
+    GroupCode out = encode_group<DT, Q_IF4, true, RHT>(x, sb, inv_tab[sb], gp, signs);
+    if (sb == 0) out.c0 = out.c1 = out.scale = 0u;
+    return out;
+}
+
+// IF4 groups whose binary32 margin is within rounding: equal candidates keep
+// FP4, anything else is decided by the binary64 rule.
+template <int DT, bool RHT>
+__device__ __noinline__ GroupCode if4_group_near(uint32_t f0, uint32_t f1, uint32_t i0,
+                                                 uint32_t i1, uint32_t sb, float inv,
+                                                 const char *gp, uint32_t signs)
+{
+    const bool int4 = !(candidates_coincide(f0, i0) && candidates_coincide(f1, i1)) &&
+                      int4_wins_exact<DT, RHT>(gp, inv, signs);
+    GroupCode out;
+    out.c0 = int4 ? i0 : f0;
+    out.c1 = int4 ? i1 : f1;
+    out.scale = int4 ? (sb | 0x80u) : sb;
+    return out;
+}
+
+// 1.5 * 2^23 + 8: fma(v, fl(7/6), kMagic8) leaves k + 8 in bits 0-3 of the
+// result and zeros in bits 4-7 whenever |k| = |RNE(v * fl(7/6))| <= 7.
+constexpr float kMagic8 = 12582920.0f;
+
+// IF4 encode of one group, fast path.  Block scale by Markstein quotients
+// (exact unless flagged below); both candidates without the INT4 clamp (it is
+// the identity for every block scale E4M3 code 8..125: the largest |v| is
+// then at most 6 * 17/16 = 6.375 and 6.375 * fl(7/6) < 7.5); the decision by
+// binary32 error sums with the band of encode_group.  One branch leaves the
+// path for every rare case: a flagged block scale (tiny amax, a quotient of
+// 2^100 or more, Inf/NaN), a block scale code 1..7 or 126 (the clamp may
+// act), or a margin within the band.
+template <int DT, bool RHT>
+__device__ __forceinline__ GroupCode encode_if4(const f2_t (&xv)[8], float amax, float ts,
+                                              float rts, const float *inv_tab, const char *x,
+                                              uint32_t g, uint32_t gpr, int64_t ld_bytes,
+                                              uint32_t signs)
+{
+    constexpr int GB = 16 * elem_bytes<DT>();
+    const float r6 = __uint_as_float(0x3E2AAAABu);          // RN(1/6)
+    float q = __fmul_rn(amax, r6);
+    q = __fmaf_rn(__fmaf_rn(-q, 6.0f, amax), r6, q);
+    const float s = __fmul_rn(q, rts);
+    const float t = __fmaf_rn(__fmaf_rn(-s, ts, q), rts, s);
+    const uint32_t sb = e4m3_from_f32(t) & 0x7Fu;
+    const bool general = !(amax >= 0x1p-100f && s < 0x1p100f) || (sb - 1u) < 7u || sb == 0x7Eu;
+    const float inv = inv_tab[sb];
+
+    const f2_t INV = f2_pack(inv, inv);
+    f2_t v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = f2_mul(xv[j], INV);
+    const f2_t lo[4] = {v[0], v[1], v[2], v[3]};
+    const f2_t hi[4] = {v[4], v[5], v[6], v[7]};
+    f2_t dlo[4], dhi[4];
+    const uint32_t f0 = fp4_word<true>(lo, dlo);
+    const uint32_t f1 = fp4_word<true>(hi, dhi);
+
+    const f2_t C76 = f2_pack(c76(), c76());
+    const f2_t M8 = f2_pack(kMagic8, kMagic8);
+    const f2_t NM8 = f2_pack(-kMagic8, -kMagic8);
+    const f2_t NC67 = f2_pack(-c67(), -c67());
+    f2_t ef = f2_pack(0.0f, 0.0f), ei = f2_pack(0.0f, 0.0f);
+    uint32_t pb[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const f2_t r = f2_fma(v[j], C76, M8);                // M8 + RNE(v * fl(7/6))
+        const f2_t di = f2_fma(f2_add(r, NM8), NC67, v[j]);   // v - k * fl(6/7), one rounding
+        const f2_t df = j < 4 ? dlo[j] : dhi[j - 4];
+        ef = f2_fma(df, df, ef);
+        ei = f2_fma(di, di, ei);
+        float re, ro;
+        f2_unpack(r, re, ro);
+        // byte 0: (k_even + 8) | (k_odd + 8) << 4
+        pb[j] = __float_as_uint(ro) * 16u + __float_as_uint(re);
+    }
+    // gather the bytes, then offset-8 nibbles -> two's complement nibbles
+    const uint32_t i0 = prmt(prmt(pb[0], pb[1], 0x0040u), prmt(pb[2], pb[3], 0x0040u), 0x5410u) ^
+                        0x88888888u;
+    const uint32_t i1 = prmt(prmt(pb[4], pb[5], 0x0040u), prmt(pb[6], pb[7], 0x0040u), 0x5410u) ^
+                        0x88888888u;
+
+    float a0, a1, b0, b1;
+    f2_unpack(ef, a0, a1);
+    f2_unpack(ei, b0, b1);
+    const float e_fp = __fadd_rn(a0, a1), e_int = __fadd_rn(b0, b1);
+    const float d = __fsub_rn(e_fp, e_int);
+    const float S = __fadd_rn(e_fp, e_int);
+    const float band = __fmul_rn(__fadd_rn(S, 1.0f), 0x1p-18f);
+    const bool int4 = d > band;
+    // S == 0: every binary32 square is zero, so every error is (a) zero or
+    // (b) below 2^-75, where both candidates are 0: the sums tie, FP4 stays
+    const bool near = !(fabsf(d) > band) && S != 0.0f;
+    GroupCode out;
+    if (general || near) {
+        const char *gp = group_addr<GB>(x, g, gpr, ld_bytes);
+        out = general ? if4_group_general<DT, RHT>(amax, ts, rts, inv_tab, gp, signs)
+                      : if4_group_near<DT, RHT>(f0, f1, i0, i1, sb, inv, gp, signs);
+    } else {
+        out.c0 = int4 ? i0 : f0;
+        out.c1 = int4 ? i1 : f1;
+        out.scale = int4 ? (sb | 0x80u) : sb;
+        // sb == 0: inv = 0, both candidates are (signed) zeros, the sums 0
+        if (sb == 0) out.c0 = out.c1 = 0u;
+    }
+    return out;
+}
+
 // Encode group g from its raw bits r and store its codes and scale byte.
 // Returns true when an input element is Inf or NaN.
 template <int DT, int MODE, bool RHT>
 __device__ __forceinline__ bool quantize_one(const Raw<DT> &r, uint32_t g, const char *x,
-                                             int64_t ld_bytes, uint32_t gpr, int contig, float ts,
-                                             float rts, const float *inv_tab, const float *eff_tab,
+                                             int64_t ld_bytes, uint32_t gpr, float ts, float rts,
+                                             const float *inv_tab, const float *eff_tab,
                                              uint8_t *codes, uint8_t *scales,
                                              const SignMasks &sm, uint32_t signs)
 {
@@ -686,45 +822,47 @@ __device__ __forceinline__ bool quantize_one(const Raw<DT> &r, uint32_t g, const
         amax = unpack_group_rht<DT>(r, sm, xv, nonfinite);
     else
         amax = unpack_group<DT>(r, xv, nonfinite);
-    if constexpr (MODE == Q_46) {
-        const GroupCode out = encode_group_46<DT>(xv, amax, ts, rts, inv_tab, eff_tab,
-                                                  group_ptr(x, g, contig, gpr, ld_bytes, GB));
-        st_v2(codes + (int64_t)g * 8, out.c0, out.c1);
-        st_u8(scales + g, out.scale);
-        return nonfinite;
-    }
-    // block scale
-    const uint32_t sb = e4m3_from_f32(block_scale(amax, ts, rts)) & 0x7Fu;
-    // sb == 0: inv = 0 makes every candidate 0; the outputs are forced to
-    // all-zero FP4 below, without a branch around the arithmetic
-    const float inv = inv_tab[sb];
-    const char *gp = group_ptr(x, g, contig, gpr, ld_bytes, GB);
     GroupCode out;
-    // The INT4 integer needs a clamp only if some |v| * fl(7/6) can reach
-    // 7.5; |v| is monotonic in |x|, so the group's max decides.
-    if (__fmul_rn(__fmul_rn(amax, inv), c76()) >= 7.5f)
-        out = encode_group_clamped<DT, MODE, RHT>(sb, inv, gp, signs);
-    else
-        out = encode_group<DT, MODE, false, RHT>(xv, sb, inv, gp, signs);
-    if (sb == 0) out.c0 = out.c1 = out.scale = 0u;
+    if constexpr (MODE == Q_IF4) {
+        out = encode_if4<DT, RHT>(xv, amax, ts, rts, inv_tab, x, g, gpr, ld_bytes, signs);
+    } else if constexpr (MODE == Q_46) {
+        out = encode_group_46<DT>(xv, amax, ts, rts, inv_tab, eff_tab, x, g, gpr, ld_bytes);
+    } else {
+        const uint32_t sb = e4m3_from_f32(block_scale(amax, ts, rts)) & 0x7Fu;
+        // sb == 0: inv = 0 makes every candidate 0; the outputs are forced
+        // to all-zero codes below
+        const float inv = inv_tab[sb];
+        // NVINT4: the clamp can act only under block scale codes 1..7 and
+        // 126 (see encode_if4); FP4 saturates by itself
+        if (MODE == Q_NVINT4 && ((sb - 1u) < 7u || sb == 0x7Eu))
+            out = encode_group_clamped<DT, MODE, RHT>(sb, inv, group_addr<GB>(x, g, gpr, ld_bytes),
+                                                      signs);
+        else
+            out = encode_group<DT, MODE, false, RHT>(xv, sb, inv, nullptr, signs);
+        if (sb == 0) out.c0 = out.c1 = out.scale = 0u;
+    }
     st_v2(codes + (int64_t)g * 8, out.c0, out.c1);
     st_u8(scales + g, out.scale);
     return nonfinite;
 }
 
-template <int DT, int MODE, bool V8, bool RHT>
-__global__ void __launch_bounds__(256)
-quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, uint32_t ngroups,
-                int contig, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
-                const float *__restrict__ ts_ptr, int *err, int check_ts,
-                const __grid_constant__ SignMasks sm, uint32_t signs)
+// Quantizer kernel: one group per thread per step of a grid-stride loop,
+// the group's 32 (64) bytes in one (two) 256-bit loads, and the loads of the
+// next PF groups in flight while the current one is encoded (PF = 2 for the
+// light single-candidate modes, whose few instructions per group would not
+// otherwise hide the memory latency; 1 for the rest, which keeps them at four
+// resident blocks per SM).
+template <int DT, int MODE, bool V8, bool RHT, int PF>
+__global__ void __launch_bounds__(256, DT == DT_F32 ? 3 : 4)
+quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr,
+                       uint32_t ngroups, int contig, uint8_t *__restrict__ codes,
+                       uint8_t *__restrict__ scales, const float *__restrict__ ts_ptr, int *err,
+                       int check_ts, const __grid_constant__ SignMasks sm, uint32_t signs)
 {
     constexpr int GB = 16 * elem_bytes<DT>();
     const float ts = *ts_ptr;
     if (check_ts && blockIdx.x == 0 && threadIdx.x == 0 && !ts_valid(ts) && err)
         atomicOr(err, IF4_DEV_BAD_SCALE);
-    // inv_tab[c] = fl(1 / fl(E4M3(c) * ts)), the reciprocal of every block
-    // scale this tensor can use; inv_tab[0] = 0 (an underflowed block scale)
     __shared__ float inv_tab[128];
     __shared__ float eff_tab[MODE == Q_46 ? 128 : 1];
     if (threadIdx.x < 128) {
@@ -734,25 +872,29 @@ quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, uint
     }
     const float rts = __frcp_rn(ts);
     __syncthreads();
-
+    // the address of a group: contiguous tensors without a division
+    const uint32_t gpr_eff = contig ? ngroups : gpr;
+    auto addr = [&](uint32_t g) -> const char * {
+        return contig ? x + (int64_t)g * GB : group_addr<GB>(x, g, gpr, ld_bytes);
+    };
     const uint32_t stride = gridDim.x * blockDim.x;
     uint32_t g = blockIdx.x * blockDim.x + threadIdx.x;
     bool saw_nonfinite = false;
-    // Two register buffers, used in turn: the next group's load is in flight
-    // while the current one is encoded, with no copy between them.
-    Raw<DT> buf[2];
-    if (g < ngroups) load_group<DT, V8>(group_ptr(x, g, contig, gpr, ld_bytes, GB), buf[0]);
+    // PF + 1 register buffers used in turn (g < 2^31 and the stride is far
+    // below 2^31, so g + 2 * stride cannot wrap)
+    Raw<DT> buf[PF + 1];
+    if (g < ngroups) load_group<DT, V8>(addr(g), buf[0]);
+    if (PF == 2 && g + stride < ngroups) load_group<DT, V8>(addr(g + stride), buf[1]);
     for (; g < ngroups;) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const uint32_t gn = g + stride;
-            const bool more = gn < ngroups && gn > g;
-            if (more) load_group<DT, V8>(group_ptr(x, gn, contig, gpr, ld_bytes, GB), buf[half ^ 1]);
-            saw_nonfinite |= quantize_one<DT, MODE, RHT>(buf[half], g, x, ld_bytes, gpr, contig,
-                                                          ts, rts, inv_tab, eff_tab, codes, scales,
-                                                          sm, signs);
-            g = more ? gn : ngroups;
-            if (!more) break;
+        for (int ph = 0; ph <= PF; ++ph) {
+            const uint32_t gp = g + PF * stride;
+            if (gp < ngroups) load_group<DT, V8>(addr(gp), buf[(ph + PF) % (PF + 1)]);
+            saw_nonfinite |= quantize_one<DT, MODE, RHT>(buf[ph], g, x, ld_bytes, gpr_eff, ts,
+                                                          rts, inv_tab, eff_tab, codes, scales, sm,
+                                                          signs);
+            g += stride;
+            if (g >= ngroups) break;
         }
     }
     if (saw_nonfinite && err) atomicOr(err, IF4_DEV_NONFINITE);
@@ -1125,17 +1267,23 @@ int dispatch_amax(int dt, const Shape &s, const void *x, unsigned int *amax_bits
     }
 }
 
-template <int DT, int MODE, bool V8, bool RHT>
+template <int DT, int MODE, bool RHT>
 int launch_quant(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
                  const float *ts, int *err, int check_ts, cudaStream_t st, const DeviceInfo &d,
                  const SignMasks &sm, uint32_t signs)
 {
     if (s.ngroups == 0) return IF4_OK;
-    auto k = quantize_kernel<DT, MODE, V8, RHT>;
-    static const int occ = resident_blocks(k, 256);
-    const uint32_t grid = grid_for(occ, d, s.ngroups, 256);
-    k<<<grid, 256, 0, st>>>(static_cast<const char *>(x), s.ld_bytes, s.gpr, s.ngroups,
-                            s.contig ? 1 : 0, codes, scales, ts, err, check_ts, sm, signs);
+    constexpr int PF = (DT != DT_F32 && (MODE == Q_NVFP4 || MODE == Q_NVINT4)) ? 2 : 1;
+    auto launch = [&](auto k) {
+        static const int occ = resident_blocks(k, 256);
+        const uint32_t grid = grid_for(occ, d, s.ngroups, 256);
+        k<<<grid, 256, 0, st>>>(static_cast<const char *>(x), s.ld_bytes, s.gpr, s.ngroups,
+                                s.contig ? 1 : 0, codes, scales, ts, err, check_ts, sm, signs);
+    };
+    if (s.v8)
+        launch(quantize_kernel<DT, MODE, true, RHT, PF>);
+    else
+        launch(quantize_kernel<DT, MODE, false, RHT, PF>);
     return launch_status();
 }
 
@@ -1144,10 +1292,7 @@ int dispatch_quant_dt(const Shape &s, const void *x, uint8_t *codes, uint8_t *sc
                       const float *ts, int *err, int check_ts, cudaStream_t st,
                       const DeviceInfo &d, const SignMasks &sm, uint32_t signs)
 {
-    return s.v8 ? launch_quant<DT, MODE, true, RHT>(s, x, codes, scales, ts, err, check_ts, st, d,
-                                                    sm, signs)
-                : launch_quant<DT, MODE, false, RHT>(s, x, codes, scales, ts, err, check_ts, st,
-                                                     d, sm, signs);
+    return launch_quant<DT, MODE, RHT>(s, x, codes, scales, ts, err, check_ts, st, d, sm, signs);
 }
 
 template <int MODE, bool RHT>
