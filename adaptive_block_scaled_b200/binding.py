@@ -52,6 +52,8 @@ def _load():
         "if4_tensor_amax_rht": [_vp, _int, _i64, _i64, _i64, ctypes.c_uint32, _vp, _vp, _vp],
         "if4_quantize_rht": [_vp, _int, _i64, _i64, _i64, ctypes.c_uint32, _vp, _vp, _vp, _int,
                              _vp, _vp],
+        "if4_quantize_fused": [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                               _vp],
         "if4_decode_f16": [_vp, _vp, _i64, _i64, _vp, _vp],
         "if4_gemm_f16": [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
         "if4_linear_workspace_bytes": [_i64, _i64, _i64],
@@ -156,6 +158,25 @@ def if4_quantize_rht(x, signs, codes, scales, ts, ts_mode=TS_COMPUTE, err_flag=N
                                 _stream(stream)), "if4_quantize_rht")
 
 
+def if4_quantize_fused(x, codes, scales, nv_codes, nv_scales, ts, sync_words, err_flag=None,
+                       stream=None):
+    rows, cols, ld = _matrix(x, "x")
+    _u8(codes, "codes", (rows, cols // 2))
+    _u8(scales, "scales", (rows, cols // 16))
+    if (nv_codes is None) != (nv_scales is None):
+        raise ValueError("nv_codes and nv_scales go together")
+    if nv_codes is not None:
+        _u8(nv_codes, "nv_codes", (rows, cols // 2))
+        _u8(nv_scales, "nv_scales", (rows, cols // 16))
+    if sync_words.dtype != torch.int32 or sync_words.numel() < FUSED_SYNC_WORDS:
+        raise ValueError(f"sync_words must be an int32 device tensor of at least "
+                         f"{FUSED_SYNC_WORDS} elements")
+    _check(lib.if4_quantize_fused(_ptr(x), _dtype(x, "x"), rows, cols, ld, _ptr(codes),
+                                  _ptr(scales), _ptr(nv_codes), _ptr(nv_scales), _ptr(ts),
+                                  _ptr(sync_words), _ptr(err_flag), _stream(stream)),
+           "if4_quantize_fused")
+
+
 def nvint4_quantize(x, codes, scales, ts, ts_mode=TS_COMPUTE, err_flag=None, stream=None):
     _quantize_call(lib.nvint4_quantize, "nvint4_quantize", x, codes, scales, ts, ts_mode,
                    err_flag, stream)
@@ -234,6 +255,7 @@ def if4_linear_noalloc(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, c, err_
 
 
 LINEAR_NOALLOC_MAX_BYTES = 32 * 1024 * 1024
+FUSED_SYNC_WORDS = 64
 
 
 # ---------------------------------------------------- allocating helpers ---
@@ -268,6 +290,22 @@ def quantize_rht(x, signs, ts=None, err_flag=None, stream=None):
         ts_t, ts_mode = ts, TS_GIVEN
     if4_quantize_rht(x, signs, codes, scales, ts_t, ts_mode, err_flag, stream)
     return codes, scales, ts_t
+
+
+def quantize_fused(x, with_nvfp4=True, sync_words=None, err_flag=None, stream=None):
+    """amax, tensor scale, IF4 quantize (and NVFP4) in one launch.  Returns
+    (codes, scales, ts) or (codes, scales, ts, nv_codes, nv_scales)."""
+    rows, cols, _ = _matrix(x, "x")
+    dev = x.device
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+    nv_codes = torch.empty_like(codes) if with_nvfp4 else None
+    nv_scales = torch.empty_like(scales) if with_nvfp4 else None
+    ts = torch.empty(1, dtype=torch.float32, device=dev)
+    if sync_words is None:
+        sync_words = torch.zeros(FUSED_SYNC_WORDS, dtype=torch.int32, device=dev)
+    if4_quantize_fused(x, codes, scales, nv_codes, nv_scales, ts, sync_words, err_flag, stream)
+    return (codes, scales, ts, nv_codes, nv_scales) if with_nvfp4 else (codes, scales, ts)
 
 
 def dequantize(codes, scales, ts, dtype=torch.bfloat16, stream=None):

@@ -186,6 +186,14 @@ __device__ __forceinline__ unsigned long long f2_from_bf16x2(uint32_t w)
     return r;
 }
 
+// Wall clock in nanoseconds, for bounded waits.
+__device__ __forceinline__ unsigned long long globaltimer_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 // ----------------------------------------------------------- integers ----
 
 __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)

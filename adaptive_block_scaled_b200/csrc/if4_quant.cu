@@ -391,6 +391,7 @@ __device__ __noinline__ bool int4_wins_rare(uint32_t f0, uint32_t f1, uint32_t i
 struct GroupCode {
     uint32_t c0, c1;   // codes of elements 0..7 and 8..15
     uint32_t scale;    // scale byte
+    uint32_t f0, f1;   // IF4 paths: the FP4 candidate's codes (the NVFP4 codes)
 };
 
 // Encode one group from its 16 inputs x (pairs), the block scale byte sb and
@@ -440,6 +441,8 @@ __device__ __forceinline__ GroupCode encode_group(const f2_t (&x)[8], uint32_t s
         f2_t dlo[4], dhi[4];
         out.c0 = fp4_word<true>(lo, dlo);
         out.c1 = fp4_word<true>(hi, dhi);
+        out.f0 = out.c0;
+        out.f1 = out.c1;
         f2_t ef = f2_pack(0.0f, 0.0f), ei = f2_pack(0.0f, 0.0f);
         f2_t r[8];
 #pragma unroll
@@ -697,7 +700,7 @@ __device__ __noinline__ GroupCode if4_group_general(float amax, float ts, float 
 #pragma unroll
     for (int j = 0; j < 8; ++j) x[j] = f2_pack(y[2 * j], y[2 * j + 1]);
     GroupCode out = encode_group<DT, Q_IF4, true, RHT>(x, sb, inv_tab[sb], gp, signs);
-    if (sb == 0) out.c0 = out.c1 = out.scale = 0u;
+    if (sb == 0) out.c0 = out.c1 = out.scale = out.f0 = out.f1 = 0u;
     return out;
 }
 
@@ -714,6 +717,8 @@ __device__ __noinline__ GroupCode if4_group_near(uint32_t f0, uint32_t f1, uint3
     out.c0 = int4 ? i0 : f0;
     out.c1 = int4 ? i1 : f1;
     out.scale = int4 ? (sb | 0x80u) : sb;
+    out.f0 = f0;
+    out.f1 = f1;
     return out;
 }
 
@@ -796,23 +801,26 @@ __device__ __forceinline__ GroupCode encode_if4(const f2_t (&xv)[8], float amax,
         out = general ? if4_group_general<DT, RHT>(amax, ts, rts, inv_tab, gp, signs)
                       : if4_group_near<DT, RHT>(f0, f1, i0, i1, sb, inv, gp, signs);
     } else {
-        out.c0 = int4 ? i0 : f0;
-        out.c1 = int4 ? i1 : f1;
-        out.scale = int4 ? (sb | 0x80u) : sb;
         // sb == 0: inv = 0, both candidates are (signed) zeros, the sums 0
-        if (sb == 0) out.c0 = out.c1 = 0u;
+        out.f0 = sb == 0 ? 0u : f0;
+        out.f1 = sb == 0 ? 0u : f1;
+        out.c0 = int4 ? i0 : out.f0;
+        out.c1 = int4 ? i1 : out.f1;
+        out.scale = int4 ? (sb | 0x80u) : sb;
     }
     return out;
 }
 
 // Encode group g from its raw bits r and store its codes and scale byte.
 // Returns true when an input element is Inf or NaN.
-template <int DT, int MODE, bool RHT>
+template <int DT, int MODE, bool RHT, bool NV = false>
 __device__ __forceinline__ bool quantize_one(const Raw<DT> &r, uint32_t g, const char *x,
                                              int64_t ld_bytes, uint32_t gpr, float ts, float rts,
                                              const float *inv_tab, const float *eff_tab,
                                              uint8_t *codes, uint8_t *scales,
-                                             const SignMasks &sm, uint32_t signs)
+                                             const SignMasks &sm, uint32_t signs,
+                                             uint8_t *nv_codes = nullptr,
+                                             uint8_t *nv_scales = nullptr)
 {
     constexpr int GB = 16 * elem_bytes<DT>();
     f2_t xv[8];
@@ -843,6 +851,11 @@ __device__ __forceinline__ bool quantize_one(const Raw<DT> &r, uint32_t g, const
     }
     st_v2(codes + (int64_t)g * 8, out.c0, out.c1);
     st_u8(scales + g, out.scale);
+    if constexpr (NV && MODE == Q_IF4) {
+        // the NVFP4 comparator: the FP4 candidate under the same block scale
+        st_v2(nv_codes + (int64_t)g * 8, out.f0, out.f1);
+        st_u8(nv_scales + g, out.scale & 0x7Fu);
+    }
     return nonfinite;
 }
 
@@ -923,15 +936,15 @@ __device__ __forceinline__ uint32_t group_absmax_bits(const Raw<DT> &r)
 }
 
 // Tensor amax: max |x| over the tensor, accumulated as float bits with atomicMax into
-// *amax_bits (zeroed by the caller's stream).  Each thread keeps four group
-// loads in flight.
+// *amax_bits (zeroed by the caller's stream).  Each thread keeps eight group
+// loads (four for f32) in flight.
 template <int DT, bool V8, bool RHT>
 __global__ void __launch_bounds__(256)
 amax_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, uint32_t ngroups,
             int contig, unsigned int *amax_bits, int *err, const __grid_constant__ SignMasks sm)
 {
     constexpr int GB = 16 * elem_bytes<DT>();
-    constexpr int U = 4;
+    constexpr int U = DT == DT_F32 ? 4 : 8;
     uint32_t m = 0;
     const uint32_t stride = gridDim.x * blockDim.x;
     for (uint64_t g0 = blockIdx.x * blockDim.x + threadIdx.x; g0 < ngroups;
@@ -970,15 +983,154 @@ amax_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, uint32_t
 }
 
 // ts = amax / 2688, 1 for amax == 0, floored at 2^-117 (NaN stays NaN).
-__global__ void tensor_scale_kernel(const float *amax, float *ts)
+__device__ __forceinline__ float tensor_scale_of(float a)
 {
-    const float a = *amax;
     float t = 1.0f;
     if (a != 0.0f) {
         t = __fdiv_rn(a, 2688.0f);
         if (t < kTsFloor) t = kTsFloor;
     }
-    *ts = t;
+    return t;
+}
+
+__global__ void tensor_scale_kernel(const float *amax, float *ts)
+{
+    *ts = tensor_scale_of(*amax);
+}
+
+// ------------------------------------------- single-launch quantizer ----
+//
+// amax, tensor scale, IF4 quantize and (optionally) the NVFP4 comparator in
+// one cooperative launch: every block is resident, so the blocks can meet
+// at a grid barrier between the amax pass and the encode pass.  The encode
+// pass reads the tensor a second time; for tensors that fit in the 126 MB
+// L2 that read is served from L2.
+
+constexpr unsigned long long kGridWaitNs = 1000000000ull;   // 1 s
+
+// Grid barrier that also produces the tensor scale.  sync[0] counts
+// arrivals and sync[1] accumulates the float bits of the tensor amax (one
+// 128-byte line, written by the arriving blocks); sync[32] is the generation
+// and sync[33] carries ts to the other blocks (another line, polled by the
+// waiting blocks).  The last block to arrive computes ts, stores it to
+// *ts_out, puts sync[0] and sync[1] back to zero and moves the generation
+// on; the others wait (bounded) for the generation to move.  Called by one
+// thread per block.  Returns false (and sets IF4_DEV_TIMEOUT) when the wait
+// runs out.
+__device__ __noinline__ bool grid_tensor_scale(uint32_t *sync, uint32_t block_max_bits,
+                                               float *ts_out, int *err, float &ts)
+{
+    volatile uint32_t *vs = sync;
+    if (block_max_bits != 0u) atomicMax(&sync[1], block_max_bits);
+    const uint32_t gen = vs[32];
+    __threadfence();
+    const uint32_t arrived = atomicAdd(&sync[0], 1u);
+    if (arrived == gridDim.x - 1) {
+        __threadfence();
+        const float t = tensor_scale_of(__uint_as_float(atomicAdd(&sync[1], 0u)));
+        *ts_out = t;
+        vs[33] = __float_as_uint(t);
+        vs[1] = 0u;
+        vs[0] = 0u;
+        __threadfence();
+        atomicAdd(&sync[32], 1u);
+    } else {
+        const unsigned long long t0 = globaltimer_ns();
+        while (vs[32] == gen) {
+            if (globaltimer_ns() - t0 > kGridWaitNs) {
+                if (err) atomicOr(err, IF4_DEV_TIMEOUT);
+                return false;
+            }
+            __nanosleep(200);
+        }
+        __threadfence();
+    }
+    ts = __uint_as_float(vs[33]);
+    return true;
+}
+
+template <int DT, bool V8, bool RHT, bool NV>
+__global__ void __launch_bounds__(256, DT == DT_F32 ? 3 : 4)
+quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr,
+                      uint32_t ngroups, int contig, uint8_t *__restrict__ codes,
+                      uint8_t *__restrict__ scales, uint8_t *__restrict__ nv_codes,
+                      uint8_t *__restrict__ nv_scales, float *ts_out, uint32_t *sync, int *err,
+                      const __grid_constant__ SignMasks sm, uint32_t signs)
+{
+    constexpr int GB = 16 * elem_bytes<DT>();
+    __shared__ float inv_tab[128];
+    __shared__ uint32_t warp_max[8];
+    __shared__ float ts_sh;
+    __shared__ int ok_sh;
+    const uint32_t gpr_eff = contig ? ngroups : gpr;
+    auto addr = [&](uint32_t g) -> const char * {
+        return contig ? x + (int64_t)g * GB : group_addr<GB>(x, g, gpr, ld_bytes);
+    };
+    const uint32_t stride = gridDim.x * blockDim.x;
+    const uint32_t g_first = blockIdx.x * blockDim.x + threadIdx.x;
+
+    // pass 1: max |x| (of the transform, with RHT), six loads in flight
+    uint32_t m = 0;
+    constexpr int U = DT == DT_F32 ? 3 : 6;
+    for (uint64_t g0 = g_first; g0 < ngroups; g0 += (uint64_t)U * stride) {
+        Raw<DT> r[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint64_t g = g0 + (uint64_t)u * stride;
+            if (g < ngroups) load_group<DT, V8>(addr((uint32_t)g), r[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (g0 + (uint64_t)u * stride < ngroups) {
+                if constexpr (RHT) {
+                    f2_t xv[8];
+                    bool nf;
+                    m = max(m, __float_as_uint(unpack_group_rht<DT>(r[u], sm, xv, nf)));
+                } else {
+                    m = max(m, group_absmax_bits<DT>(r[u]));
+                }
+            }
+    }
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) warp_max[warp] = m;
+    // the encode pass's first group does not depend on ts: its load is in
+    // flight while the block waits at the grid barrier
+    Raw<DT> buf[2];
+    uint32_t g = g_first;
+    if (g < ngroups) load_group<DT, V8>(addr(g), buf[0]);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b = max(b, warp_max[w]);
+        if (b >= 0x7F800000u && err) atomicOr(err, IF4_DEV_NONFINITE);
+        float t = 1.0f;
+        ok_sh = grid_tensor_scale(sync, b, ts_out, err, t) ? 1 : 0;
+        ts_sh = t;
+    }
+    __syncthreads();
+    if (!ok_sh) return;
+
+    // pass 2: the encode, as quantize_kernel
+    const float ts = ts_sh;
+    if (threadIdx.x < 128) {
+        const float eff = __fmul_rn(f32_from_e4m3(threadIdx.x), ts);
+        inv_tab[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __frcp_rn(eff);
+    }
+    const float rts = __frcp_rn(ts);
+    __syncthreads();
+    for (; g < ngroups;) {
+#pragma unroll
+        for (int ph = 0; ph < 2; ++ph) {
+            const uint32_t gn = g + stride;
+            if (gn < ngroups) load_group<DT, V8>(addr(gn), buf[ph ^ 1]);
+            quantize_one<DT, Q_IF4, RHT, NV>(buf[ph], g, x, ld_bytes, gpr_eff, ts, rts, inv_tab,
+                                             nullptr, codes, scales, sm, signs, nv_codes,
+                                             nv_scales);
+            g = gn;
+            if (g >= ngroups) break;
+        }
+    }
 }
 
 // ------------------------------------------------ dequantize, fp16 decode --
@@ -1022,7 +1174,7 @@ __device__ __forceinline__ void decode_word(uint32_t w, uint32_t base, float (&q
 
 // Decode one group (code words w0, w1, scale byte sb) and store its 16
 // outputs at p.
-template <int ODT, bool UNIT_TS>
+template <int ODT, bool UNIT_TS, bool V8 = false>
 __device__ __forceinline__ void dequant_group(uint32_t w0, uint32_t w1, uint32_t sb, float ts,
                                               uint32_t lut_addr, char *p)
 {
@@ -1051,10 +1203,15 @@ __device__ __forceinline__ void dequant_group(uint32_t w0, uint32_t w1, uint32_t
             b[2 * j] = __float_as_uint(lo);
             b[2 * j + 1] = __float_as_uint(hi);
         }
-        st_v4(p, a[0], a[1], a[2], a[3]);
-        st_v4(p + 16, a[4], a[5], a[6], a[7]);
-        st_v4(p + 32, b[0], b[1], b[2], b[3]);
-        st_v4(p + 48, b[4], b[5], b[6], b[7]);
+        if constexpr (V8) {
+            st_v8(p, a);
+            st_v8(p + 32, b);
+        } else {
+            st_v4(p, a[0], a[1], a[2], a[3]);
+            st_v4(p + 16, a[4], a[5], a[6], a[7]);
+            st_v4(p + 32, b[0], b[1], b[2], b[3]);
+            st_v4(p + 48, b[4], b[5], b[6], b[7]);
+        }
     } else {
         uint32_t o[8];
 #pragma unroll
@@ -1065,8 +1222,14 @@ __device__ __forceinline__ void dequant_group(uint32_t w0, uint32_t w1, uint32_t
             f2_unpack(yb[j], lo, hi);
             o[4 + j] = pack_out2<ODT>(lo, hi);
         }
-        st_v4(p, o[0], o[1], o[2], o[3]);
-        st_v4(p + 16, o[4], o[5], o[6], o[7]);
+        // one 256-bit store fills a whole 32-byte sector; two 128-bit
+        // stores would each write half of every sector they touch
+        if constexpr (V8) {
+            st_v8(p, o);
+        } else {
+            st_v4(p, o[0], o[1], o[2], o[3]);
+            st_v4(p + 16, o[4], o[5], o[6], o[7]);
+        }
     }
 }
 
@@ -1074,7 +1237,7 @@ __device__ __forceinline__ void dequant_group(uint32_t w0, uint32_t w1, uint32_t
 // operand decode), else multiply by *ts.  One thread per group (lanes of a
 // warp own consecutive groups, so loads and stores are contiguous spans); the
 // next group's codes and scale are loaded before the current one is decoded.
-template <int ODT, bool UNIT_TS>
+template <int ODT, bool UNIT_TS, bool V8>
 __global__ void __launch_bounds__(256)
 dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
                   const float *__restrict__ ts_ptr, uint32_t gpr, uint32_t ngroups,
@@ -1100,7 +1263,7 @@ dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__
             ld_nc_v2(codes + (int64_t)gn * 8, b0, b1);
             bs = ld_nc_u8(scales + gn);
         }
-        dequant_group<ODT, UNIT_TS>(a0, a1, as, ts, lut_addr,
+        dequant_group<ODT, UNIT_TS, V8>(a0, a1, as, ts, lut_addr,
                                     const_cast<char *>(group_ptr(y, g, contig, gpr, ld_bytes, 16 * OB)));
         if (!more) break;
         g = gn;
@@ -1110,7 +1273,7 @@ dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__
             ld_nc_v2(codes + (int64_t)gn * 8, a0, a1);
             as = ld_nc_u8(scales + gn);
         }
-        dequant_group<ODT, UNIT_TS>(b0, b1, bs, ts, lut_addr,
+        dequant_group<ODT, UNIT_TS, V8>(b0, b1, bs, ts, lut_addr,
                                     const_cast<char *>(group_ptr(y, g, contig, gpr, ld_bytes, 16 * OB)));
         if (!more) break;
         g = gn;
@@ -1349,16 +1512,66 @@ int quantize_entry(const void *x, int x_dtype, int64_t rows, int64_t cols, int64
                                      ts_mode == IF4_TS_GIVEN ? 1 : 0, st, d, signs);
 }
 
+// Single-launch quantizer: a cooperative launch of at most one wave, so
+// every block is resident when the blocks meet at the grid barrier.
+template <int DT, bool V8, bool RHT, bool NV>
+int launch_fused(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
+                 uint8_t *nv_codes, uint8_t *nv_scales, float *ts, uint32_t *sync, int *err,
+                 cudaStream_t st, const DeviceInfo &d, const SignMasks &sm, uint32_t signs)
+{
+    auto k = quantize_fused_kernel<DT, V8, RHT, NV>;
+    static const int occ = resident_blocks(k, 256);
+    const uint32_t grid = grid_for(occ, d, s.ngroups, 256);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k, static_cast<const char *>(x), s.ld_bytes, s.gpr, s.ngroups,
+                           s.contig ? 1 : 0, codes, scales, nv_codes, nv_scales, ts, sync, err, sm,
+                           signs) != cudaSuccess)
+        return IF4_ERR_CUDA;
+    return launch_status();
+}
+
+template <int DT, bool RHT>
+int dispatch_fused_dt(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
+                      uint8_t *nv_codes, uint8_t *nv_scales, float *ts, uint32_t *sync, int *err,
+                      cudaStream_t st, const DeviceInfo &d, const SignMasks &sm, uint32_t signs)
+{
+    const bool nv = nv_codes != nullptr;
+    if (s.v8)
+        return nv ? launch_fused<DT, true, RHT, true>(s, x, codes, scales, nv_codes, nv_scales, ts,
+                                                      sync, err, st, d, sm, signs)
+                  : launch_fused<DT, true, RHT, false>(s, x, codes, scales, nv_codes, nv_scales,
+                                                       ts, sync, err, st, d, sm, signs);
+    return nv ? launch_fused<DT, false, RHT, true>(s, x, codes, scales, nv_codes, nv_scales, ts,
+                                                   sync, err, st, d, sm, signs)
+              : launch_fused<DT, false, RHT, false>(s, x, codes, scales, nv_codes, nv_scales, ts,
+                                                    sync, err, st, d, sm, signs);
+}
+
 template <int ODT, bool UNIT_TS>
 int launch_dequant(const Shape &s, const uint8_t *codes, const uint8_t *scales, const float *ts,
                    void *y, cudaStream_t st, const DeviceInfo &d)
 {
     if (s.ngroups == 0) return IF4_OK;
-    auto k = dequantize_kernel<ODT, UNIT_TS>;
-    static const int occ = resident_blocks(k, 256);
-    const uint32_t grid = grid_for(occ, d, s.ngroups, 256);
-    k<<<grid, 256, 0, st>>>(codes, scales, ts, s.gpr, s.ngroups, static_cast<char *>(y),
-                            s.ld_bytes, s.contig ? 1 : 0);
+    auto launch = [&](auto k) {
+        static const int occ = resident_blocks(k, 256);
+        const uint32_t grid = grid_for(occ, d, s.ngroups, 256);
+        k<<<grid, 256, 0, st>>>(codes, scales, ts, s.gpr, s.ngroups, static_cast<char *>(y),
+                                s.ld_bytes, s.contig ? 1 : 0);
+    };
+    // 32-byte aligned base and rows: 256-bit stores
+    if (s.v8)
+        launch(dequantize_kernel<ODT, UNIT_TS, true>);
+    else
+        launch(dequantize_kernel<ODT, UNIT_TS, false>);
     return launch_status();
 }
 
@@ -1454,6 +1667,44 @@ int if4_quantize_rht(const void *x, int x_dtype, int64_t rows, int64_t cols, int
 {
     return quantize_entry<Q_IF4, true>(x, x_dtype, rows, cols, ld_x, codes, scales, ts, ts_mode,
                                        err_flag, stream, signs & 0xFFFFu);
+}
+
+int if4_quantize_fused(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                       uint8_t *codes, uint8_t *scales, uint8_t *nv_codes, uint8_t *nv_scales,
+                       float *ts, uint32_t *sync_words, int *err_flag, void *stream)
+{
+    Shape s;
+    int rc = check_tensor(x, x_dtype, rows, cols, ld_x, s);
+    if (rc != IF4_OK) return rc;
+    if (ts == nullptr || sync_words == nullptr) return IF4_ERR_NULL;
+    if ((nv_codes == nullptr) != (nv_scales == nullptr)) return IF4_ERR_NULL;
+    if (s.ngroups > 0 && (codes == nullptr || scales == nullptr)) return IF4_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(codes) % 16 != 0 ||
+        reinterpret_cast<uintptr_t>(nv_codes) % 16 != 0 ||
+        reinterpret_cast<uintptr_t>(ts) % 4 != 0 || reinterpret_cast<uintptr_t>(sync_words) % 256 != 0)
+        return IF4_ERR_ALIGN;
+    DeviceInfo d;
+    rc = check_device(d);
+    if (rc != IF4_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (s.ngroups == 0) {
+        // an empty tensor: amax 0, ts 1, nothing to encode
+        if (cudaMemsetAsync(ts, 0, sizeof(float), st) != cudaSuccess) return IF4_ERR_CUDA;
+        tensor_scale_kernel<<<1, 1, 0, st>>>(ts, ts);
+        return launch_status();
+    }
+    const SignMasks sm = sign_masks(x_dtype, 0);
+    switch (x_dtype) {
+    case IF4_F32:
+        return dispatch_fused_dt<DT_F32, false>(s, x, codes, scales, nv_codes, nv_scales, ts,
+                                                sync_words, err_flag, st, d, sm, 0);
+    case IF4_BF16:
+        return dispatch_fused_dt<DT_BF16, false>(s, x, codes, scales, nv_codes, nv_scales, ts,
+                                                 sync_words, err_flag, st, d, sm, 0);
+    default:
+        return dispatch_fused_dt<DT_F16, false>(s, x, codes, scales, nv_codes, nv_scales, ts,
+                                                sync_words, err_flag, st, d, sm, 0);
+    }
 }
 
 int if4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts, int64_t rows,

@@ -53,7 +53,7 @@ def parse():
     p.add_argument("--kernel-only", default=None,
                    choices=["amax", "if4_quantize", "if4_dequantize", "nvfp4_quantize", "gemm",
                             "nvint4_quantize", "nvfp4_4over6_quantize", "if4_quantize_rht",
-                            "if4_decode_f16"],
+                            "if4_decode_f16", "fused_quantize"],
                    help="launch only this kernel, warmup+steps times (for ncu captures)")
     return p.parse_args()
 
@@ -274,11 +274,13 @@ class Step:
                 y=torch.empty((self.rows, self.cols), dtype=torch.bfloat16, device=dev),
                 ncodes=torch.empty((self.rows, self.cols // 2), dtype=torch.uint8, device=dev),
                 nscales=torch.empty((self.rows, self.cols // 16), dtype=torch.uint8, device=dev),
+                sync=torch.zeros(64, dtype=torch.int32, device=dev),
             )
             self.sets.append(s)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.kernels = ["amax", "scale", "if4_quantize", "if4_dequantize", "nvfp4_quantize"]
-        self.launches_per_step = 5
+        self.kernels = ["fused_quantize", "amax", "scale", "if4_quantize", "if4_dequantize",
+                        "nvfp4_quantize"]
+        self.launches_per_step = 2
 
     def bytes_per_set(self):
         s = self.sets[0]
@@ -301,7 +303,10 @@ class Step:
         if name == "if4_decode_f16":
             b.if4_decode_f16(s["codes"], s["scales"], s["y"].view(torch.float16))
             return
-        if name == "amax":
+        if name == "fused_quantize":
+            b.if4_quantize_fused(s["x"], s["codes"], s["scales"], s["ncodes"], s["nscales"],
+                                 s["ts"], s["sync"], self.err)
+        elif name == "amax":
             b.if4_tensor_amax(s["x"], s["amax"], self.err)
         elif name == "scale":
             b.if4_tensor_scale(s["amax"], s["ts"])
@@ -314,8 +319,17 @@ class Step:
         else:
             raise ValueError(name)
 
-    def run(self, i, events=None, side=None):
-        """One step on buffer set i.  With a side stream, the NVFP4 quantizer
+    def run(self, i):
+        """One step on buffer set i: the single-launch quantizer (tensor amax,
+        tensor scale, IF4 codes and the NVFP4 comparator), then the IF4
+        dequantizer to bf16."""
+        b, s = self.b, self.sets[i % len(self.sets)]
+        b.if4_quantize_fused(s["x"], s["codes"], s["scales"], s["ncodes"], s["nscales"], s["ts"],
+                             s["sync"], self.err)
+        b.if4_dequantize(s["codes"], s["scales"], s["ts"], s["y"])
+
+    def run_unfused(self, i, events=None, side=None):
+        """The same step as five launches.  With a side stream, the NVFP4 quantizer
         (which needs only ts) runs on it beside IF4 quantize -> dequantize:
         the two quantizers read the same input at about the same time."""
         b, s = self.b, self.sets[i % len(self.sets)]
@@ -373,7 +387,10 @@ def kernel_times(step, names, reps):
 def kernel_table(ms, n_elem, in_bytes, pk):
     q_bytes = in_bytes + n_elem // 2 + n_elem // 16
     dq_bytes = n_elem // 2 + n_elem // 16 + 2 * n_elem
-    nbytes = {"amax": in_bytes, "scale": 8, "if4_quantize": q_bytes, "if4_dequantize": dq_bytes,
+    # the single-launch quantizer: x once, IF4 and NVFP4 codes and scales
+    fused_bytes = in_bytes + 2 * (n_elem // 2 + n_elem // 16)
+    nbytes = {"fused_quantize": fused_bytes, "amax": in_bytes, "scale": 8,
+              "if4_quantize": q_bytes, "if4_dequantize": dq_bytes,
               "nvfp4_quantize": q_bytes, "nvint4_quantize": q_bytes,
               "nvfp4_4over6_quantize": q_bytes, "if4_quantize_rht": q_bytes,
               "if4_decode_f16": dq_bytes}
@@ -426,7 +443,7 @@ def quality_report(x_cpu, step):
 
 def measure_e2e(x_cpu, steps, warmup):
     """The same step through the C ABI from pinned host memory: per step, the
-    H2D copy of the input, the five kernels, and the D2H copy of every result
+    H2D copy of the input, the two launches, and the D2H copy of every result
     (IF4 codes, scales and tensor scale, the bf16 dequantized tensor, NVFP4
     codes and scales), all inside the timed region.  Consecutive steps
     alternate between two streams with their own buffers, so one step's
@@ -443,7 +460,7 @@ def measure_e2e(x_cpu, steps, warmup):
         lanes.append(dict(
             stream=torch.cuda.Stream(),
             x=torch.empty_like(h_x, device=dev),
-            amax=torch.empty(1, dtype=torch.float32, device=dev),
+            sync=torch.zeros(64, dtype=torch.int32, device=dev),
             d={k: torch.empty(sh, dtype=dt, device=dev) for k, (sh, dt) in outs.items()},
             h={k: torch.empty(sh, dtype=dt, pin_memory=True) for k, (sh, dt) in outs.items()}))
     err = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -453,11 +470,9 @@ def measure_e2e(x_cpu, steps, warmup):
         with torch.cuda.stream(L["stream"]):
             d = L["d"]
             L["x"].copy_(h_x, non_blocking=True)
-            b.if4_tensor_amax(L["x"], L["amax"], err)
-            b.if4_tensor_scale(L["amax"], d["ts"])
-            b.if4_quantize(L["x"], d["codes"], d["scales"], d["ts"], b.TS_GIVEN, err)
+            b.if4_quantize_fused(L["x"], d["codes"], d["scales"], d["ncodes"], d["nscales"],
+                                 d["ts"], L["sync"], err)
             b.if4_dequantize(d["codes"], d["scales"], d["ts"], d["y"])
-            b.nvfp4_quantize(L["x"], d["ncodes"], d["nscales"], d["ts"], b.TS_GIVEN, err)
             for k in L["h"]:
                 L["h"][k].copy_(d[k], non_blocking=True)
 
@@ -563,18 +578,20 @@ def run_ours(args):
     if int(step.err.item()) != 0:
         raise RuntimeError(f"device error flag {int(step.err.item())} during warm-up")
 
-    # One CUDA graph per buffer set holds a whole step (5 kernels and the
-    # memset that zeroes amax), so host launch overhead does not pace the GPU;
-    # the NVFP4 comparator is a parallel branch of the graph.
-    graphs = []
-    side = torch.cuda.Stream()
-    for i in range(sets):
+    # The timed steps are captured as one CUDA graph (each step on the next
+    # buffer set in turn), so neither host launch overhead nor the gaps
+    # between graph launches pace the GPU; the warm-up steps are a graph of
+    # their own, replayed first.
+    def capture(fn, n, **kw):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            step.run(i, side=side)
-        graphs.append(g)
-    for i in range(max(args.warmup, sets)):
-        graphs[i % sets].replay()
+            for i in range(n):
+                fn(i, **kw)
+        return g
+
+    warm = capture(step.run, max(args.warmup, sets))
+    timed = capture(step.run, args.steps)
+    warm.replay()
     torch.cuda.synchronize()
 
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -582,18 +599,32 @@ def run_ours(args):
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         start.record()
-        for i in range(args.steps):
-            graphs[i % sets].replay()
+        timed.replay()
         stop.record()
         torch.cuda.synchronize()
     barrier(world)
     ms_local = start.elapsed_time(stop) / args.steps
     ms = max_over_ranks(ms_local, world)
+    del warm
+
+    # the same step as five launches (NVFP4 on a parallel graph branch), for
+    # comparison
+    side = torch.cuda.Stream()
+    uwarm = capture(step.run_unfused, sets, side=side)
+    utimed = capture(step.run_unfused, args.steps, side=side)
+    uwarm.replay()
+    torch.cuda.synchronize()
+    start.record()
+    utimed.replay()
+    stop.record()
+    torch.cuda.synchronize()
+    ms_unfused = start.elapsed_time(stop) / args.steps
+    del uwarm, utimed
 
     kern_ms = kernel_times(step, step.kernels, max(2, args.steps // sets))
     if int(step.err.item()) != 0:
         raise RuntimeError(f"device error flag {int(step.err.item())}")
-    graphs_keep = graphs
+    graphs_keep = timed
 
     value = world * n_elem / (ms * 1e-3) / 1e9
     q_bytes = in_bytes + n_elem // 2 + n_elem // 16
@@ -601,18 +632,23 @@ def run_ours(args):
     extra = kernel_table(kernel_times(step, Step.EXTRA, max(2, args.steps // sets)), n_elem,
                          in_bytes, pk)
 
-    top = kernels["if4_quantize"]
-    roofline = {"bound": "hbm", "kernel": "if4_quantize (tensor scale given)",
-                "achieved": top["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": top["gbs"] / pk["hbm_gbs"],
-                "peak_source": f"{pk['source']} hbm_gbs (copy bandwidth, read+write)",
-                "algorithmic_bytes_per_launch": q_bytes,
-                "traffic": None}
-    traffic_file = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(traffic_file):
-        tr = json.load(open(traffic_file)).get(args.workload, {}).get("if4_quantize")
-        if tr:
-            roofline["traffic"] = tr
+    def roof(name, label):
+        k = kernels[name]
+        r = {"bound": "hbm", "kernel": label, "achieved": k["gbs"], "peak": pk["hbm_gbs"],
+             "unit": "GB/s", "frac": k["gbs"] / pk["hbm_gbs"],
+             "peak_source": f"{pk['source']} hbm_gbs (copy bandwidth, read+write; of measured)",
+             "algorithmic_bytes_per_launch": k["bytes"], "traffic": None}
+        traffic_file = os.path.join(ROOT, "profiles", "traffic.json")
+        if os.path.exists(traffic_file):
+            tr = json.load(open(traffic_file)).get(args.workload, {}).get(name)
+            if tr:
+                r["traffic"] = tr
+        return r
+
+    # the dominant kernel of the step is the single-launch quantizer; the
+    # IF4 quantizer alone (tensor scale given) is reported beside it
+    roofline = roof("fused_quantize", "if4_quantize_fused (amax + scale + IF4 + NVFP4)")
+    roofline_if4 = roof("if4_quantize", "if4_quantize (tensor scale given)")
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -623,12 +659,14 @@ def run_ours(args):
                        "group": 16, "parallelism": f"independent tensors x{world}",
                        "l2": f"rotating {sets} buffer sets, {sets * per_set / 1e6:.0f} MB "
                              f"(inputs {sets * in_bytes / 1e6:.0f} MB > 3x126 MB L2)",
-                       "launch": "one CUDA graph per step (NVFP4 on a parallel branch after "
-                                 "the tensor scale); per-kernel times from one graph per "
-                                 "kernel over all sets",
-                       "step": "amax, scale, IF4 quantize, IF4 dequantize (bf16), NVFP4 quantize"},
+                       "launch": "the timed steps as one CUDA graph; per-kernel times from "
+                                 "one graph per kernel over all sets",
+                       "step": "single-launch quantizer (amax, scale, IF4 quantize, NVFP4 "
+                               "quantize), then IF4 dequantize (bf16)"},
             "gpu_launches": step.launches_per_step * args.steps,
-            "kernels": kernels, "kernels_outside_step": extra, "roofline": roofline}
+            "ms_per_step_unfused": ms_unfused,
+            "kernels": kernels, "kernels_outside_step": extra, "roofline": roofline,
+            "roofline_if4_quantize": roofline_if4}
     if rank == 0:
         line["clocks"] = clk.summary()
         line["quality"] = quality_report(x_cpu, step)
@@ -674,7 +712,8 @@ def run_kernel_only(args):
     b.if4_tensor_scale(s["amax"], s["ts"])
     b.if4_quantize(s["x"], s["codes"], s["scales"], s["ts"], b.TS_GIVEN, step.err)
     torch.cuda.synchronize()
-    calls = {name: (lambda name=name: step.run_one(name, 0)) for name in Step.EXTRA}
+    calls = {name: (lambda name=name: step.run_one(name, 0))
+             for name in Step.EXTRA + ["fused_quantize"]}
     calls.update({
         "amax": lambda: b.if4_tensor_amax(s["x"], s["amax"], step.err),
         "if4_quantize": lambda: b.if4_quantize(s["x"], s["codes"], s["scales"], s["ts"],

@@ -146,6 +146,33 @@ int if4_quantize_rht(const void *x, int x_dtype, int64_t rows, int64_t cols, int
                      int *err_flag, void *stream);
 
 /*
+ * Single-launch quantizer: tensor amax, tensor scale and IF4 quantize (as
+ * if4_quantize with IF4_TS_COMPUTE), plus, when nv_codes / nv_scales are
+ * given, the NVFP4 comparator of nvfp4_quantize under the same tensor scale,
+ * all in one cooperative kernel launch that reads x for the amax and again
+ * for the encode.  Results are byte-identical to those calls.
+ *
+ * sync_words: 64 uint32 (256 bytes) of device memory, 256-byte aligned,
+ * owned by the caller, all zero before the first call.  Word 0 counts
+ * arrivals at the grid barrier and word 1 accumulates the amax; every call
+ * that completes leaves both at zero.  Word 32 counts barrier generations
+ * and word 33 keeps the last ts; they may hold any value.  The rest is
+ * unused.  So one allocation serves any number
+ * of calls that run one after another; calls that may run at the same time
+ * (other streams) need their own.  After a call that set IF4_DEV_TIMEOUT (a
+ * block waited more than 1 s at the grid barrier; no codes were written)
+ * the words must be zeroed again.
+ *
+ * nv_codes / nv_scales: both NULL (IF4 only) or both given.  err_flag may be
+ * NULL; IF4_DEV_NONFINITE and IF4_DEV_TIMEOUT are reported there.  Other
+ * rules as if4_quantize.  The pages have no counterpart: this is a fusion of
+ * the steps above.
+ */
+int if4_quantize_fused(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                       uint8_t *codes, uint8_t *scales, uint8_t *nv_codes, uint8_t *nv_scales,
+                       float *ts, uint32_t *sync_words, int *err_flag, void *stream);
+
+/*
  * Comparator, all-INT4 ("NVINT4"): the 7/6-scaled INT4 candidate of
  * if4_quantize for every group, bit 7 set wherever the block scale is
  * nonzero (gist.science section 3, item 2, and section 4: IF4 is compared with
@@ -217,6 +244,8 @@ int if4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_t
                void *c, int *err_flag, void *stream);
 
 /* Size of the scratch array behind if4_linear_noalloc (32 MiB per device). */
+#define IF4_FUSED_SYNC_WORDS 64u
+
 #define IF4_LINEAR_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
 
 /*

@@ -25,6 +25,7 @@ def lib():
     L.if4_tensor_amax.argtypes = [vp, i, i64, i64, i64, vp, vp, vp]
     L.if4_tensor_scale.argtypes = [vp, vp, vp]
     L.if4_decode_f16.argtypes = [vp, vp, i64, i64, vp, vp]
+    L.if4_quantize_fused.argtypes = [vp, i, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp]
     L.if4_status_str.restype = ctypes.c_char_p
     return L
 
@@ -90,6 +91,25 @@ def test_quantize_host_validation(lib, fn):
     assert f(A, 1, 4, 32, 36, A, A, A, 0, None, None) == 4
     assert f(A, 1, 4, 32, 32, A + 8, A, A, 0, None, None) == 4
     assert f(A, 1, 4, 32, 32, A, A, A + 2, 0, None, None) == 4
+
+
+def test_fused_quantize_host_validation(lib):
+    f = lib.if4_quantize_fused
+    # null x / codes / ts / sync words, half of the NVFP4 pair
+    assert f(None, 1, 4, 32, 32, A, A, None, None, A, A, None, None) == 1
+    assert f(A, 1, 4, 32, 32, None, A, None, None, A, A, None, None) == 1
+    assert f(A, 1, 4, 32, 32, A, A, None, None, None, A, None, None) == 1
+    assert f(A, 1, 4, 32, 32, A, A, None, None, A, None, None, None) == 1
+    assert f(A, 1, 4, 32, 32, A, A, A, None, A, A, None, None) == 1
+    # shape, dtype, alignment of x, codes, nv_codes, ts, sync words
+    assert f(A, 1, 4, 24, 24, A, A, None, None, A, A, None, None) == 2
+    assert f(A, 9, 4, 32, 32, A, A, None, None, A, A, None, None) == 3
+    assert f(A + 8, 1, 4, 32, 32, A, A, None, None, A, A, None, None) == 4
+    assert f(A, 1, 4, 32, 32, A + 8, A, None, None, A, A, None, None) == 4
+    assert f(A, 1, 4, 32, 32, A, A, A + 8, A, A, A, None, None) == 4
+    assert f(A, 1, 4, 32, 32, A, A, None, None, A + 2, A, None, None) == 4
+    assert f(A, 1, 4, 32, 32, A, A, None, None, A, A + 4, None, None) == 4
+    assert f(A, 1, 4, 32, 32, A, A, None, None, A, A + 128, None, None) == 4
 
 
 def test_dequantize_and_decode_host_validation(lib):

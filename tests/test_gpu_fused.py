@@ -1,0 +1,116 @@
+"""GPU parity of the single-launch quantizer (if4_quantize_fused): tensor
+amax, tensor scale, IF4 codes and the NVFP4 comparator from one cooperative
+launch must equal the oracle byte for byte, and equal the separate calls.
+Words 0 (arrivals) and 1 (amax) of the synchronisation words must come back
+zero after every call; word 32 counts barrier generations, word 33 keeps ts."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from adaptive_block_scaled_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def B():
+    from adaptive_block_scaled_b200 import binding
+    return binding
+
+
+def fused(x_dev, sync=None, with_nvfp4=True):
+    b = B()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if sync is None:
+        sync = torch.zeros(b.FUSED_SYNC_WORDS, dtype=torch.int32, device="cuda")
+    out = b.quantize_fused(x_dev, with_nvfp4=with_nvfp4, sync_words=sync, err_flag=err)
+    torch.cuda.synchronize()
+    w = sync.tolist()
+    assert w[0] == 0 and w[1] == 0, w[:2]
+    return [o.cpu().numpy() for o in out], int(err.item())
+
+
+def check(x_cpu, label, x_dev=None):
+    x_np = x_cpu.float().numpy()
+    ref = oracle.quantize_tensor(x_np)
+    nv = oracle.quantize(x_np, ref["ts"], mode=oracle.MODE_NVFP4)
+    (codes, scales, ts, ncodes, nscales), err = fused(x_cpu.cuda() if x_dev is None else x_dev)
+    assert err == 0
+    assert np.float32(ts[0]).view(np.uint32) == np.float32(ref["ts"]).view(np.uint32), label
+    assert np.array_equal(scales, ref["scales"]), label
+    assert np.array_equal(codes, ref["codes"]), label
+    assert np.array_equal(nscales, nv["scales"]), label
+    assert np.array_equal(ncodes, nv["codes"]), label
+    print(f"[fused {label}] groups={scales.size} ok")
+
+
+def test_fused_on_small_and_weight_workloads():
+    check(workloads.small_fp32(0), "small_fp32_256x1024")
+    check(workloads.llm_weight(0), "weight_bf16_4096x4096")
+
+
+def test_fused_on_activation_and_gradient_like_rows():
+    check(workloads.activation_outliers(0, tokens=1024, hidden=8192), "activation rows")
+    check(workloads.hadamard_gradient(0, rows=1024, cols=4096), "gradient rows")
+
+
+@pytest.mark.parametrize("shape", [(1, 16), (7, 80), (33, 272), (1000, 16), (300, 4096)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+def test_fused_ragged_shapes_and_dtypes(shape, dtype):
+    g = torch.Generator().manual_seed(shape[0] * 31 + shape[1])
+    x = (torch.randn(shape, generator=g) * 5).to(dtype)
+    check(x, f"{shape} {dtype}")
+
+
+def test_fused_tiny_groups_and_zeros():
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((64, 256)).astype(np.float32)
+    x *= np.exp2(-rng.integers(0, 24, (64, 16))).repeat(16, axis=1).astype(np.float32)
+    x[0, 0] = 1000.0
+    x[1, :16] = -0.0
+    x[3] = 0.0
+    check(torch.from_numpy(x), "tiny groups")
+
+
+def test_fused_all_zero_and_empty():
+    (codes, scales, ts, nc, ns), err = fused(torch.zeros((5, 64), dtype=torch.bfloat16,
+                                                         device="cuda"))
+    assert err == 0 and ts[0] == 1.0 and not codes.any() and not scales.any() and not nc.any()
+    (codes, scales, ts, nc, ns), err = fused(torch.zeros((0, 64), dtype=torch.bfloat16,
+                                                         device="cuda"))
+    assert err == 0 and ts[0] == 1.0 and codes.shape == (0, 32)
+
+
+def test_fused_strided_rows_and_unaligned_base():
+    base = workloads.llm_weight(1, rows=256, cols=1024 + 64)
+    x_dev = base.cuda()[:, 8:8 + 1024]
+    assert x_dev.data_ptr() % 32 == 16
+    check(base[:, 8:8 + 1024].contiguous(), "strided", x_dev=x_dev)
+
+
+def test_fused_equals_separate_calls_and_reuses_sync_words():
+    b = B()
+    sync = torch.zeros(b.FUSED_SYNC_WORDS, dtype=torch.int32, device="cuda")
+    for seed in range(3):
+        x = workloads.llm_weight(seed, rows=512, cols=2048).cuda()
+        (codes, scales, ts, nc, ns), err = fused(x, sync=sync)
+        c2, s2, t2 = b.quantize(x)
+        n2, m2, _ = b.quantize(x, "nvfp4", ts=t2)
+        torch.cuda.synchronize()
+        assert err == 0 and ts[0] == t2.item()
+        assert np.array_equal(codes, c2.cpu().numpy()) and np.array_equal(scales, s2.cpu().numpy())
+        assert np.array_equal(nc, n2.cpu().numpy()) and np.array_equal(ns, m2.cpu().numpy())
+
+
+def test_fused_if4_only():
+    x = workloads.llm_weight(5, rows=128, cols=1024)
+    ref = oracle.quantize_tensor(x.float().numpy())
+    (codes, scales, ts), err = fused(x.cuda(), with_nvfp4=False)
+    assert err == 0 and np.array_equal(codes, ref["codes"]) and np.array_equal(scales, ref["scales"])
+
+
+def test_fused_nonfinite_sets_flag_and_leaves_sync_zero():
+    x = torch.randn(64, 256).to(torch.bfloat16)
+    x[7, 9] = float("inf")
+    _, err = fused(x.cuda())
+    assert err & B().DEV_NONFINITE
