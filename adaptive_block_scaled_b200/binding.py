@@ -60,6 +60,8 @@ def _load():
         "if4_linear": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_size_t,
                        _vp, _vp, _vp],
         "if4_linear_noalloc": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
+        "if4_linear_quantized": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
+                                 ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp, _vp],
         "if4_status_str": [_int],
         "if4_version": [],
     }
@@ -252,6 +254,25 @@ def if4_linear_noalloc(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, c, err_
     _check(lib.if4_linear_noalloc(_ptr(a_codes), _ptr(a_scales), _ptr(a_ts), _ptr(b_codes),
                                   _ptr(b_scales), _ptr(b_ts), M, N, K, _ptr(c),
                                   _ptr(err_flag), _stream(stream)), "if4_linear_noalloc")
+
+
+def if4_linear_quantized(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, workspace, c_codes,
+                         c_scales, c_ts, c=None, err_flag=None, stream=None):
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = b_codes.shape[0]
+    _u8(a_codes, "a_codes", (M, K // 2))
+    _u8(a_scales, "a_scales", (M, K // 16))
+    _u8(b_codes, "b_codes", (N, K // 2))
+    _u8(b_scales, "b_scales", (N, K // 16))
+    _u8(c_codes, "c_codes", (M, N // 2))
+    _u8(c_scales, "c_scales", (M, N // 16))
+    if c is not None and (c.dtype != torch.bfloat16 or not c.is_contiguous()):
+        raise ValueError("c must be a contiguous bf16 tensor")
+    _check(lib.if4_linear_quantized(_ptr(a_codes), _ptr(a_scales), _ptr(a_ts), _ptr(b_codes),
+                                    _ptr(b_scales), _ptr(b_ts), M, N, K, _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _ptr(c),
+                                    _ptr(c_codes), _ptr(c_scales), _ptr(c_ts), _ptr(err_flag),
+                                    _stream(stream)), "if4_linear_quantized")
 
 
 LINEAR_NOALLOC_MAX_BYTES = 32 * 1024 * 1024

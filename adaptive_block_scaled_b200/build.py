@@ -25,10 +25,10 @@ COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler",
 # the arithmetic contract's back, so that file is built with -fmad=false.
 SOURCES = [
     ("if4_quant.cu", ["-fmad=false"]),
-    ("if4_linear.cu", []),
+    ("if4_linear.cu", ["-fmad=false"]),   # shares the IF4 encoder (no contraction)
     ("if4_linear_noalloc.cu", []),
 ]
-HEADERS = ["if4_device.cuh", "exports.map"]
+HEADERS = ["if4_device.cuh", "if4_encode.cuh", "exports.map"]
 
 
 def _nvcc():

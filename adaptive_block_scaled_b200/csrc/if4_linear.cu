@@ -32,6 +32,7 @@
 #include <mutex>
 
 #include "../../include/if4.h"
+#include "if4_encode.cuh"
 
 namespace {
 
@@ -46,7 +47,8 @@ constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int TMEM_COLS = 2 * BN;            // two accumulators
 constexpr int NUM_THREADS = 192;             // 6 warps
 constexpr int EPI_WARP0 = 2;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
+                           512 /*inverse block scales of the IF4 output*/;
 constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;   // 1 s per wait
 
 // instruction descriptor, kind::f16: D f32, A f16, B f16, both K-major,
@@ -196,10 +198,91 @@ __device__ __forceinline__ uint32_t bf16x2(float lo, float hi)
     return r;
 }
 
-__device__ __forceinline__ void st_v4(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+
+// ------------------------------------------------- IF4 output epilogue ----
+//
+// With the IF4 output, each epilogue thread holds one row of a 32-column
+// chunk of C, i.e. two whole groups of 16 along N, the contiguous dimension.
+// It rounds them to bf16 (the values a separate if4_quantize of the bf16 C
+// would read) and encodes them with the quantizer's own group encoder under
+// the given tensor scale, so the codes equal those of that separate call.
+
+struct OutQ {
+    uint8_t *codes;         // [M, N/2]
+    uint8_t *scales;        // [M, N/16]
+    float ts, rts;          // tensor scale of C and its reciprocal
+    const float *inv_tab;   // fl(1 / fl(E4M3(c) * ts)), shared memory
+};
+
+// Inverse block-scale table of the IF4 output and the check of its tensor
+// scale, by threads 0..127 of a CTA.
+__device__ __forceinline__ void out_inv_table(float *inv_tab, const float *c_ts, int *err)
 {
-    asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" :: "l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
-                 : "memory");
+    if (threadIdx.x < 128) {
+        const float ts = *c_ts;
+        const float eff = __fmul_rn(f32_from_e4m3(threadIdx.x), ts);
+        inv_tab[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __frcp_rn(eff);
+        if (threadIdx.x == 0 && blockIdx.x == 0 && !(ts >= 0x1p-117f && ts <= 0x1p117f) && err)
+            atomicOr(err, IF4_DEV_BAD_SCALE);
+    }
+}
+
+// One output group of 16 bf16 values (8 words, element 2j in the low half of
+// word j): IF4 codes and scale byte to codes_p / scale_p.  True on Inf/NaN.
+__device__ __forceinline__ bool quantize_out_group(const uint32_t *w, const OutQ &oq,
+                                                   uint8_t *codes_p, uint8_t *scale_p)
+{
+    uint32_t m = 0;
+    f2_t xv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        m = absmax_bf16x2(m, w[j]);
+        xv[j] = f2_from_bf16x2(w[j]);
+    }
+    const uint32_t m16 = max(m & 0x7FFFu, (m >> 16) & 0x7FFFu);
+    const float amax = __uint_as_float(m16 << 16);
+    const If4Fast f = if4_fast(xv, amax, oq.ts, oq.rts, oq.inv_tab);
+    const GroupCode out = if4_finish(f, amax, oq.ts, oq.rts, oq.inv_tab, [&](float (&y)[16]) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f2_unpack(xv[j], y[2 * j], y[2 * j + 1]);
+    });
+    st_v2(codes_p, out.c0, out.c1);
+    st_u8(scale_p, out.scale);
+    return m16 >= 0x7F80u;
+}
+
+// Store one row's 32-column chunk (raw fp32 accumulators r, scaled by
+// `scale`): bf16 to C when c is given, IF4 when QOUT.  True on Inf/NaN.
+template <bool QOUT>
+__device__ __forceinline__ bool store_chunk(const uint32_t (&r)[32], float scale, int row, int M,
+                                            int N, int col0, __nv_bfloat16 *c, const OutQ &oq)
+{
+    if (row >= M) return false;
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        w[i] = bf16x2(__fmul_rn(__uint_as_float(r[2 * i]), scale),
+                      __fmul_rn(__uint_as_float(r[2 * i + 1]), scale));
+    if (c != nullptr) {
+        __nv_bfloat16 *crow = c + (int64_t)row * N;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            if (col0 + q * 8 < N)
+                st_v4(crow + col0 + q * 8, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    }
+    bool nonfinite = false;
+    if constexpr (QOUT) {
+        const int64_t gpr = N / 16;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int col = col0 + 16 * h;
+            if (col < N) {
+                const int64_t gi = (int64_t)row * gpr + col / 16;
+                nonfinite |= quantize_out_group(w + 8 * h, oq, oq.codes + gi * 8, oq.scales + gi);
+            }
+        }
+    }
+    return nonfinite;
 }
 
 // ------------------------------------------------------------- kernel ----
@@ -215,11 +298,14 @@ struct TileIter {
     }
 };
 
+template <bool QOUT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_f16_tcgen05(const __grid_constant__ CUtensorMap tmap_a,
                  const __grid_constant__ CUtensorMap tmap_b,
                  const float *__restrict__ a_ts, const float *__restrict__ b_ts,
-                 __nv_bfloat16 *__restrict__ c, int M, int N, int K, int *err)
+                 __nv_bfloat16 *__restrict__ c, int M, int N, int K, int *err,
+                 uint8_t *__restrict__ c_codes, uint8_t *__restrict__ c_scales,
+                 const float *__restrict__ c_ts)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -234,9 +320,11 @@ gemm_f16_tcgen05(const __grid_constant__ CUtensorMap tmap_a,
     uint64_t *drain = acc_empty + 2;          // [1]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    float *inv_tab = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 256);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    if constexpr (QOUT) out_inv_table(inv_tab, c_ts, err);
     const TileIter it{(M + BM - 1) / BM, (N + BN - 1) / BN,
                       ((M + BM - 1) / BM) * ((N + BN - 1) / BN)};
     const int k_blocks = (K + BK - 1) / BK;
@@ -333,6 +421,12 @@ gemm_f16_tcgen05(const __grid_constant__ CUtensorMap tmap_a,
         const int quarter = warp & 3;                 // TMEM lanes this warp may read
         const int row_in_tile = quarter * 32 + lane;
         const float scale = __fmul_rn(*a_ts, *b_ts);
+        OutQ oq{c_codes, c_scales, 1.0f, 1.0f, inv_tab};
+        if constexpr (QOUT) {
+            oq.ts = *c_ts;
+            oq.rts = __frcp_rn(oq.ts);
+        }
+        bool nonfinite = false;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < it.tiles; t += gridDim.x) {
@@ -344,32 +438,18 @@ gemm_f16_tcgen05(const __grid_constant__ CUtensorMap tmap_a,
             if (!ok) break;
             tc_fence_after();
             const int row = m0 + row_in_tile;
-            __nv_bfloat16 *crow = c + (int64_t)row * N;
 #pragma unroll 1
             for (int chunk = 0; chunk < BN / 32; ++chunk) {
                 uint32_t r[32];
                 tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) +
                               (uint32_t)(acc * BN + chunk * 32), r);
-                const int col0 = n0 + chunk * 32;
-                if (row < M) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int col = col0 + q * 8;
-                        if (col < N) {
-                            uint32_t p[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                p[e] = bf16x2(__fmul_rn(__uint_as_float(r[q * 8 + 2 * e]), scale),
-                                              __fmul_rn(__uint_as_float(r[q * 8 + 2 * e + 1]), scale));
-                            st_v4(crow + col, p[0], p[1], p[2], p[3]);
-                        }
-                    }
-                }
+                nonfinite |= store_chunk<QOUT>(r, scale, row, M, N, n0 + chunk * 32, c, oq);
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&acc_empty[acc]));
             if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         }
+        if (nonfinite && err) atomicOr(err, IF4_DEV_NONFINITE);
     }
 
     tc_fence_before();
@@ -405,7 +485,7 @@ constexpr int PSTAGES = 6;
 constexpr int PA_BYTES = PBM * BK * 2;    // 16 KB
 constexpr int PB_BYTES = PBNH * BK * 2;   // 16 KB
 constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;
-constexpr int PSMEM_BYTES = PSTAGES * PSTAGE_BYTES + 1024 + 256;
+constexpr int PSMEM_BYTES = PSTAGES * PSTAGE_BYTES + 1024 + 256 + 512;
 constexpr uint32_t PIDESC = (1u << 4) | ((uint32_t)(PBN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 
 __device__ __forceinline__ uint32_t cta_rank()
@@ -463,11 +543,14 @@ __device__ __forceinline__ void umma_commit_both(uint32_t bar)
 
 }  // namespace pair
 
+template <bool QOUT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_f16_tcgen05_2sm(const __grid_constant__ CUtensorMap tmap_a,
                      const __grid_constant__ CUtensorMap tmap_b,
                      const float *__restrict__ a_ts, const float *__restrict__ b_ts,
-                     __nv_bfloat16 *__restrict__ c, int M, int N, int K, int *err)
+                     __nv_bfloat16 *__restrict__ c, int M, int N, int K, int *err,
+                     uint8_t *__restrict__ c_codes, uint8_t *__restrict__ c_scales,
+                     const float *__restrict__ c_ts)
 {
     using namespace pair;
     extern __shared__ uint8_t smem_raw[];
@@ -483,6 +566,8 @@ gemm_f16_tcgen05_2sm(const __grid_constant__ CUtensorMap tmap_a,
     uint64_t *drain = acc_empty + 2;          // [1], leader
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    float *inv_tab = reinterpret_cast<float *>(smem + PSTAGES * PSTAGE_BYTES + 256);
+    if constexpr (QOUT) out_inv_table(inv_tab, c_ts, err);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -582,6 +667,12 @@ gemm_f16_tcgen05_2sm(const __grid_constant__ CUtensorMap tmap_a,
         const int quarter = warp & 3;
         const int row_in_cta = quarter * 32 + lane;
         const float scale = __fmul_rn(*a_ts, *b_ts);
+        OutQ oq{c_codes, c_scales, 1.0f, 1.0f, inv_tab};
+        if constexpr (QOUT) {
+            oq.ts = *c_ts;
+            oq.rts = __frcp_rn(oq.ts);
+        }
+        bool nonfinite = false;
         const uint32_t acc_empty_leader0 = map_to(smem_u32(&acc_empty[0]), 0);
         const uint32_t acc_empty_leader1 = map_to(smem_u32(&acc_empty[1]), 0);
         int acc = 0;
@@ -594,32 +685,18 @@ gemm_f16_tcgen05_2sm(const __grid_constant__ CUtensorMap tmap_a,
             if (!ok) break;
             tc_fence_after();
             const int row = m0 + row_in_cta;
-            __nv_bfloat16 *crow = c + (int64_t)row * N;
 #pragma unroll 1
             for (int chunk = 0; chunk < PBN / 32; ++chunk) {
                 uint32_t r[32];
                 tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) +
                               (uint32_t)(acc * PBN + chunk * 32), r);
-                const int col0 = n0 + chunk * 32;
-                if (row < M) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int col = col0 + q * 8;
-                        if (col < N) {
-                            uint32_t pk[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                pk[e] = bf16x2(__fmul_rn(__uint_as_float(r[q * 8 + 2 * e]), scale),
-                                               __fmul_rn(__uint_as_float(r[q * 8 + 2 * e + 1]), scale));
-                            st_v4(crow + col, pk[0], pk[1], pk[2], pk[3]);
-                        }
-                    }
-                }
+                nonfinite |= store_chunk<QOUT>(r, scale, row, M, N, n0 + chunk * 32, c, oq);
             }
             tc_fence_before();
             arrive_remote(acc ? acc_empty_leader1 : acc_empty_leader0);
             if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         }
+        if (nonfinite && err) atomicOr(err, IF4_DEV_NONFINITE);
     }
 
     tc_fence_before();
@@ -695,24 +772,34 @@ int check_gemm_args(const void *a, const void *b, const float *a_ts, const float
     return IF4_OK;
 }
 
-int launch_gemm(const void *a, const void *b, const float *a_ts, const float *b_ts, int64_t M,
-                int64_t N, int64_t K, void *c, int *err, cudaStream_t st)
+// Output of a launch: bf16 C (may be null when QOUT) and, when QOUT, the
+// IF4 codes and scales of C under the tensor scale *c_ts.
+struct GemmOut {
+    void *c;
+    uint8_t *c_codes, *c_scales;
+    const float *c_ts;
+};
+
+template <bool QOUT>
+int launch_gemm_t(const void *a, const void *b, const float *a_ts, const float *b_ts, int64_t M,
+                  int64_t N, int64_t K, const GemmOut &o, int *err, cudaStream_t st)
 {
     int sms = 0;
     int rc = sm_count_checked(sms);
     if (rc != IF4_OK) return rc;
+    __nv_bfloat16 *c = static_cast<__nv_bfloat16 *>(o.c);
     // A CTA pair per 256 x 256 tile when both dimensions fill a pair tile,
     // otherwise one CTA per 128 x 256 tile.
     const bool use_pair = M >= 256 && N >= 256 && sms >= 2;
     CUtensorMap ma, mb;
     if (use_pair) {
+        auto kernel = gemm_f16_tcgen05_2sm<QOUT>;
         if (!make_map(&ma, a, M, K, pair::PBM) || !make_map(&mb, b, N, K, pair::PBNH))
             return IF4_ERR_CUDA;
         static std::once_flag attr2_once;
         static cudaError_t attr2_rc = cudaSuccess;
-        std::call_once(attr2_once, [] {
-            attr2_rc = cudaFuncSetAttribute(gemm_f16_tcgen05_2sm,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+        std::call_once(attr2_once, [&kernel] {
+            attr2_rc = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             pair::PSMEM_BYTES);
         });
         if (attr2_rc != cudaSuccess) return IF4_ERR_CUDA;
@@ -734,9 +821,9 @@ int launch_gemm(const void *a, const void *b, const float *a_ts, const float *b_
         // must share a GPC, so this can be below sms / 2)
         static std::once_flag clusters_once;
         static int resident_pairs = 0;
-        std::call_once(clusters_once, [&cfg] {
+        std::call_once(clusters_once, [&cfg, &kernel] {
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, gemm_f16_tcgen05_2sm, &cfg) == cudaSuccess)
+            if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess)
                 resident_pairs = n;
             else
                 (void)cudaGetLastError();
@@ -745,25 +832,32 @@ int launch_gemm(const void *a, const void *b, const float *a_ts, const float *b_
         if (pairs > sms / 2) pairs = sms / 2;
         if (tiles < pairs) pairs = tiles;
         cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
-        if (cudaLaunchKernelEx(&cfg, gemm_f16_tcgen05_2sm, ma, mb, a_ts, b_ts,
-                               static_cast<__nv_bfloat16 *>(c), (int)M, (int)N, (int)K, err) !=
-            cudaSuccess)
+        if (cudaLaunchKernelEx(&cfg, kernel, ma, mb, a_ts, b_ts, c, (int)M, (int)N, (int)K, err,
+                               o.c_codes, o.c_scales, o.c_ts) != cudaSuccess)
             return IF4_ERR_CUDA;
         return cudaGetLastError() == cudaSuccess ? IF4_OK : IF4_ERR_CUDA;
     }
+    auto kernel = gemm_f16_tcgen05<QOUT>;
     if (!make_map(&ma, a, M, K, BM) || !make_map(&mb, b, N, K, BN)) return IF4_ERR_CUDA;
     static std::once_flag attr_once;
     static cudaError_t attr_rc = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_rc = cudaFuncSetAttribute(gemm_f16_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    std::call_once(attr_once, [&kernel] {
+        attr_rc = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SMEM_BYTES);
     });
     if (attr_rc != cudaSuccess) return IF4_ERR_CUDA;
     const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = (int)(tiles < sms ? tiles : sms);
-    gemm_f16_tcgen05<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(
-        ma, mb, a_ts, b_ts, static_cast<__nv_bfloat16 *>(c), (int)M, (int)N, (int)K, err);
+    kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ma, mb, a_ts, b_ts, c, (int)M, (int)N, (int)K,
+                                                  err, o.c_codes, o.c_scales, o.c_ts);
     return cudaGetLastError() == cudaSuccess ? IF4_OK : IF4_ERR_CUDA;
+}
+
+int launch_gemm(const void *a, const void *b, const float *a_ts, const float *b_ts, int64_t M,
+                int64_t N, int64_t K, void *c, int *err, cudaStream_t st)
+{
+    const GemmOut o{c, nullptr, nullptr, nullptr};
+    return launch_gemm_t<false>(a, b, a_ts, b_ts, M, N, K, o, err, st);
 }
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -804,6 +898,34 @@ int if4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_t
     rc = if4_decode_f16(b_codes, b_scales, N, K, wb, stream);
     if (rc != IF4_OK) return rc;
     return launch_gemm(wa, wb, a_ts, b_ts, M, N, K, c, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+int if4_linear_quantized(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_ts,
+                         const uint8_t *b_codes, const uint8_t *b_scales, const float *b_ts,
+                         int64_t M, int64_t N, int64_t K, void *workspace, size_t ws_bytes,
+                         void *c, uint8_t *c_codes, uint8_t *c_scales, const float *c_ts,
+                         int *err_flag, void *stream)
+{
+    if (!a_codes || !a_scales || !b_codes || !b_scales || !c_codes || !c_scales || !c_ts)
+        return IF4_ERR_NULL;
+    // c is optional here; the shared checks see the codes pointer in its place
+    int rc = check_gemm_args(a_codes, b_codes, a_ts, b_ts, M, N, K, c ? c : c_codes, err_flag);
+    if (rc != IF4_OK) return rc;
+    if (N % 16 != 0) return IF4_ERR_SHAPE;
+    if (reinterpret_cast<uintptr_t>(c_codes) % 16 != 0 || reinterpret_cast<uintptr_t>(c_ts) % 4 != 0)
+        return IF4_ERR_ALIGN;
+    const size_t need = if4_linear_workspace_bytes(M, N, K);
+    if (workspace == nullptr || ws_bytes < need) return IF4_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return IF4_ERR_ALIGN;
+    uint8_t *wa = static_cast<uint8_t *>(workspace);
+    uint8_t *wb = wa + align_up((size_t)M * (size_t)K * 2, 256);
+    rc = if4_decode_f16(a_codes, a_scales, M, K, wa, stream);
+    if (rc != IF4_OK) return rc;
+    rc = if4_decode_f16(b_codes, b_scales, N, K, wb, stream);
+    if (rc != IF4_OK) return rc;
+    const GemmOut o{c, c_codes, c_scales, c_ts};
+    return launch_gemm_t<true>(wa, wb, a_ts, b_ts, M, N, K, o, err_flag,
+                               static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

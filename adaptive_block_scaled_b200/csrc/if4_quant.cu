@@ -26,26 +26,11 @@
 
 #include "../../include/if4.h"
 #include "if4_device.cuh"
+#include "if4_encode.cuh"
 
 using namespace if4dev;
 
 namespace {
-
-// fl(7/6) and fl(6/7) in binary32, and 1.5 * 2^23: adding it to |t| < 2^22
-// leaves round-to-nearest-even(t) in the low mantissa bits.
-__device__ __forceinline__ float c76() { return __uint_as_float(0x3F955555u); }
-__device__ __forceinline__ float c67() { return __uint_as_float(0x3F5B6DB7u); }
-constexpr float kMagic = 12582912.0f;
-
-constexpr float kTsFloor = 0x1p-117f;
-constexpr float kTsCeil = 0x1p117f;
-
-enum { DT_F32 = IF4_F32, DT_BF16 = IF4_BF16, DT_F16 = IF4_F16 };
-
-// Quantizer modes: IF4 (lower-error candidate), NVFP4 (FP4 always), NVINT4
-// (7/6-scaled INT4 always), 4/6 (NVFP4 with the block maximum mapped to 6 or
-// to 4, lower x-domain error kept).
-enum { Q_IF4 = 0, Q_NVFP4 = 1, Q_NVINT4 = 2, Q_46 = 3 };
 
 // --------------------------------------------------------- group loads ----
 
@@ -230,276 +215,6 @@ __device__ __forceinline__ void reload_group(const char *p, uint32_t signs, floa
     if constexpr (RHT) hadamard16_scalar(y, signs);
 }
 
-// ------------------------------------------------------- the quantizer ----
-
-// FP4 candidates of four element pairs (elements 0..7 of a word): one code
-// word (element 0 in bits 0-3) and, when ERR, the differences qf - v of all
-// eight elements as four pairs.  The E2M1 bytes stay in 8-bit registers, the
-// decoded values stay f16 (they are exact there) and each difference is one
-// mixed-precision subtract, i.e. one rounding of the exact qf - v.  Operands
-// are passed as 64-bit register pairs so no moves are needed around the
-// paired-float arithmetic.
-template <bool ERR>
-__device__ __forceinline__ uint32_t fp4_word(const f2_t (&v)[4], f2_t (&d)[4])
-{
-    uint32_t word;
-    if constexpr (ERR) {
-        asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 h0, h1, h2, h3;\n\t"
-            ".reg .b16 l0, l1, l2, l3, u0, u1, u2, u3;\n\t"
-            ".reg .f32 x<8>, e<8>;\n\t"
-            "mov.b64 {x0, x1}, %5;\n\t"
-            "mov.b64 {x2, x3}, %6;\n\t"
-            "mov.b64 {x4, x5}, %7;\n\t"
-            "mov.b64 {x6, x7}, %8;\n\t"
-            "cvt.rn.satfinite.e2m1x2.f32 b0, x1, x0;\n\t"
-            "cvt.rn.satfinite.e2m1x2.f32 b1, x3, x2;\n\t"
-            "cvt.rn.satfinite.e2m1x2.f32 b2, x5, x4;\n\t"
-            "cvt.rn.satfinite.e2m1x2.f32 b3, x7, x6;\n\t"
-            "mov.b32 %0, {b0, b1, b2, b3};\n\t"
-            "cvt.rn.f16x2.e2m1x2 h0, b0;\n\t"
-            "cvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
-            "cvt.rn.f16x2.e2m1x2 h2, b2;\n\t"
-            "cvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
-            "mov.b32 {l0, u0}, h0;\n\t"
-            "mov.b32 {l1, u1}, h1;\n\t"
-            "mov.b32 {l2, u2}, h2;\n\t"
-            "mov.b32 {l3, u3}, h3;\n\t"
-            "sub.rn.f32.f16 e0, l0, x0;\n\t"
-            "sub.rn.f32.f16 e1, u0, x1;\n\t"
-            "sub.rn.f32.f16 e2, l1, x2;\n\t"
-            "sub.rn.f32.f16 e3, u1, x3;\n\t"
-            "sub.rn.f32.f16 e4, l2, x4;\n\t"
-            "sub.rn.f32.f16 e5, u2, x5;\n\t"
-            "sub.rn.f32.f16 e6, l3, x6;\n\t"
-            "sub.rn.f32.f16 e7, u3, x7;\n\t"
-            "mov.b64 %1, {e0, e1};\n\t"
-            "mov.b64 %2, {e2, e3};\n\t"
-            "mov.b64 %3, {e4, e5};\n\t"
-            "mov.b64 %4, {e6, e7};\n\t}"
-            : "=r"(word), "=l"(d[0]), "=l"(d[1]), "=l"(d[2]), "=l"(d[3])
-            : "l"(v[0]), "l"(v[1]), "l"(v[2]), "l"(v[3]));
-    } else {
-        asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .f32 x<8>;\n\t"
-            "mov.b64 {x0, x1}, %1;\n\t"
-            "mov.b64 {x2, x3}, %2;\n\t"
-            "mov.b64 {x4, x5}, %3;\n\t"
-            "mov.b64 {x6, x7}, %4;\n\t"
-            "cvt.rn.satfinite.e2m1x2.f32 b0, x1, x0;\n\t"
-            "cvt.rn.satfinite.e2m1x2.f32 b1, x3, x2;\n\t"
-            "cvt.rn.satfinite.e2m1x2.f32 b2, x5, x4;\n\t"
-            "cvt.rn.satfinite.e2m1x2.f32 b3, x7, x6;\n\t"
-            "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-            : "=r"(word) : "l"(v[0]), "l"(v[1]), "l"(v[2]), "l"(v[3]));
-    }
-    return word;
-}
-
-// INT4 candidate of an element pair: r = 1.5*2^23 + RNE(v * fl(7/6)), one
-// fused multiply-add, so the integer is the exact product rounded once (bits
-// 0-3 of r are the nibble); d = v - k*fl(6/7) with one rounding (the rule's
-// value is fl(6k/7) = fl(k*fl(6/7)); the difference is at most 2^-22).
-template <bool CLAMP>
-__device__ __forceinline__ void int4_pair(f2_t v, f2_t &r, f2_t &d)
-{
-    const f2_t C76 = f2_pack(c76(), c76());
-    const f2_t M = f2_pack(kMagic, kMagic);
-    r = f2_fma(v, C76, M);
-    if constexpr (CLAMP) {
-        float r0, r1;
-        f2_unpack(r, r0, r1);
-        r0 = fminf(fmaxf(r0, kMagic - 7.0f), kMagic + 7.0f);
-        r1 = fminf(fmaxf(r1, kMagic - 7.0f), kMagic + 7.0f);
-        r = f2_pack(r0, r1);
-    }
-    const f2_t NC67 = f2_pack(-c67(), -c67());
-    d = f2_fma(f2_sub(r, M), NC67, v);
-}
-
-// Pack the low nibbles of 8 magic-biased floats (elements 0..7) into a word,
-// element 0 in bits 0-3.
-__device__ __forceinline__ uint32_t pack_int4_nibbles(const f2_t (&r)[4])
-{
-    uint32_t e[4], o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float a, b;
-        f2_unpack(r[j], a, b);
-        e[j] = __float_as_uint(a);
-        o[j] = __float_as_uint(b);
-    }
-    // gather byte 0 of each: even elements -> E, odd elements -> O
-    uint32_t E = prmt(prmt(e[0], e[1], 0x0040u), prmt(e[2], e[3], 0x0040u), 0x5410u);
-    uint32_t O = prmt(prmt(o[0], o[1], 0x0040u), prmt(o[2], o[3], 0x0040u), 0x5410u);
-    return (E & 0x0F0F0F0Fu) | ((O << 4) & 0xF0F0F0F0u);
-}
-
-// True when every element's FP4 and INT4 candidates of one code word have
-// the same value.  The two grids share only 0 and +-6, so that means, per
-// nibble: the FP4 magnitude is 0 and k = 0, or the FP4 nibble is +6 (0x7) and
-// k = 7, or -6 (0xF) and k = -7 (0x9).  Then the two error sums add identical
-// terms in the same order, so they are equal in any precision and the rule
-// keeps FP4.  Evaluated on all eight nibbles at once.
-__device__ __forceinline__ bool candidates_coincide(uint32_t fp4, uint32_t int4)
-{
-    const uint32_t m = fp4 & 0x77777777u;                       // magnitudes
-    const uint32_t is6 = m & (m >> 1) & (m >> 2) & 0x11111111u;  // magnitude 7 (value 6)
-    const uint32_t nz = (m | (m >> 1) | (m >> 2)) & 0x11111111u; // magnitude != 0
-    const uint32_t sgn = (fp4 >> 3) & 0x11111111u;               // FP4 sign bits
-    // expected INT4 nibble: 0 for magnitude 0, 7 for +6, 9 for -6
-    const uint32_t want = (is6 * 0xFu) & (0x77777777u ^ (sgn * 0xEu));
-    return (nz & ~is6) == 0u && int4 == want;
-}
-
-// Binary64 squared-error sums of both candidates in element order: the
-// decision rule itself, used only when the binary32 margin of a group is too
-// small to trust.  It re-reads the group's 16 inputs (still in L2) and walks
-// them one by one, so the common path keeps no extra registers for it.  The
-// INT4 integer is always clamped here; the clamp is the identity whenever the
-// fast path skipped it.
-template <int DT, bool RHT>
-__device__ __noinline__ bool int4_wins_exact(const char *p, float inv, uint32_t signs)
-{
-    float xs[16];
-    reload_group<DT, RHT>(p, signs, xs);
-    double ef = 0.0, ei = 0.0;
-#pragma unroll 1
-    for (int i = 0; i < 16; ++i) {
-        const float v = __fmul_rn(xs[i], inv);
-        const uint32_t h = f16x2_from_e2m1x2(e2m1x2_from_f32(v, 0.0f));
-        const float qf = f16lo_to_f32(h);
-        float r = __fmaf_rn(v, c76(), kMagic);
-        r = fminf(fmaxf(r, kMagic - 7.0f), kMagic + 7.0f);
-        const float qi = __fmul_rn(__fsub_rn(r, kMagic), c67());
-        const double df = __dsub_rn((double)v, (double)qf);
-        const double di = __dsub_rn((double)v, (double)qi);
-        ef = __dadd_rn(ef, __dmul_rn(df, df));
-        ei = __dadd_rn(ei, __dmul_rn(di, di));
-    }
-    return ei < ef;
-}
-
-// The IF4 choice for a group whose binary32 margin is within rounding: equal
-// candidates keep FP4, anything else is decided by the binary64 rule.
-template <int DT, bool RHT>
-__device__ __noinline__ bool int4_wins_rare(uint32_t f0, uint32_t f1, uint32_t i0, uint32_t i1,
-                                            const char *p, float inv, uint32_t signs)
-{
-    if (candidates_coincide(f0, i0) && candidates_coincide(f1, i1)) return false;
-    return int4_wins_exact<DT, RHT>(p, inv, signs);
-}
-
-struct GroupCode {
-    uint32_t c0, c1;   // codes of elements 0..7 and 8..15
-    uint32_t scale;    // scale byte
-    uint32_t f0, f1;   // IF4 paths: the FP4 candidate's codes (the NVFP4 codes)
-};
-
-// Encode one group from its 16 inputs x (pairs), the block scale byte sb and
-// the reciprocal inv of its decoded scale.
-//
-// Decision, fast path: the two squared-error sums are accumulated in binary32
-// (two lanes of 8 terms each, then one add).  The FP4 differences qf - v are
-// exact (v and qf are within a factor of two of each other, or qf = 0); an
-// INT4 difference is off by at most 2^-22 (k*fl(6/7) is not rounded before
-// the subtraction) plus one rounding.  With Cauchy-Schwarz and sqrt(E) <=
-// (1 + E)/2, the binary32 difference of the sums is within (9u + 2^-20) S +
-// 2^-20 + 2^-40 of the binary64 rule (u = 2^-24, S = sum of both errors).
-// Outside the band 2^-18 (S + 1) its sign is the rule's; inside it the group
-// is decided by the rule itself.
-template <int DT, int MODE, bool CLAMP, bool RHT>
-__device__ __forceinline__ GroupCode encode_group(const f2_t (&x)[8], uint32_t sb, float inv,
-                                                const char *p, uint32_t signs)
-{
-    const f2_t INV = f2_pack(inv, inv);
-    f2_t v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = f2_mul(x[j], INV);
-    const f2_t lo[4] = {v[0], v[1], v[2], v[3]};
-    const f2_t hi[4] = {v[4], v[5], v[6], v[7]};
-    GroupCode out;
-    out.scale = sb;
-    if constexpr (MODE == Q_NVFP4) {
-        f2_t unused[4];
-        out.c0 = fp4_word<false>(lo, unused);
-        out.c1 = fp4_word<false>(hi, unused);
-        return out;
-    } else if constexpr (MODE == Q_NVINT4) {
-        f2_t r[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            f2_t unused;
-            int4_pair<CLAMP>(v[j], r[j], unused);
-        }
-        const f2_t rlo[4] = {r[0], r[1], r[2], r[3]};
-        const f2_t rhi[4] = {r[4], r[5], r[6], r[7]};
-        out.c0 = pack_int4_nibbles(rlo);
-        out.c1 = pack_int4_nibbles(rhi);
-        out.scale = sb | 0x80u;
-        return out;
-    } else {
-        f2_t df[8];
-        f2_t dlo[4], dhi[4];
-        out.c0 = fp4_word<true>(lo, dlo);
-        out.c1 = fp4_word<true>(hi, dhi);
-        out.f0 = out.c0;
-        out.f1 = out.c1;
-        f2_t ef = f2_pack(0.0f, 0.0f), ei = f2_pack(0.0f, 0.0f);
-        f2_t r[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) { df[j] = dlo[j]; df[4 + j] = dhi[j]; }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            f2_t di;
-            int4_pair<CLAMP>(v[j], r[j], di);
-            ef = f2_fma(df[j], df[j], ef);
-            ei = f2_fma(di, di, ei);
-        }
-        float a0, a1, b0, b1;
-        f2_unpack(ef, a0, a1);
-        f2_unpack(ei, b0, b1);
-        const float e_fp = __fadd_rn(a0, a1), e_int = __fadd_rn(b0, b1);
-        const float d = __fsub_rn(e_fp, e_int);
-        const float band = __fmul_rn(__fadd_rn(__fadd_rn(e_fp, e_int), 1.0f), 0x1p-18f);
-        const f2_t rlo[4] = {r[0], r[1], r[2], r[3]};
-        const f2_t rhi[4] = {r[4], r[5], r[6], r[7]};
-        const uint32_t i0 = pack_int4_nibbles(rlo), i1 = pack_int4_nibbles(rhi);
-        bool int4 = d > 0.0f;
-        if (!(fabsf(d) > band))      // rare: the binary32 margin is within rounding
-            int4 = int4_wins_rare<DT, RHT>(out.c0, out.c1, i0, i1, p, inv, signs);
-        if (int4) {
-            out.c0 = i0;
-            out.c1 = i1;
-            out.scale = sb | 0x80u;
-        }
-        return out;
-    }
-}
-
-// Block scale sb_f = fl(fl(amax / 6) / ts), each quotient by Markstein's
-// method: with y = RN(1/b), q = RN(a y), r = a - b q (exact by FMA), RN(q +
-// r y) is the correctly rounded a / b when no quotient over- or underflows.
-// Below amax = 2^-100 the IEEE division is used; a second quotient of 2^100 or
-// more is returned unrefined (any value that large saturates to 448, as the
-// exact one does); a second quotient below 2^-126 rounds to the E4M3 code 0
-// either way.
-__device__ __noinline__ float block_scale_ieee(float amax, float div, float ts)
-{
-    return __fdiv_rn(__fdiv_rn(amax, div), ts);
-}
-
-__device__ __forceinline__ float block_scale(float amax, float ts, float rts)
-{
-    const float r6 = __uint_as_float(0x3E2AAAABu);          // RN(1/6)
-    float q = __fmul_rn(amax, r6);
-    q = __fmaf_rn(__fmaf_rn(-q, 6.0f, amax), r6, q);
-    const float s = __fmul_rn(q, rts);
-    const float t = __fmaf_rn(__fmaf_rn(-s, ts, q), rts, s);
-    // rare: tiny amax (IEEE division), or a quotient beyond 2^100 (saturates)
-    if (!(amax >= 0x1p-100f && s < 0x1p100f))
-        return amax >= 0x1p-100f ? s : block_scale_ieee(amax, 6.0f, ts);
-    return t;
-}
-
 __device__ __forceinline__ bool ts_valid(float ts)
 {
     return ts >= kTsFloor && ts <= kTsCeil;   // false for NaN
@@ -530,7 +245,7 @@ __device__ __noinline__ GroupCode encode_group_clamped(uint32_t sb, float inv, c
     f2_t x[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) x[j] = f2_pack(y[2 * j], y[2 * j + 1]);
-    return encode_group<DT, MODE, true, RHT>(x, sb, inv, p, signs);
+    return encode_group<MODE, true>(x, sb, inv, y);
 }
 
 // Address of group g of a [rows, gpr groups] tensor with row stride
@@ -684,48 +399,6 @@ __device__ __forceinline__ GroupCode encode_group_46(const f2_t (&x)[8], float a
     return out;
 }
 
-// IF4 groups off the fast path (rare): a block scale that the quotients of
-// the fast path do not give exactly, or one under which the INT4 integer may
-// need its clamp.  The block scale with its exact fallbacks, then the encode
-// with the clamp, from the group re-read from memory.
-template <int DT, bool RHT>
-__device__ __noinline__ GroupCode if4_group_general(float amax, float ts, float rts,
-                                                    const float *inv_tab, const char *gp,
-                                                    uint32_t signs)
-{
-    const uint32_t sb = e4m3_from_f32(block_scale(amax, ts, rts)) & 0x7Fu;
-    float y[16];
-    reload_group<DT, RHT>(gp, signs, y);
-    f2_t x[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) x[j] = f2_pack(y[2 * j], y[2 * j + 1]);
-    GroupCode out = encode_group<DT, Q_IF4, true, RHT>(x, sb, inv_tab[sb], gp, signs);
-    if (sb == 0) out.c0 = out.c1 = out.scale = out.f0 = out.f1 = 0u;
-    return out;
-}
-
-// IF4 groups whose binary32 margin is within rounding: equal candidates keep
-// FP4, anything else is decided by the binary64 rule.
-template <int DT, bool RHT>
-__device__ __noinline__ GroupCode if4_group_near(uint32_t f0, uint32_t f1, uint32_t i0,
-                                                 uint32_t i1, uint32_t sb, float inv,
-                                                 const char *gp, uint32_t signs)
-{
-    const bool int4 = !(candidates_coincide(f0, i0) && candidates_coincide(f1, i1)) &&
-                      int4_wins_exact<DT, RHT>(gp, inv, signs);
-    GroupCode out;
-    out.c0 = int4 ? i0 : f0;
-    out.c1 = int4 ? i1 : f1;
-    out.scale = int4 ? (sb | 0x80u) : sb;
-    out.f0 = f0;
-    out.f1 = f1;
-    return out;
-}
-
-// 1.5 * 2^23 + 8: fma(v, fl(7/6), kMagic8) leaves k + 8 in bits 0-3 of the
-// result and zeros in bits 4-7 whenever |k| = |RNE(v * fl(7/6))| <= 7.
-constexpr float kMagic8 = 12582920.0f;
-
 // IF4 encode of one group, fast path.  Block scale by Markstein quotients
 // (exact unless flagged below); both candidates without the INT4 clamp (it is
 // the identity for every block scale E4M3 code 8..125: the largest |v| is
@@ -741,74 +414,10 @@ __device__ __forceinline__ GroupCode encode_if4(const f2_t (&xv)[8], float amax,
                                               uint32_t signs)
 {
     constexpr int GB = 16 * elem_bytes<DT>();
-    const float r6 = __uint_as_float(0x3E2AAAABu);          // RN(1/6)
-    float q = __fmul_rn(amax, r6);
-    q = __fmaf_rn(__fmaf_rn(-q, 6.0f, amax), r6, q);
-    const float s = __fmul_rn(q, rts);
-    const float t = __fmaf_rn(__fmaf_rn(-s, ts, q), rts, s);
-    const uint32_t sb = e4m3_from_f32(t) & 0x7Fu;
-    const bool general = !(amax >= 0x1p-100f && s < 0x1p100f) || (sb - 1u) < 7u || sb == 0x7Eu;
-    const float inv = inv_tab[sb];
-
-    const f2_t INV = f2_pack(inv, inv);
-    f2_t v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = f2_mul(xv[j], INV);
-    const f2_t lo[4] = {v[0], v[1], v[2], v[3]};
-    const f2_t hi[4] = {v[4], v[5], v[6], v[7]};
-    f2_t dlo[4], dhi[4];
-    const uint32_t f0 = fp4_word<true>(lo, dlo);
-    const uint32_t f1 = fp4_word<true>(hi, dhi);
-
-    const f2_t C76 = f2_pack(c76(), c76());
-    const f2_t M8 = f2_pack(kMagic8, kMagic8);
-    const f2_t NM8 = f2_pack(-kMagic8, -kMagic8);
-    const f2_t NC67 = f2_pack(-c67(), -c67());
-    f2_t ef = f2_pack(0.0f, 0.0f), ei = f2_pack(0.0f, 0.0f);
-    uint32_t pb[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const f2_t r = f2_fma(v[j], C76, M8);                // M8 + RNE(v * fl(7/6))
-        const f2_t di = f2_fma(f2_add(r, NM8), NC67, v[j]);   // v - k * fl(6/7), one rounding
-        const f2_t df = j < 4 ? dlo[j] : dhi[j - 4];
-        ef = f2_fma(df, df, ef);
-        ei = f2_fma(di, di, ei);
-        float re, ro;
-        f2_unpack(r, re, ro);
-        // byte 0: (k_even + 8) | (k_odd + 8) << 4
-        pb[j] = __float_as_uint(ro) * 16u + __float_as_uint(re);
-    }
-    // gather the bytes, then offset-8 nibbles -> two's complement nibbles
-    const uint32_t i0 = prmt(prmt(pb[0], pb[1], 0x0040u), prmt(pb[2], pb[3], 0x0040u), 0x5410u) ^
-                        0x88888888u;
-    const uint32_t i1 = prmt(prmt(pb[4], pb[5], 0x0040u), prmt(pb[6], pb[7], 0x0040u), 0x5410u) ^
-                        0x88888888u;
-
-    float a0, a1, b0, b1;
-    f2_unpack(ef, a0, a1);
-    f2_unpack(ei, b0, b1);
-    const float e_fp = __fadd_rn(a0, a1), e_int = __fadd_rn(b0, b1);
-    const float d = __fsub_rn(e_fp, e_int);
-    const float S = __fadd_rn(e_fp, e_int);
-    const float band = __fmul_rn(__fadd_rn(S, 1.0f), 0x1p-18f);
-    const bool int4 = d > band;
-    // S == 0: every binary32 square is zero, so every error is (a) zero or
-    // (b) below 2^-75, where both candidates are 0: the sums tie, FP4 stays
-    const bool near = !(fabsf(d) > band) && S != 0.0f;
-    GroupCode out;
-    if (general || near) {
-        const char *gp = group_addr<GB>(x, g, gpr, ld_bytes);
-        out = general ? if4_group_general<DT, RHT>(amax, ts, rts, inv_tab, gp, signs)
-                      : if4_group_near<DT, RHT>(f0, f1, i0, i1, sb, inv, gp, signs);
-    } else {
-        // sb == 0: inv = 0, both candidates are (signed) zeros, the sums 0
-        out.f0 = sb == 0 ? 0u : f0;
-        out.f1 = sb == 0 ? 0u : f1;
-        out.c0 = int4 ? i0 : out.f0;
-        out.c1 = int4 ? i1 : out.f1;
-        out.scale = int4 ? (sb | 0x80u) : sb;
-    }
-    return out;
+    const If4Fast f = if4_fast(xv, amax, ts, rts, inv_tab);
+    return if4_finish(f, amax, ts, rts, inv_tab, [&](float (&y)[16]) {
+        reload_group<DT, RHT>(group_addr<GB>(x, g, gpr, ld_bytes), signs, y);
+    });
 }
 
 // Encode group g from its raw bits r and store its codes and scale byte.
@@ -846,7 +455,7 @@ __device__ __forceinline__ bool quantize_one(const Raw<DT> &r, uint32_t g, const
             out = encode_group_clamped<DT, MODE, RHT>(sb, inv, group_addr<GB>(x, g, gpr, ld_bytes),
                                                       signs);
         else
-            out = encode_group<DT, MODE, false, RHT>(xv, sb, inv, nullptr, signs);
+            out = encode_group<MODE, false>(xv, sb, inv, nullptr);
         if (sb == 0) out.c0 = out.c1 = out.scale = 0u;
     }
     st_v2(codes + (int64_t)g * 8, out.c0, out.c1);

@@ -545,6 +545,29 @@ def linear_report(pk, steps=20, warmup=3):
     e1.record()
     torch.cuda.synchronize()
     t_cublas = e0.elapsed_time(e1) / steps
+    # the same linear with its output quantized to IF4 in the epilogue (no
+    # bf16 C), against the bf16 linear followed by a separate IF4 quantize
+    c_ts = torch.ones(1, dtype=torch.float32, device=dev)
+    b.if4_tensor_amax(c, c_ts)
+    b.if4_tensor_scale(c_ts, c_ts)
+    c_codes = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
+    c_scales = torch.empty((M, N // 16), dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    t_q = timed(lambda: b.if4_linear_quantized(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], ws,
+                                               c_codes, c_scales, c_ts, err_flag=err))
+    t_sep = timed(lambda: (b.if4_linear(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], ws, c, err),
+                           b.if4_quantize(c, c_codes, c_scales, c_ts, b.TS_GIVEN, err)))
     flops = 2.0 * M * N * K
     gemm_tf = flops / (t[2] * 1e-3) / 1e12
     total = sum(t)
@@ -552,6 +575,7 @@ def linear_report(pk, steps=20, warmup=3):
             "decode_a_ms": t[0], "decode_b_ms": t[1], "gemm_ms": t[2], "linear_ms": total,
             "gemm_tflops": gemm_tf, "linear_tflops": flops / (total * 1e-3) / 1e12,
             "cublas_f16_ms": t_cublas, "cublas_f16_tflops": flops / (t_cublas * 1e-3) / 1e12,
+            "linear_if4_out_ms": t_q, "linear_then_quantize_ms": t_sep,
             "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": pk["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": gemm_tf / pk["bf16_tflops"],
                          "peak_source": f"{pk['source']} bf16_tflops (burst); fp16 dense rate = bf16"}}

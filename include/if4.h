@@ -243,6 +243,32 @@ int if4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_t
                int64_t M, int64_t N, int64_t K, void *workspace, size_t ws_bytes,
                void *c, int *err_flag, void *stream);
 
+/*
+ * IF4 x IF4 linear with an IF4 output: the product of if4_linear, rounded to
+ * bf16 exactly as there, then quantized to IF4 along N (groups of 16
+ * columns of each row of C) under the given tensor scale *c_ts, inside the
+ * GEMM's epilogue.  The codes and scales equal those of
+ * if4_quantize(C, IF4_BF16, M, N, N, ..., c_ts, IF4_TS_GIVEN) on the bf16
+ * C of if4_linear.  The output never exists as a bf16 tensor unless c is
+ * given (then it is written too, as by if4_linear).
+ *
+ * The tensor scale of C has to be known before the GEMM runs (for example
+ * the previous step's, as with delayed scaling); an invalid one sets
+ * IF4_DEV_BAD_SCALE, and Inf/NaN in C set IF4_DEV_NONFINITE.  The pages'
+ * W4A4 training feeds quantized activations into the next linear (companion
+ * "MAC Unit: Decoding Two Formats from One Sign Bit"); fusing that quantize
+ * into the producing GEMM is this library's choice.
+ *
+ * c_codes: uint8 [M, N/2], 16-byte aligned; c_scales: uint8 [M, N/16];
+ * c_ts: device float; c: bf16 [M, N] or NULL.  N % 16 == 0.  Other rules,
+ * the workspace and the errors as if4_linear.
+ */
+int if4_linear_quantized(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_ts,
+                         const uint8_t *b_codes, const uint8_t *b_scales, const float *b_ts,
+                         int64_t M, int64_t N, int64_t K, void *workspace, size_t ws_bytes,
+                         void *c, uint8_t *c_codes, uint8_t *c_scales, const float *c_ts,
+                         int *err_flag, void *stream);
+
 /* Size of the scratch array behind if4_linear_noalloc (32 MiB per device). */
 #define IF4_FUSED_SYNC_WORDS 64u
 

@@ -26,6 +26,8 @@ def lib():
     L.if4_tensor_scale.argtypes = [vp, vp, vp]
     L.if4_decode_f16.argtypes = [vp, vp, i64, i64, vp, vp]
     L.if4_quantize_fused.argtypes = [vp, i, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.if4_linear_quantized.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, ctypes.c_size_t,
+                                       vp, vp, vp, vp, vp, vp]
     L.if4_status_str.restype = ctypes.c_char_p
     return L
 
@@ -110,6 +112,20 @@ def test_fused_quantize_host_validation(lib):
     assert f(A, 1, 4, 32, 32, A, A, None, None, A + 2, A, None, None) == 4
     assert f(A, 1, 4, 32, 32, A, A, None, None, A, A + 4, None, None) == 4
     assert f(A, 1, 4, 32, 32, A, A, None, None, A, A + 128, None, None) == 4
+
+
+def test_linear_quantized_host_validation(lib):
+    f = lib.if4_linear_quantized
+    W = 1 << 30
+    # null output codes / scales / tensor scale
+    assert f(A, A, A, A, A, A, 128, 256, 64, A, W, None, None, A, A, A, None) == 1
+    assert f(A, A, A, A, A, A, 128, 256, 64, A, W, None, A, None, A, A, None) == 1
+    assert f(A, A, A, A, A, A, 128, 256, 64, A, W, None, A, A, None, A, None) == 1
+    # N % 16, misaligned codes / ts, too small a workspace
+    assert f(A, A, A, A, A, A, 128, 264, 64, A, W, None, A, A, A, A, None) == 2
+    assert f(A, A, A, A, A, A, 128, 256, 64, A, W, None, A + 8, A, A, A, None) == 4
+    assert f(A, A, A, A, A, A, 128, 256, 64, A, W, None, A, A, A + 2, A, None) == 4
+    assert f(A, A, A, A, A, A, 128, 256, 64, A, 16, None, A, A, A, A, None) == 6
 
 
 def test_dequantize_and_decode_host_validation(lib):

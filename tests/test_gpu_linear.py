@@ -151,3 +151,53 @@ def test_pair_and_single_cta_paths_agree():
     full = gemm(a, b, 0.5, 2.0)
     parts = torch.cat([gemm(a[i:i + 128].contiguous(), b, 0.5, 2.0) for i in range(0, M, 128)])
     assert torch.equal(full, parts)
+
+
+@pytest.mark.parametrize("M,N,K", [(512, 512, 1024), (300, 528, 256), (128, 256, 64)])
+def test_linear_quantized_output_equals_separate_quantize(M, N, K):
+    """The IF4 output of the epilogue equals if4_quantize of the bf16 C of
+    if4_linear under the same given tensor scale, byte for byte, on both GEMM
+    kernels (M >= 256 uses CTA pairs), with a ragged last 32-column chunk
+    (N % 32 == 16), with and without the bf16 C written beside it, and with a
+    small given scale that saturates block scales (the epilogue's rare path)."""
+    bb = B()
+    a, b = workloads.linear_operands(4, M=M, N=N, K=K)
+    aq, bq = _quantized(a), _quantized(b)
+    c_ref = _linear(aq, bq, M, N, K)
+    c_np = c_ref.float().cpu().numpy()
+    ts_data = oracle.tensor_scale(np.float32(np.max(np.abs(c_np))))
+    ws = torch.empty(bb.if4_linear_workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
+    for factor, write_c in ((1.0, True), (1.0, False), (0.05, False)):
+        c_ts = np.float32(ts_data * factor)
+        t = torch.tensor([c_ts], dtype=torch.float32, device="cuda")
+        codes = torch.empty((M, N // 2), dtype=torch.uint8, device="cuda")
+        scales = torch.empty((M, N // 16), dtype=torch.uint8, device="cuda")
+        c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda") if write_c else None
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        bb.if4_linear_quantized(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], ws, codes, scales, t,
+                                c=c, err_flag=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        if write_c:
+            assert torch.equal(c, c_ref)
+        ref = oracle.quantize(c_np, c_ts)
+        assert np.array_equal(scales.cpu().numpy(), ref["scales"]), (M, N, K, factor)
+        assert np.array_equal(codes.cpu().numpy(), ref["codes"]), (M, N, K, factor)
+        if factor < 1.0:
+            assert np.any((ref["scales"] & 0x7F) == 0x7E)     # saturated block scales
+
+
+def test_linear_quantized_output_flags_invalid_scale():
+    bb = B()
+    M, N, K = 128, 256, 64
+    a, b = workloads.linear_operands(5, M=M, N=N, K=K)
+    aq, bq = _quantized(a), _quantized(b)
+    ws = torch.empty(bb.if4_linear_workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
+    codes = torch.empty((M, N // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((M, N // 16), dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t = torch.tensor([0.0], dtype=torch.float32, device="cuda")
+    bb.if4_linear_quantized(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], ws, codes, scales, t,
+                            err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & bb.DEV_BAD_SCALE
