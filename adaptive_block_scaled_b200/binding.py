@@ -54,6 +54,8 @@ def _load():
                              _vp, _vp],
         "if4_quantize_fused": [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                _vp],
+        "if4_quantize_fused_rht": [_vp, _int, _i64, _i64, _i64, ctypes.c_uint32, _vp, _vp, _vp,
+                                   _vp, _vp, _vp, _vp, _vp],
         "if4_decode_f16": [_vp, _vp, _i64, _i64, _vp, _vp],
         "if4_gemm_f16": [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
         "if4_linear_workspace_bytes": [_i64, _i64, _i64],
@@ -161,7 +163,9 @@ def if4_quantize_rht(x, signs, codes, scales, ts, ts_mode=TS_COMPUTE, err_flag=N
 
 
 def if4_quantize_fused(x, codes, scales, nv_codes, nv_scales, ts, sync_words, err_flag=None,
-                       stream=None):
+                       stream=None, signs=None):
+    """signs=None: the plain single-launch quantizer; an int: the same on the
+    random-sign Hadamard transform of x (if4_quantize_fused_rht)."""
     rows, cols, ld = _matrix(x, "x")
     _u8(codes, "codes", (rows, cols // 2))
     _u8(scales, "scales", (rows, cols // 16))
@@ -173,10 +177,17 @@ def if4_quantize_fused(x, codes, scales, nv_codes, nv_scales, ts, sync_words, er
     if sync_words.dtype != torch.int32 or sync_words.numel() < FUSED_SYNC_WORDS:
         raise ValueError(f"sync_words must be an int32 device tensor of at least "
                          f"{FUSED_SYNC_WORDS} elements")
-    _check(lib.if4_quantize_fused(_ptr(x), _dtype(x, "x"), rows, cols, ld, _ptr(codes),
-                                  _ptr(scales), _ptr(nv_codes), _ptr(nv_scales), _ptr(ts),
-                                  _ptr(sync_words), _ptr(err_flag), _stream(stream)),
-           "if4_quantize_fused")
+    if signs is None:
+        _check(lib.if4_quantize_fused(_ptr(x), _dtype(x, "x"), rows, cols, ld, _ptr(codes),
+                                      _ptr(scales), _ptr(nv_codes), _ptr(nv_scales), _ptr(ts),
+                                      _ptr(sync_words), _ptr(err_flag), _stream(stream)),
+               "if4_quantize_fused")
+    else:
+        _check(lib.if4_quantize_fused_rht(_ptr(x), _dtype(x, "x"), rows, cols, ld,
+                                          int(signs) & 0xFFFF, _ptr(codes), _ptr(scales),
+                                          _ptr(nv_codes), _ptr(nv_scales), _ptr(ts),
+                                          _ptr(sync_words), _ptr(err_flag), _stream(stream)),
+               "if4_quantize_fused_rht")
 
 
 def nvint4_quantize(x, codes, scales, ts, ts_mode=TS_COMPUTE, err_flag=None, stream=None):
@@ -313,9 +324,10 @@ def quantize_rht(x, signs, ts=None, err_flag=None, stream=None):
     return codes, scales, ts_t
 
 
-def quantize_fused(x, with_nvfp4=True, sync_words=None, err_flag=None, stream=None):
-    """amax, tensor scale, IF4 quantize (and NVFP4) in one launch.  Returns
-    (codes, scales, ts) or (codes, scales, ts, nv_codes, nv_scales)."""
+def quantize_fused(x, with_nvfp4=True, sync_words=None, err_flag=None, stream=None, signs=None):
+    """amax, tensor scale, IF4 quantize (and NVFP4) in one launch, of x or,
+    with signs, of its random-sign Hadamard transform.  Returns (codes,
+    scales, ts) or (codes, scales, ts, nv_codes, nv_scales)."""
     rows, cols, _ = _matrix(x, "x")
     dev = x.device
     codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
@@ -325,7 +337,8 @@ def quantize_fused(x, with_nvfp4=True, sync_words=None, err_flag=None, stream=No
     ts = torch.empty(1, dtype=torch.float32, device=dev)
     if sync_words is None:
         sync_words = torch.zeros(FUSED_SYNC_WORDS, dtype=torch.int32, device=dev)
-    if4_quantize_fused(x, codes, scales, nv_codes, nv_scales, ts, sync_words, err_flag, stream)
+    if4_quantize_fused(x, codes, scales, nv_codes, nv_scales, ts, sync_words, err_flag, stream,
+                       signs)
     return (codes, scales, ts, nv_codes, nv_scales) if with_nvfp4 else (codes, scales, ts)
 
 

@@ -219,6 +219,15 @@ __device__ __forceinline__ uint32_t absmax_f16x2(uint32_t a, uint32_t b)
     return r;
 }
 
+// max(|a|, |b|) as float bits with NaN propagated; the result's sign bit is
+// sign(a) ^ sign(b) and must be masked off by the caller
+__device__ __forceinline__ uint32_t absmax_f32(uint32_t a, float b)
+{
+    uint32_t r;
+    asm("max.NaN.xorsign.abs.f32 %0, %1, %2;" : "=r"(r) : "r"(a), "f"(b));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
 {
     uint32_t r;

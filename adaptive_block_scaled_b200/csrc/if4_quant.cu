@@ -71,13 +71,17 @@ template <int DT>
 __device__ __forceinline__ float unpack_group(const Raw<DT> &r, f2_t (&x)[8], bool &nonfinite)
 {
     if constexpr (DT == DT_F32) {
-        uint32_t m = 0;
+        // max |x| in two chains of one instruction per element (NaN
+        // propagates; the sign bit it leaves is masked off)
+        uint32_t m0 = 0, m1 = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            uint32_t a = r.w[2 * j], b = r.w[2 * j + 1];
-            m = max(m, max(a & 0x7FFFFFFFu, b & 0x7FFFFFFFu));
+            const uint32_t a = r.w[2 * j], b = r.w[2 * j + 1];
+            m0 = absmax_f32(m0, __uint_as_float(a));
+            m1 = absmax_f32(m1, __uint_as_float(b));
             x[j] = f2_pack(__uint_as_float(a), __uint_as_float(b));
         }
+        const uint32_t m = absmax_f32(m0, __uint_as_float(m1)) & 0x7FFFFFFFu;
         nonfinite = m >= 0x7F800000u;
         return __uint_as_float(m);
     } else {
@@ -188,13 +192,15 @@ __device__ __forceinline__ float unpack_group_rht(const Raw<DT> &r, const SignMa
         }
     }
     hadamard16(x);
-    uint32_t m = 0;
+    uint32_t m0 = 0, m1 = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         float a, b;
         f2_unpack(x[j], a, b);
-        m = max(m, max(__float_as_uint(a) & 0x7FFFFFFFu, __float_as_uint(b) & 0x7FFFFFFFu));
+        m0 = absmax_f32(m0, a);
+        m1 = absmax_f32(m1, b);
     }
+    const uint32_t m = absmax_f32(m0, __uint_as_float(m1)) & 0x7FFFFFFFu;
     nonfinite = m >= 0x7F800000u;
     return __uint_as_float(m);
 }
@@ -680,7 +686,7 @@ quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr
 
     // pass 1: max |x| (of the transform, with RHT), six loads in flight
     uint32_t m = 0;
-    constexpr int U = DT == DT_F32 ? 3 : 6;
+    constexpr int U = (DT == DT_F32 || RHT) ? 3 : 6;
     for (uint64_t g0 = g_first; g0 < ngroups; g0 += (uint64_t)U * stride) {
         Raw<DT> r[U];
 #pragma unroll
@@ -1184,6 +1190,45 @@ int launch_dequant(const Shape &s, const uint8_t *codes, const uint8_t *scales, 
     return launch_status();
 }
 
+template <bool RHT>
+int fused_entry(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                uint8_t *codes, uint8_t *scales, uint8_t *nv_codes, uint8_t *nv_scales, float *ts,
+                uint32_t *sync_words, int *err_flag, void *stream, uint32_t signs)
+{
+    Shape s;
+    int rc = check_tensor(x, x_dtype, rows, cols, ld_x, s);
+    if (rc != IF4_OK) return rc;
+    if (ts == nullptr || sync_words == nullptr) return IF4_ERR_NULL;
+    if ((nv_codes == nullptr) != (nv_scales == nullptr)) return IF4_ERR_NULL;
+    if (s.ngroups > 0 && (codes == nullptr || scales == nullptr)) return IF4_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(codes) % 16 != 0 ||
+        reinterpret_cast<uintptr_t>(nv_codes) % 16 != 0 ||
+        reinterpret_cast<uintptr_t>(ts) % 4 != 0 || reinterpret_cast<uintptr_t>(sync_words) % 256 != 0)
+        return IF4_ERR_ALIGN;
+    DeviceInfo d;
+    rc = check_device(d);
+    if (rc != IF4_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (s.ngroups == 0) {
+        // an empty tensor: amax 0, ts 1, nothing to encode
+        if (cudaMemsetAsync(ts, 0, sizeof(float), st) != cudaSuccess) return IF4_ERR_CUDA;
+        tensor_scale_kernel<<<1, 1, 0, st>>>(ts, ts);
+        return launch_status();
+    }
+    const SignMasks sm = sign_masks(x_dtype, signs);
+    switch (x_dtype) {
+    case IF4_F32:
+        return dispatch_fused_dt<DT_F32, RHT>(s, x, codes, scales, nv_codes, nv_scales, ts,
+                                                sync_words, err_flag, st, d, sm, signs);
+    case IF4_BF16:
+        return dispatch_fused_dt<DT_BF16, RHT>(s, x, codes, scales, nv_codes, nv_scales, ts,
+                                                 sync_words, err_flag, st, d, sm, signs);
+    default:
+        return dispatch_fused_dt<DT_F16, RHT>(s, x, codes, scales, nv_codes, nv_scales, ts,
+                                                sync_words, err_flag, st, d, sm, signs);
+    }
+}
+
 }  // namespace
 
 // ================================================================ C ABI ====
@@ -1282,38 +1327,17 @@ int if4_quantize_fused(const void *x, int x_dtype, int64_t rows, int64_t cols, i
                        uint8_t *codes, uint8_t *scales, uint8_t *nv_codes, uint8_t *nv_scales,
                        float *ts, uint32_t *sync_words, int *err_flag, void *stream)
 {
-    Shape s;
-    int rc = check_tensor(x, x_dtype, rows, cols, ld_x, s);
-    if (rc != IF4_OK) return rc;
-    if (ts == nullptr || sync_words == nullptr) return IF4_ERR_NULL;
-    if ((nv_codes == nullptr) != (nv_scales == nullptr)) return IF4_ERR_NULL;
-    if (s.ngroups > 0 && (codes == nullptr || scales == nullptr)) return IF4_ERR_NULL;
-    if (reinterpret_cast<uintptr_t>(codes) % 16 != 0 ||
-        reinterpret_cast<uintptr_t>(nv_codes) % 16 != 0 ||
-        reinterpret_cast<uintptr_t>(ts) % 4 != 0 || reinterpret_cast<uintptr_t>(sync_words) % 256 != 0)
-        return IF4_ERR_ALIGN;
-    DeviceInfo d;
-    rc = check_device(d);
-    if (rc != IF4_OK) return rc;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (s.ngroups == 0) {
-        // an empty tensor: amax 0, ts 1, nothing to encode
-        if (cudaMemsetAsync(ts, 0, sizeof(float), st) != cudaSuccess) return IF4_ERR_CUDA;
-        tensor_scale_kernel<<<1, 1, 0, st>>>(ts, ts);
-        return launch_status();
-    }
-    const SignMasks sm = sign_masks(x_dtype, 0);
-    switch (x_dtype) {
-    case IF4_F32:
-        return dispatch_fused_dt<DT_F32, false>(s, x, codes, scales, nv_codes, nv_scales, ts,
-                                                sync_words, err_flag, st, d, sm, 0);
-    case IF4_BF16:
-        return dispatch_fused_dt<DT_BF16, false>(s, x, codes, scales, nv_codes, nv_scales, ts,
-                                                 sync_words, err_flag, st, d, sm, 0);
-    default:
-        return dispatch_fused_dt<DT_F16, false>(s, x, codes, scales, nv_codes, nv_scales, ts,
-                                                sync_words, err_flag, st, d, sm, 0);
-    }
+    return fused_entry<false>(x, x_dtype, rows, cols, ld_x, codes, scales, nv_codes, nv_scales, ts,
+                              sync_words, err_flag, stream, 0u);
+}
+
+int if4_quantize_fused_rht(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                           uint32_t signs, uint8_t *codes, uint8_t *scales, uint8_t *nv_codes,
+                           uint8_t *nv_scales, float *ts, uint32_t *sync_words, int *err_flag,
+                           void *stream)
+{
+    return fused_entry<true>(x, x_dtype, rows, cols, ld_x, codes, scales, nv_codes, nv_scales, ts,
+                             sync_words, err_flag, stream, signs & 0xFFFFu);
 }
 
 int if4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts, int64_t rows,

@@ -173,6 +173,18 @@ int if4_quantize_fused(const void *x, int x_dtype, int64_t rows, int64_t cols, i
                        float *ts, uint32_t *sync_words, int *err_flag, void *stream);
 
 /*
+ * The same single launch on the random-sign Hadamard transform of x (see
+ * if4_quantize_rht): the amax, the tensor scale, the IF4 codes and the
+ * NVFP4 comparator are those of the transformed tensor, equal to
+ * if4_quantize_rht(IF4_TS_COMPUTE) and nvfp4_quantize of the transformed
+ * tensor under that ts.  signs: bits 0-15 as for if4_quantize_rht.
+ */
+int if4_quantize_fused_rht(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                           uint32_t signs, uint8_t *codes, uint8_t *scales, uint8_t *nv_codes,
+                           uint8_t *nv_scales, float *ts, uint32_t *sync_words, int *err_flag,
+                           void *stream);
+
+/*
  * Comparator, all-INT4 ("NVINT4"): the 7/6-scaled INT4 candidate of
  * if4_quantize for every group, bit 7 set wherever the block scale is
  * nonzero (gist.science section 3, item 2, and section 4: IF4 is compared with

@@ -26,6 +26,8 @@ def lib():
     L.if4_tensor_scale.argtypes = [vp, vp, vp]
     L.if4_decode_f16.argtypes = [vp, vp, i64, i64, vp, vp]
     L.if4_quantize_fused.argtypes = [vp, i, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.if4_quantize_fused_rht.argtypes = [vp, i, i64, i64, i64, ctypes.c_uint32, vp, vp, vp, vp,
+                                         vp, vp, vp, vp]
     L.if4_linear_quantized.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, ctypes.c_size_t,
                                        vp, vp, vp, vp, vp, vp]
     L.if4_status_str.restype = ctypes.c_char_p
@@ -112,6 +114,10 @@ def test_fused_quantize_host_validation(lib):
     assert f(A, 1, 4, 32, 32, A, A, None, None, A + 2, A, None, None) == 4
     assert f(A, 1, 4, 32, 32, A, A, None, None, A, A + 4, None, None) == 4
     assert f(A, 1, 4, 32, 32, A, A, None, None, A, A + 128, None, None) == 4
+    g = lib.if4_quantize_fused_rht
+    assert g(A, 1, 4, 32, 32, 0x1234, A, A, None, None, None, A, None, None) == 1
+    assert g(A, 1, 4, 24, 24, 0x1234, A, A, None, None, A, A, None, None) == 2
+    assert g(A, 1, 4, 32, 32, 0x1234, A, A, None, None, A, A + 64, None, None) == 4
 
 
 def test_linear_quantized_host_validation(lib):

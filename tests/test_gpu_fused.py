@@ -114,3 +114,32 @@ def test_fused_nonfinite_sets_flag_and_leaves_sync_zero():
     x[7, 9] = float("inf")
     _, err = fused(x.cuda())
     assert err & B().DEV_NONFINITE
+
+
+@pytest.mark.parametrize("signs", [0x0000, 0xA5C3])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+def test_fused_rht_matches_oracle_and_separate_calls(signs, dtype):
+    """The single launch on the random-sign Hadamard transform: ts, IF4 and
+    NVFP4 of the transformed tensor, against the oracle (transform, then
+    quantize) and against if4_quantize_rht + nvfp4 of the transform."""
+    b = B()
+    g = torch.Generator().manual_seed(signs + 17)
+    x = (torch.randn((96, 1024), generator=g) * 3).to(dtype)
+    x[:, 5] *= 40                                   # an outlier channel
+    x_np = x.float().numpy()
+    ref = oracle.quantize_tensor_rht(x_np, signs)
+    y = oracle.rht(x_np, signs)
+    nv = oracle.quantize(y, ref["ts"], mode=oracle.MODE_NVFP4)
+    sync = torch.zeros(b.FUSED_SYNC_WORDS, dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    codes, scales, ts, nc, ns = b.quantize_fused(x.cuda(), sync_words=sync, err_flag=err,
+                                                 signs=signs)
+    c2, s2, t2 = b.quantize_rht(x.cuda(), signs)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and sync[0].item() == 0 and sync[1].item() == 0
+    assert np.float32(ts.item()) == ref["ts"] and ts.item() == t2.item()
+    assert np.array_equal(scales.cpu().numpy(), ref["scales"])
+    assert np.array_equal(codes.cpu().numpy(), ref["codes"])
+    assert torch.equal(codes, c2) and torch.equal(scales, s2)
+    assert np.array_equal(ns.cpu().numpy(), nv["scales"])
+    assert np.array_equal(nc.cpu().numpy(), nv["codes"])
