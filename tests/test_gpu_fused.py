@@ -143,3 +143,34 @@ def test_fused_rht_matches_oracle_and_separate_calls(signs, dtype):
     assert torch.equal(codes, c2) and torch.equal(scales, s2)
     assert np.array_equal(ns.cpu().numpy(), nv["scales"])
     assert np.array_equal(nc.cpu().numpy(), nv["codes"])
+
+
+def test_fused_grid_barrier_times_out_cleanly():
+    """Failure detection without a fault: an arrival counter preset so that
+    no block is ever the last to arrive means nobody releases the grid
+    barrier.  Every block's wait is bounded (1 s of the global timer); the
+    kernel must end with IF4_DEV_TIMEOUT in the error word, write no codes,
+    and leave the context usable: with the words zeroed again, the next call
+    is correct."""
+    import time
+    b = B()
+    x = workloads.llm_weight(6, rows=256, cols=1024).cuda()
+    sync = torch.zeros(b.FUSED_SYNC_WORDS, dtype=torch.int32, device="cuda")
+    sync[0] = 1 << 30                      # arrivals never reach gridDim - 1
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    codes = torch.full((256, 512), 0xAB, dtype=torch.uint8, device="cuda")
+    scales = torch.full((256, 64), 0xAB, dtype=torch.uint8, device="cuda")
+    ts = torch.zeros(1, dtype=torch.float32, device="cuda")
+    t0 = time.time()
+    b.if4_quantize_fused(x, codes, scales, None, None, ts, sync, err)
+    torch.cuda.synchronize()
+    waited = time.time() - t0
+    assert int(err.item()) & b.DEV_TIMEOUT
+    assert 0.5 < waited < 30, waited
+    assert torch.all(codes == 0xAB) and torch.all(scales == 0xAB)
+    # the context still works
+    sync.zero_()
+    err.zero_()
+    (c2, s2, t2), e2 = fused(x, sync=sync, with_nvfp4=False)
+    ref = oracle.quantize_tensor(x.float().cpu().numpy())
+    assert e2 == 0 and np.array_equal(c2, ref["codes"]) and np.array_equal(s2, ref["scales"])
