@@ -19,7 +19,9 @@
 //   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 accumulators)
 //               and one thread issues tcgen05.mma (M=128, N=256, K=16)
 //   warps 2-5   epilogue: tcgen05.ld of the finished accumulator, scale,
-//               bf16 RNE, global stores; the next tile's MMAs run meanwhile
+//               bf16 RNE, global stores; the next tile's MMAs run meanwhile.
+//               With the IF4 output (QOUT) they also encode each row's
+//               16-column groups with the quantizer's group encoder.
 // Every mbarrier wait is bounded by a wall-clock limit; on expiry the kernel
 // sets IF4_DEV_TIMEOUT in the error word, stops issuing work, drains what is
 // in flight (bounded), frees its tensor memory and returns.

@@ -15,7 +15,15 @@
 // thread's registers, and the outputs are one 8-byte code store and one scale
 // byte.  Lanes of a warp own consecutive groups, so each warp-wide load or
 // store touches one contiguous span.  A grid-stride loop keeps the next
-// group's load in flight while the current one is computed.
+// group's load in flight while the current one is computed.  The group
+// encoder itself (block scale, candidates, decision) is in if4_encode.cuh,
+// shared with the linear's IF4-output epilogue.
+//
+// Kernels here: the tensor amax and tensor scale; the quantizer for IF4 and
+// its comparators (NVFP4, NVINT4, 4/6), optionally on the random-sign
+// Hadamard transform; the single-launch quantizer (amax, grid barrier, encode)
+// in one cooperative launch; the dequantizer and the fp16 operand decode of
+// the linear.
 
 #include <cuda_runtime.h>
 
@@ -1065,14 +1073,6 @@ int launch_quant(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
     return launch_status();
 }
 
-template <int DT, int MODE, bool RHT>
-int dispatch_quant_dt(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
-                      const float *ts, int *err, int check_ts, cudaStream_t st,
-                      const DeviceInfo &d, const SignMasks &sm, uint32_t signs)
-{
-    return launch_quant<DT, MODE, RHT>(s, x, codes, scales, ts, err, check_ts, st, d, sm, signs);
-}
-
 template <int MODE, bool RHT>
 int dispatch_quant(int dt, const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
                    const float *ts, int *err, int check_ts, cudaStream_t st, const DeviceInfo &d,
@@ -1081,13 +1081,13 @@ int dispatch_quant(int dt, const Shape &s, const void *x, uint8_t *codes, uint8_
     const SignMasks sm = sign_masks(dt, signs);
     switch (dt) {
     case IF4_F32:
-        return dispatch_quant_dt<DT_F32, MODE, RHT>(s, x, codes, scales, ts, err, check_ts, st, d,
+        return launch_quant<DT_F32, MODE, RHT>(s, x, codes, scales, ts, err, check_ts, st, d,
                                                     sm, signs);
     case IF4_BF16:
-        return dispatch_quant_dt<DT_BF16, MODE, RHT>(s, x, codes, scales, ts, err, check_ts, st,
+        return launch_quant<DT_BF16, MODE, RHT>(s, x, codes, scales, ts, err, check_ts, st,
                                                      d, sm, signs);
     default:
-        return dispatch_quant_dt<DT_F16, MODE, RHT>(s, x, codes, scales, ts, err, check_ts, st, d,
+        return launch_quant<DT_F16, MODE, RHT>(s, x, codes, scales, ts, err, check_ts, st, d,
                                                     sm, signs);
     }
 }
