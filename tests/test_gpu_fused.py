@@ -174,3 +174,13 @@ def test_fused_grid_barrier_times_out_cleanly():
     (c2, s2, t2), e2 = fused(x, sync=sync, with_nvfp4=False)
     ref = oracle.quantize_tensor(x.float().cpu().numpy())
     assert e2 == 0 and np.array_equal(c2, ref["codes"]) and np.array_equal(s2, ref["scales"])
+
+
+@pytest.mark.parametrize("name", ["activation_bf16_8192x8192", "gradient_bf16_16384x4096"])
+def test_fused_full_size_workloads(name):
+    """The single launch at the full sizes of the large workloads (one
+    134 MB bf16 tensor each): every code, scale byte and the tensor scale
+    against the oracle, and the NVFP4 output too."""
+    x = (workloads.activation_outliers(0) if name.startswith("activation")
+         else workloads.hadamard_gradient(0))
+    check(x, name)

@@ -201,3 +201,28 @@ def test_linear_quantized_output_flags_invalid_scale():
                             err_flag=err)
     torch.cuda.synchronize()
     assert int(err.item()) & bb.DEV_BAD_SCALE
+
+
+def test_linear_quantized_output_full_workload():
+    """The IF4 output of the 8192 x 4096 x 4096 linear, every group, against
+    the oracle's quantization of the same bf16 C under the same scale."""
+    bb = B()
+    M, N, K = 8192, 4096, 4096
+    a, b = workloads.linear_operands(0, M=M, N=N, K=K)
+    aq, bq = _quantized(a), _quantized(b)
+    c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    codes = torch.empty((M, N // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((M, N // 16), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(bb.if4_linear_workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    c_ts = torch.ones(1, dtype=torch.float32, device="cuda")
+    bb.if4_linear(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], ws, c, err)
+    bb.if4_tensor_amax(c, c_ts, err)
+    bb.if4_tensor_scale(c_ts, c_ts)
+    bb.if4_linear_quantized(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], ws, codes, scales, c_ts,
+                            err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ref = oracle.quantize(c.float().cpu().numpy(), np.float32(c_ts.item()))
+    assert np.array_equal(scales.cpu().numpy(), ref["scales"])
+    assert np.array_equal(codes.cpu().numpy(), ref["codes"])
