@@ -53,7 +53,7 @@ def parse():
     p.add_argument("--kernel-only", default=None,
                    choices=["amax", "if4_quantize", "if4_dequantize", "nvfp4_quantize", "gemm",
                             "nvint4_quantize", "nvfp4_4over6_quantize", "if4_quantize_rht",
-                            "if4_decode_f16", "fused_quantize"],
+                            "if4_decode_f16", "fused_quantize", "fused_quantize_rht"],
                    help="launch only this kernel, warmup+steps times (for ncu captures)")
     return p.parse_args()
 
@@ -275,6 +275,7 @@ class Step:
                 ncodes=torch.empty((self.rows, self.cols // 2), dtype=torch.uint8, device=dev),
                 nscales=torch.empty((self.rows, self.cols // 16), dtype=torch.uint8, device=dev),
                 sync=torch.zeros(64, dtype=torch.int32, device=dev),
+                ts_rht=torch.empty(1, dtype=torch.float32, device=dev),
             )
             self.sets.append(s)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -286,7 +287,8 @@ class Step:
         s = self.sets[0]
         return sum(t.numel() * t.element_size() for t in s.values())
 
-    EXTRA = ["nvint4_quantize", "nvfp4_4over6_quantize", "if4_quantize_rht", "if4_decode_f16"]
+    EXTRA = ["nvint4_quantize", "nvfp4_4over6_quantize", "if4_quantize_rht", "if4_decode_f16",
+             "fused_quantize_rht"]
 
     def run_one(self, name, i):
         b, s = self.b, self.sets[i % len(self.sets)]
@@ -299,6 +301,12 @@ class Step:
         if name == "if4_quantize_rht":
             b.if4_quantize_rht(s["x"], RHT_SIGNS, s["ncodes"], s["nscales"], s["ts"], b.TS_GIVEN,
                                self.err)
+            return
+        if name == "fused_quantize_rht":
+            # its own tensor scale: the transformed tensor's must not replace
+            # the one the step and the quality report use
+            b.if4_quantize_fused(s["x"], s["codes"], s["scales"], s["ncodes"], s["nscales"],
+                                 s["ts_rht"], s["sync"], self.err, signs=RHT_SIGNS)
             return
         if name == "if4_decode_f16":
             b.if4_decode_f16(s["codes"], s["scales"], s["y"].view(torch.float16))
@@ -389,7 +397,8 @@ def kernel_table(ms, n_elem, in_bytes, pk):
     dq_bytes = n_elem // 2 + n_elem // 16 + 2 * n_elem
     # the single-launch quantizer: x once, IF4 and NVFP4 codes and scales
     fused_bytes = in_bytes + 2 * (n_elem // 2 + n_elem // 16)
-    nbytes = {"fused_quantize": fused_bytes, "amax": in_bytes, "scale": 8,
+    nbytes = {"fused_quantize": fused_bytes, "fused_quantize_rht": fused_bytes,
+              "amax": in_bytes, "scale": 8,
               "if4_quantize": q_bytes, "if4_dequantize": dq_bytes,
               "nvfp4_quantize": q_bytes, "nvint4_quantize": q_bytes,
               "nvfp4_4over6_quantize": q_bytes, "if4_quantize_rht": q_bytes,
