@@ -186,6 +186,23 @@ __device__ __forceinline__ unsigned long long f2_from_bf16x2(uint32_t w)
     return r;
 }
 
+// Programmatic dependent launch, at the top of a kernel: the next kernel in
+// the stream may be scheduled from now on (its blocks wait in the same
+// call), then wait until every earlier kernel this one depends on has
+// finished and its memory is visible.  The wait is a no-op when the kernel
+// was launched without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_enter()
+{
+    asm volatile("griddepcontrol.launch_dependents;\n\tgriddepcontrol.wait;" ::: "memory");
+}
+
+// Let the next kernel in the stream be scheduled (it still waits for this
+// one to finish before reading anything).
+__device__ __forceinline__ void pdl_release()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Wall clock in nanoseconds, for bounded waits.
 __device__ __forceinline__ unsigned long long globaltimer_ns()
 {

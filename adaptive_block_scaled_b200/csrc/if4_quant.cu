@@ -495,6 +495,7 @@ quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr,
                        uint8_t *__restrict__ scales, const float *__restrict__ ts_ptr, int *err,
                        int check_ts, const __grid_constant__ SignMasks sm, uint32_t signs)
 {
+    pdl_enter();
     constexpr int GB = 16 * elem_bytes<DT>();
     const float ts = *ts_ptr;
     if (check_ts && blockIdx.x == 0 && threadIdx.x == 0 && !ts_valid(ts) && err)
@@ -566,6 +567,7 @@ __global__ void __launch_bounds__(256)
 amax_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, uint32_t ngroups,
             int contig, unsigned int *amax_bits, int *err, const __grid_constant__ SignMasks sm)
 {
+    pdl_enter();
     constexpr int GB = 16 * elem_bytes<DT>();
     constexpr int U = DT == DT_F32 ? 4 : 8;
     uint32_t m = 0;
@@ -618,6 +620,7 @@ __device__ __forceinline__ float tensor_scale_of(float a)
 
 __global__ void tensor_scale_kernel(const float *amax, float *ts)
 {
+    pdl_enter();
     *ts = tensor_scale_of(*amax);
 }
 
@@ -734,7 +737,9 @@ quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr
     __syncthreads();
     if (!ok_sh) return;
 
-    // pass 2: the encode, as quantize_kernel
+    // pass 2: the encode, as quantize_kernel; the next kernel in the stream
+    // may be scheduled as this grid's blocks finish
+    pdl_release();
     const float ts = ts_sh;
     if (threadIdx.x < 128) {
         const float eff = __fmul_rn(f32_from_e4m3(threadIdx.x), ts);
@@ -866,6 +871,7 @@ dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__
                   const float *__restrict__ ts_ptr, uint32_t gpr, uint32_t ngroups,
                   char *__restrict__ y, int64_t ld_bytes, int contig)
 {
+    pdl_enter();
     constexpr int OB = ODT == DT_F32 ? 4 : 2;
     __shared__ __align__(128) float lut[32];
     if (threadIdx.x < 32) lut[threadIdx.x] = code_value(threadIdx.x);
@@ -986,6 +992,27 @@ int launch_status()
     return cudaGetLastError() == cudaSuccess ? IF4_OK : IF4_ERR_CUDA;
 }
 
+// Launch of the stream-ordered kernels (amax, scale, quantize, dequantize)
+// with programmatic dependent launch: each such kernel lets the next one be
+// scheduled while it drains, and waits for its predecessor's results before
+// reading anything (pdl_enter), so stream order holds as usual.
+template <typename... KArgs, typename... Args>
+int launch_k(void (*k)(KArgs...), unsigned grid, unsigned block, cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(block, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k, args...) != cudaSuccess) return IF4_ERR_CUDA;
+    return launch_status();
+}
+
 // Blocks to launch: enough for every work item, capped at one full wave of
 // resident blocks (the kernels are grid-stride loops).  `occ` is the number
 // of resident blocks per SM, queried once per kernel instantiation.
@@ -1023,9 +1050,8 @@ int launch_amax(const Shape &s, const void *x, unsigned int *amax_bits, int *err
     auto k = amax_kernel<DT, V8, RHT>;
     static const int occ = resident_blocks(k, 256);
     const uint32_t grid = grid_for(occ, d, s.ngroups, 256);
-    k<<<grid, 256, 0, st>>>(static_cast<const char *>(x), s.ld_bytes, s.gpr, s.ngroups,
-                            s.contig ? 1 : 0, amax_bits, err, sm);
-    return launch_status();
+    return launch_k(k, grid, 256, st, static_cast<const char *>(x), s.ld_bytes, s.gpr, s.ngroups,
+                    s.contig ? 1 : 0, amax_bits, err, sm);
 }
 
 template <int DT, bool RHT>
@@ -1063,14 +1089,11 @@ int launch_quant(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
     auto launch = [&](auto k) {
         static const int occ = resident_blocks(k, 256);
         const uint32_t grid = grid_for(occ, d, s.ngroups, 256);
-        k<<<grid, 256, 0, st>>>(static_cast<const char *>(x), s.ld_bytes, s.gpr, s.ngroups,
-                                s.contig ? 1 : 0, codes, scales, ts, err, check_ts, sm, signs);
+        return launch_k(k, grid, 256, st, static_cast<const char *>(x), s.ld_bytes, s.gpr,
+                        s.ngroups, s.contig ? 1 : 0, codes, scales, ts, err, check_ts, sm, signs);
     };
-    if (s.v8)
-        launch(quantize_kernel<DT, MODE, true, RHT, PF>);
-    else
-        launch(quantize_kernel<DT, MODE, false, RHT, PF>);
-    return launch_status();
+    return s.v8 ? launch(quantize_kernel<DT, MODE, true, RHT, PF>)
+                : launch(quantize_kernel<DT, MODE, false, RHT, PF>);
 }
 
 template <int MODE, bool RHT>
@@ -1119,8 +1142,7 @@ int quantize_entry(const void *x, int x_dtype, int64_t rows, int64_t cols, int64
         rc = dispatch_amax(x_dtype, s, x, reinterpret_cast<unsigned int *>(ts), err_flag, st, d,
                            rht);
         if (rc != IF4_OK) return rc;
-        tensor_scale_kernel<<<1, 1, 0, st>>>(ts, ts);
-        rc = launch_status();
+        rc = launch_k(tensor_scale_kernel, 1, 1, st, (const float *)ts, ts);
         if (rc != IF4_OK) return rc;
     }
     return dispatch_quant<MODE, RHT>(x_dtype, s, x, codes, scales, ts, err_flag,
@@ -1179,15 +1201,12 @@ int launch_dequant(const Shape &s, const uint8_t *codes, const uint8_t *scales, 
     auto launch = [&](auto k) {
         static const int occ = resident_blocks(k, 256);
         const uint32_t grid = grid_for(occ, d, s.ngroups, 256);
-        k<<<grid, 256, 0, st>>>(codes, scales, ts, s.gpr, s.ngroups, static_cast<char *>(y),
-                                s.ld_bytes, s.contig ? 1 : 0);
+        return launch_k(k, grid, 256, st, codes, scales, ts, s.gpr, s.ngroups,
+                        static_cast<char *>(y), s.ld_bytes, s.contig ? 1 : 0);
     };
     // 32-byte aligned base and rows: 256-bit stores
-    if (s.v8)
-        launch(dequantize_kernel<ODT, UNIT_TS, true>);
-    else
-        launch(dequantize_kernel<ODT, UNIT_TS, false>);
-    return launch_status();
+    return s.v8 ? launch(dequantize_kernel<ODT, UNIT_TS, true>)
+                : launch(dequantize_kernel<ODT, UNIT_TS, false>);
 }
 
 template <bool RHT>
@@ -1212,8 +1231,7 @@ int fused_entry(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t 
     if (s.ngroups == 0) {
         // an empty tensor: amax 0, ts 1, nothing to encode
         if (cudaMemsetAsync(ts, 0, sizeof(float), st) != cudaSuccess) return IF4_ERR_CUDA;
-        tensor_scale_kernel<<<1, 1, 0, st>>>(ts, ts);
-        return launch_status();
+        return launch_k(tensor_scale_kernel, 1, 1, st, (const float *)ts, ts);
     }
     const SignMasks sm = sign_masks(x_dtype, signs);
     switch (x_dtype) {
@@ -1259,8 +1277,7 @@ int if4_tensor_scale(const float *amax, float *ts, void *stream)
     DeviceInfo d;
     int rc = check_device(d);
     if (rc != IF4_OK) return rc;
-    tensor_scale_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(amax, ts);
-    return launch_status();
+    return launch_k(tensor_scale_kernel, 1, 1, static_cast<cudaStream_t>(stream), amax, ts);
 }
 
 int if4_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,

@@ -184,3 +184,24 @@ def test_fused_full_size_workloads(name):
     x = (workloads.activation_outliers(0) if name.startswith("activation")
          else workloads.hadamard_gradient(0))
     check(x, name)
+
+
+def test_fused_then_dequantize_in_stream_order():
+    """The step's sequence: the dequantizer (launched with programmatic
+    dependent launch) right after the single launch on the same stream must
+    read the finished codes, scales and tensor scale: bit-identical to the
+    oracle's dequantization, repeated on several tensors back to back."""
+    b = B()
+    sync = torch.zeros(b.FUSED_SYNC_WORDS, dtype=torch.int32, device="cuda")
+    outs = []
+    xs = [workloads.llm_weight(s, rows=1024, cols=4096) for s in range(3)]
+    for x in xs:
+        codes, scales, ts, nc, ns = b.quantize_fused(x.cuda(), sync_words=sync)
+        y = b.dequantize(codes, scales, ts, dtype=torch.float32)
+        outs.append((y, ts))
+    torch.cuda.synchronize()
+    for x, (y, ts) in zip(xs, outs):
+        ref = oracle.quantize_tensor(x.float().numpy())
+        want = oracle.dequantize(ref["codes"], ref["scales"], ref["ts"])
+        assert np.float32(ts.item()) == ref["ts"]
+        assert np.array_equal(y.cpu().numpy().view(np.uint32), want.view(np.uint32))
