@@ -683,6 +683,8 @@ quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr
                       uint8_t *__restrict__ nv_scales, float *ts_out, uint32_t *sync, int *err,
                       const __grid_constant__ SignMasks sm, uint32_t signs)
 {
+    // wait for the previous kernel in the stream (programmatic launch)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     constexpr int GB = 16 * elem_bytes<DT>();
     __shared__ float inv_tab[128];
     __shared__ uint32_t warp_max[8];
@@ -1164,11 +1166,13 @@ int launch_fused(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
     cfg.blockDim = dim3(256, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, k, static_cast<const char *>(x), s.ld_bytes, s.gpr, s.ngroups,
                            s.contig ? 1 : 0, codes, scales, nv_codes, nv_scales, ts, sync, err, sm,
                            signs) != cudaSuccess)
