@@ -706,9 +706,11 @@ def run_ours(args):
         line["e2e"] = measure_e2e(x_cpu, max(5, args.steps // 5), 2)
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(x_cpu, args.cpu_seconds)
-        if not args.no_linear and hasattr(step.b.lib, "if4_linear"):
+        # single-GPU reports: only at N = 1, so that with N > 1 the other
+        # ranks do not wait long at the final barrier
+        if not args.no_linear and world == 1 and hasattr(step.b.lib, "if4_linear"):
             line["linear"] = linear_report(pk)
-        if not args.no_large:
+        if not args.no_large and world == 1:
             del step, graphs_keep
             torch.cuda.empty_cache()
             line["large_workloads"] = large_workloads(pk)
