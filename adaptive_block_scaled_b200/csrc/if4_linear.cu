@@ -326,7 +326,6 @@ gemm_f16_tcgen05(const __grid_constant__ CUtensorMap tmap_a,
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    if constexpr (QOUT) out_inv_table(inv_tab, c_ts, err);
     const TileIter it{(M + BM - 1) / BM, (N + BN - 1) / BN,
                       ((M + BM - 1) / BM) * ((N + BN - 1) / BN)};
     const int k_blocks = (K + BK - 1) / BK;
@@ -356,6 +355,13 @@ gemm_f16_tcgen05(const __grid_constant__ CUtensorMap tmap_a,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // programmatic launch: nothing above reads a kernel input; wait here
+    // until the kernel before this one (the operand decode) has finished
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if constexpr (QOUT) {
+        out_inv_table(inv_tab, c_ts, err);
+        __syncthreads();
+    }
 
     if (warp == 0 && lane == 0) {
         // ---------------------------------------------------- TMA producer
@@ -569,7 +575,6 @@ gemm_f16_tcgen05_2sm(const __grid_constant__ CUtensorMap tmap_a,
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     float *inv_tab = reinterpret_cast<float *>(smem + PSTAGES * PSTAGE_BYTES + 256);
-    if constexpr (QOUT) out_inv_table(inv_tab, c_ts, err);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -608,6 +613,12 @@ gemm_f16_tcgen05_2sm(const __grid_constant__ CUtensorMap tmap_a,
     cluster_sync();                      // peer barriers initialised before any remote use
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // programmatic launch: nothing above reads a kernel input
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if constexpr (QOUT) {
+        out_inv_table(inv_tab, c_ts, err);
+        __syncthreads();
+    }
 
     if (warp == 0 && lane == 0) {
         // ---------------------------------------------------- TMA producer
@@ -812,11 +823,13 @@ int launch_gemm_t(const void *a, const void *b, const float *a_ts, const float *
         cfg.blockDim = dim3(NUM_THREADS, 1, 1);
         cfg.dynamicSmemBytes = pair::PSMEM_BYTES;
         cfg.stream = st;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         // persistent: as many pairs as can be resident at once (SM pairs
@@ -834,6 +847,7 @@ int launch_gemm_t(const void *a, const void *b, const float *a_ts, const float *
         if (pairs > sms / 2) pairs = sms / 2;
         if (tiles < pairs) pairs = tiles;
         cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+        cfg.numAttrs = 2;                  // the cluster shape, then programmatic launch
         if (cudaLaunchKernelEx(&cfg, kernel, ma, mb, a_ts, b_ts, c, (int)M, (int)N, (int)K, err,
                                o.c_codes, o.c_scales, o.c_ts) != cudaSuccess)
             return IF4_ERR_CUDA;
@@ -850,8 +864,19 @@ int launch_gemm_t(const void *a, const void *b, const float *a_ts, const float *
     if (attr_rc != cudaSuccess) return IF4_ERR_CUDA;
     const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = (int)(tiles < sms ? tiles : sms);
-    kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(ma, mb, a_ts, b_ts, c, (int)M, (int)N, (int)K,
-                                                  err, o.c_codes, o.c_scales, o.c_ts);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, ma, mb, a_ts, b_ts, c, (int)M, (int)N, (int)K, err,
+                           o.c_codes, o.c_scales, o.c_ts) != cudaSuccess)
+        return IF4_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? IF4_OK : IF4_ERR_CUDA;
 }
 
