@@ -449,3 +449,34 @@ def test_rht_quantize_dtypes_shapes_and_given_scale():
     w = torch.from_numpy(rng.standard_normal((256, 512)).astype(np.float32))
     check_rht(w, 0xBEEF, "given ts", ts=np.float32(float(w.abs().max()) / 2688.0 * 0.1))
     check_rht(torch.zeros((4, 64)), 0xFFFF, "zeros")
+
+
+@pytest.mark.parametrize("ts", [2.0 ** -117, 2.0 ** -100, 2.0 ** 100, 2.0 ** 117])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_extreme_given_scales(ts, dtype):
+    """Valid tensor scales at the ends of the allowed range, on rows whose
+    magnitudes run from float32 subnormals to 3e38.  Under a tiny ts most block
+    scales saturate at 448 and x * inv overflows the float32 range for large
+    rows (the INT4 clamp, the general path, infinite errors in the binary64
+    rule), while subnormal rows get ordinary block scales; under a huge ts most
+    block scales underflow to zero.  Codes and scale bytes must equal the
+    oracle's, for IF4 and for the comparators."""
+    rng = np.random.default_rng(int(np.log2(ts)) + 200)
+    x = rng.standard_normal((64, 512)).astype(np.float32)
+    # row magnitudes from float32 subnormals (2^-140) to near the top of the range
+    mags = np.exp2(np.array([-140, -130, -124, -118, -110, -60, 0, 60, 100], np.float64))
+    x *= mags[np.arange(64) % mags.size, None].astype(np.float32)
+    x[3, :16] = np.float32(3e38)
+    xt = torch.from_numpy(x).to(dtype)
+    x_np = xt.float().numpy()
+    ref = oracle.quantize(x_np, np.float32(ts))
+    c, s, t, err = gpu_quant(xt, "if4", ts=np.float32(ts))
+    assert err == 0
+    assert np.array_equal(s, ref["scales"]), (ts, dtype)
+    assert np.array_equal(c, ref["codes"]), (ts, dtype)
+    for mode, omode in (("nvfp4", oracle.MODE_NVFP4), ("nvint4", oracle.MODE_NVINT4),
+                        ("4over6", oracle.MODE_4OVER6)):
+        r2 = oracle.quantize(x_np, np.float32(ts), mode=omode)
+        c2, s2, _, e2 = gpu_quant(xt, mode, ts=np.float32(ts))
+        assert e2 == 0
+        assert np.array_equal(s2, r2["scales"]) and np.array_equal(c2, r2["codes"]), (mode, ts)
