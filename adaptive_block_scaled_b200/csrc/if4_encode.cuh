@@ -413,7 +413,12 @@ __device__ __forceinline__ GroupCode if4_finish(const If4Fast &f, float amax, fl
                                               const float *inv_tab, Fill fill)
 {
     GroupCode out;
-    if (f.general || f.near) {
+    // A near group whose two candidates take the same values (every element
+    // 0 or +-6 on both grids; in activations, groups holding one outlier)
+    // ties exactly and keeps FP4: decided from the code words alone, without
+    // the inputs.
+    if ((f.general || f.near) &&
+        (f.general || !(candidates_coincide(f.f0, f.i0) && candidates_coincide(f.f1, f.i1)))) {
         float y[16];
         fill(y);
         out = f.general ? if4_group_general(amax, ts, rts, inv_tab, y)
