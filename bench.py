@@ -327,13 +327,18 @@ class Step:
         else:
             raise ValueError(name)
 
-    def run(self, i):
+    def run(self, i, events=None):
         """One step on buffer set i: the single-launch quantizer (tensor amax,
         tensor scale, IF4 codes and the NVFP4 comparator), then the IF4
-        dequantizer to bf16."""
+        dequantizer to bf16.  events: optional pair recorded right before
+        and right after the quantizer launch."""
         b, s = self.b, self.sets[i % len(self.sets)]
+        if events is not None:
+            events[0].record()
         b.if4_quantize_fused(s["x"], s["codes"], s["scales"], s["ncodes"], s["nscales"], s["ts"],
                              s["sync"], self.err)
+        if events is not None:
+            events[1].record()
         b.if4_dequantize(s["codes"], s["scales"], s["ts"], s["y"])
 
     def run_unfused(self, i, events=None, side=None):
@@ -368,17 +373,21 @@ class Step:
             ev[5].record()
 
 
-def kernel_times(step, names, reps):
-    """Per-kernel times: one CUDA graph per kernel launching it once on every
-    buffer set in turn, replayed `reps` times between two events on the
-    replay stream; mean time per launch (ms)."""
+def kernel_times(step, names, reps, min_launches=32):
+    """Per-kernel times: one CUDA graph per kernel launching it on every
+    buffer set in turn, as many passes over the sets as make at least
+    `min_launches` launches (so that the gap at a graph boundary, where
+    programmatic dependent launch cannot overlap two launches, is a small
+    share), replayed `reps` times between two events on the replay stream;
+    mean time per launch (ms)."""
     out = {}
     sets = len(step.sets)
+    n = sets * max(1, -(-min_launches // sets))
     for name in names:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            for i in range(sets):
-                step.run_one(name, i)
+            for i in range(n):
+                step.run_one(name, i % sets)
         g.replay()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -387,9 +396,32 @@ def kernel_times(step, names, reps):
             g.replay()
         e1.record()
         torch.cuda.synchronize()
-        out[name] = e0.elapsed_time(e1) / (reps * sets)
+        out[name] = e0.elapsed_time(e1) / (reps * n)
         del g
     return out
+
+
+def quantizer_in_sequence(step, steps, sleep_cycles=int(4e7)):
+    """Launch durations of the step's dominant kernel, the single-launch
+    quantizer, inside the step sequence: the K steps launched on the stream
+    (not as a graph: an event-record node in a graph adds microseconds of its
+    own) with a timing event recorded right before and right after each
+    quantizer launch.  The stream is first held by a sleep of about 20 ms
+    so that the host has enqueued every step before the first one runs, and
+    no launch waits for the host.  Each quantizer launch then starts after
+    the previous dequantizer has finished (the event sits between them), so
+    these durations include the launch's own ramp.  Returns (mean, median)
+    over the K launches, in ms."""
+    before = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    after = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for rep in range(2):                      # the first pass warms up
+        torch.cuda.synchronize()
+        torch.cuda._sleep(sleep_cycles)
+        for i in range(steps):
+            step.run(i, events=(before[i], after[i]))
+        torch.cuda.synchronize()
+    t = np.array([b.elapsed_time(a) for b, a in zip(before, after)])
+    return float(t.mean()), float(np.median(t))
 
 
 def kernel_table(ms, n_elem, in_bytes, pk):
@@ -654,7 +686,8 @@ def run_ours(args):
     ms_unfused = start.elapsed_time(stop) / args.steps
     del uwarm, utimed
 
-    kern_ms = kernel_times(step, step.kernels, max(2, args.steps // sets))
+    kern_ms = kernel_times(step, step.kernels, 5)
+    seq_mean, seq_median = quantizer_in_sequence(step, args.steps)
     if int(step.err.item()) != 0:
         raise RuntimeError(f"device error flag {int(step.err.item())}")
     graphs_keep = timed
@@ -662,15 +695,16 @@ def run_ours(args):
     value = world * n_elem / (ms * 1e-3) / 1e9
     q_bytes = in_bytes + n_elem // 2 + n_elem // 16
     kernels = kernel_table(kern_ms, n_elem, in_bytes, pk)
-    extra = kernel_table(kernel_times(step, Step.EXTRA, max(2, args.steps // sets)), n_elem,
-                         in_bytes, pk)
+    extra = kernel_table(kernel_times(step, Step.EXTRA, 5), n_elem, in_bytes, pk)
 
     def roof(name, label):
         k = kernels[name]
         r = {"bound": "hbm", "kernel": label, "achieved": k["gbs"], "peak": pk["hbm_gbs"],
              "unit": "GB/s", "frac": k["gbs"] / pk["hbm_gbs"],
              "peak_source": f"{pk['source']} hbm_gbs (copy bandwidth, read+write; of measured)",
-             "algorithmic_bytes_per_launch": k["bytes"], "traffic": None}
+             "algorithmic_bytes_per_launch": k["bytes"], "traffic": None,
+             "timing": "CUDA events around a graph of at least 32 back-to-back launches over "
+                       "the buffer sets, on the launching stream; mean per launch"}
         traffic_file = os.path.join(ROOT, "profiles", "traffic.json")
         if os.path.exists(traffic_file):
             tr = json.load(open(traffic_file)).get(args.workload, {}).get(name)
@@ -681,6 +715,14 @@ def run_ours(args):
     # the dominant kernel of the step is the single-launch quantizer; the
     # IF4 quantizer alone (tensor scale given) is reported beside it
     roofline = roof("fused_quantize", "if4_quantize_fused (amax + scale + IF4 + NVFP4)")
+    # the same kernel inside the step: two bounds on its share of a timed step
+    roofline["in_step"] = {
+        "event_us_mean": seq_mean * 1e3, "event_us_median": seq_median * 1e3,
+        "event_note": "events on the stream around each quantizer launch of the timed steps "
+                      "run again eagerly; includes the launch latency the events expose",
+        "step_minus_dequantize_us": (ms - kern_ms["if4_dequantize"]) * 1e3,
+        "frac_at_step_minus_dequantize": kernels["fused_quantize"]["bytes"]
+        / ((ms - kern_ms["if4_dequantize"]) * 1e-3) / 1e9 / pk["hbm_gbs"]}
     roofline_if4 = roof("if4_quantize", "if4_quantize (tensor scale given)")
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -693,7 +735,7 @@ def run_ours(args):
                        "l2": f"rotating {sets} buffer sets, {sets * per_set / 1e6:.0f} MB "
                              f"(inputs {sets * in_bytes / 1e6:.0f} MB > 3x126 MB L2)",
                        "launch": "the timed steps as one CUDA graph; per-kernel times from "
-                                 "one graph per kernel over all sets",
+                                 "one graph per kernel of at least 32 launches over all sets",
                        "step": "single-launch quantizer (amax, scale, IF4 quantize, NVFP4 "
                                "quantize), then IF4 dequantize (bf16)"},
             "gpu_launches": step.launches_per_step * args.steps,
