@@ -155,16 +155,20 @@ __device__ __forceinline__ bool candidates_coincide(uint32_t fp4, uint32_t int4)
 
 // Binary64 squared-error sums of both candidates in element order: the
 // decision rule itself, used only when the binary32 margin of a group is too
-// small to trust.  It walks the group's 16 inputs y (in local memory, filled
-// by the caller's rare branch) one by one, so the common path keeps no extra
-// registers for it.  The INT4 integer is always clamped here; the clamp is
-// the identity whenever the fast path skipped it.
+// small to trust.  It takes the group's 16 inputs y from memory (filled by
+// the caller's rare branch), so the common path keeps no extra registers for
+// them; all 16 are loaded before the sums start, so that a local array that
+// has left L1 costs one round trip, not sixteen.  The INT4 integer is always
+// clamped here; the clamp is the identity whenever the fast path skipped it.
 __device__ __noinline__ bool int4_wins_exact(const float *y, float inv)
 {
+    float yv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) yv[i] = y[i];
     double ef = 0.0, ei = 0.0;
-#pragma unroll 1
+#pragma unroll
     for (int i = 0; i < 16; ++i) {
-        const float v = __fmul_rn(y[i], inv);
+        const float v = __fmul_rn(yv[i], inv);
         const uint32_t h = f16x2_from_e2m1x2(e2m1x2_from_f32(v, 0.0f));
         const float qf = f16lo_to_f32(h);
         float r = __fmaf_rn(v, c76(), kMagic);

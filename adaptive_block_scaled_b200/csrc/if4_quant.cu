@@ -327,20 +327,25 @@ __device__ __forceinline__ uint32_t fp4_word_values(const f2_t (&v)[4], f2_t (&q
 
 // Binary64 reconstruction errors of the two 4/6 candidates in element order
 // (the rule itself), for groups whose binary32 margin is within rounding.
+// The 16 inputs are all loaded before the sums start (one round trip).
 template <int DT>
 __device__ __noinline__ bool four_wins_exact(const char *p, float inv6, float eff6, float inv4,
                                              float eff4)
 {
-    double e6 = 0.0, e4 = 0.0;
-#pragma unroll 1
+    float xv[16];
+#pragma unroll
     for (int i = 0; i < 16; ++i) {
-        float x;
         if constexpr (DT == DT_F32)
-            x = __ldg(reinterpret_cast<const float *>(p) + i);
+            xv[i] = __ldg(reinterpret_cast<const float *>(p) + i);
         else if constexpr (DT == DT_BF16)
-            x = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(p) + i) << 16);
+            xv[i] = __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(p) + i) << 16);
         else
-            x = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short *>(p) + i)));
+            xv[i] = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short *>(p) + i)));
+    }
+    double e6 = 0.0, e4 = 0.0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float x = xv[i];
         const float q6 = f16lo_to_f32(f16x2_from_e2m1x2(e2m1x2_from_f32(__fmul_rn(x, inv6), 0.0f)));
         const float q4 = f16lo_to_f32(f16x2_from_e2m1x2(e2m1x2_from_f32(__fmul_rn(x, inv4), 0.0f)));
         const double d6 = __dsub_rn((double)x, (double)__fmul_rn(q6, eff6));
@@ -638,40 +643,55 @@ constexpr unsigned long long kGridWaitNs = 1000000000ull;   // 1 s
 // arrivals and sync[1] accumulates the float bits of the tensor amax (one
 // 128-byte line, written by the arriving blocks); sync[32] is the generation
 // and sync[33] carries ts to the other blocks (another line, polled by the
-// waiting blocks).  The last block to arrive computes ts, stores it to
-// *ts_out, puts sync[0] and sync[1] back to zero and moves the generation
-// on; the others wait (bounded) for the generation to move.  Called by one
-// thread per block.  Returns false (and sets IF4_DEV_TIMEOUT) when the wait
-// runs out.
-__device__ __noinline__ bool grid_tensor_scale(uint32_t *sync, uint32_t block_max_bits,
-                                               float *ts_out, int *err, float &ts)
+// waiting blocks, read and written as one 64-bit word).  Each arriving block
+// adds its maximum without waiting (a relaxed reduction) and then its
+// arrival with acquire-release order, so the last block to arrive sees every
+// maximum.  That block computes ts, stores it to *ts_out, puts sync[0] and
+// sync[1] back to zero and publishes the next generation together with ts in
+// one release store; the others poll that word (bounded) with acquire loads.
+// `gen0` is the generation the block read at its start: it cannot move before
+// every block, this one included, has arrived.  Called by one thread per
+// block.  Returns false (and sets IF4_DEV_TIMEOUT) when the wait runs out.
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t *p)
 {
-    volatile uint32_t *vs = sync;
-    if (block_max_bits != 0u) atomicMax(&sync[1], block_max_bits);
-    const uint32_t gen = vs[32];
-    __threadfence();
-    const uint32_t arrived = atomicAdd(&sync[0], 1u);
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __noinline__ bool grid_tensor_scale(uint32_t *sync, uint32_t gen0,
+                                               uint32_t block_max_bits, float *ts_out, int *err,
+                                               float &ts)
+{
+    if (block_max_bits != 0u)
+        asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;"
+                     :: "l"(sync + 1), "r"(block_max_bits) : "memory");
+    uint32_t arrived;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                 : "=r"(arrived) : "l"(sync) : "memory");
+    unsigned long long word;
     if (arrived == gridDim.x - 1) {
-        __threadfence();
-        const float t = tensor_scale_of(__uint_as_float(atomicAdd(&sync[1], 0u)));
+        const float t = tensor_scale_of(__uint_as_float(ld_relaxed_gpu(sync + 1)));
         *ts_out = t;
-        vs[33] = __float_as_uint(t);
-        vs[1] = 0u;
-        vs[0] = 0u;
-        __threadfence();
-        atomicAdd(&sync[32], 1u);
+        asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" :: "l"(sync + 1) : "memory");
+        asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" :: "l"(sync) : "memory");
+        word = ((unsigned long long)__float_as_uint(t) << 32) | (unsigned long long)(gen0 + 1u);
+        asm volatile("st.release.gpu.global.b64 [%0], %1;" :: "l"(sync + 32), "l"(word)
+                     : "memory");
     } else {
         const unsigned long long t0 = globaltimer_ns();
-        while (vs[32] == gen) {
+        for (;;) {
+            asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(word) : "l"(sync + 32)
+                         : "memory");
+            if ((uint32_t)word != gen0) break;
             if (globaltimer_ns() - t0 > kGridWaitNs) {
                 if (err) atomicOr(err, IF4_DEV_TIMEOUT);
                 return false;
             }
-            __nanosleep(200);
+            __nanosleep(100);
         }
-        __threadfence();
     }
-    ts = __uint_as_float(vs[33]);
+    ts = __uint_as_float((uint32_t)(word >> 32));
     return true;
 }
 
@@ -685,6 +705,7 @@ quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr
 {
     // wait for the previous kernel in the stream (programmatic launch)
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    const uint32_t gen0 = threadIdx.x == 0 ? ld_relaxed_gpu(sync + 32) : 0u;
     constexpr int GB = 16 * elem_bytes<DT>();
     __shared__ float inv_tab[128];
     __shared__ uint32_t warp_max[8];
@@ -733,7 +754,7 @@ quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr
         for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b = max(b, warp_max[w]);
         if (b >= 0x7F800000u && err) atomicOr(err, IF4_DEV_NONFINITE);
         float t = 1.0f;
-        ok_sh = grid_tensor_scale(sync, b, ts_out, err, t) ? 1 : 0;
+        ok_sh = grid_tensor_scale(sync, gen0, b, ts_out, err, t) ? 1 : 0;
         ts_sh = t;
     }
     __syncthreads();

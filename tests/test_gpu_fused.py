@@ -205,3 +205,40 @@ def test_fused_then_dequantize_in_stream_order():
         want = oracle.dequantize(ref["codes"], ref["scales"], ref["ts"])
         assert np.float32(ts.item()) == ref["ts"]
         assert np.array_equal(y.cpu().numpy().view(np.uint32), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("shape,dtype", [((4096, 4096), torch.bfloat16),
+                                         ((4096, 4192), torch.bfloat16),
+                                         ((4096, 4256), torch.bfloat16),
+                                         ((4096, 4096), torch.float16),
+                                         ((4096, 2048), torch.float32),
+                                         ((4096, 2112), torch.float32),
+                                         ((333, 4096), torch.bfloat16)])
+def test_fused_weight_sized_shapes(shape, dtype):
+    """Contiguous tensors of 1.4-17.4 M elements in each input type, around
+    the size of the weight workload, with an outlier channel and a row count
+    (333) that leaves a ragged last round of the grid: every code, scale byte
+    and the tensor scale against the oracle."""
+    g = torch.Generator().manual_seed(shape[0] + shape[1])
+    x = (torch.randn(shape, generator=g) * 0.02).to(dtype)
+    x[:, 7] *= 30                                   # an outlier channel
+    check(x, f"{shape} {dtype}")
+
+
+def test_fused_contiguous_and_strided_agree():
+    """The same weight tensor as a contiguous tensor and as a strided view
+    of a padded buffer (the two addressing paths of the kernel):
+    byte-identical outputs."""
+    b = B()
+    x = workloads.llm_weight(3)
+    pad = torch.zeros((4096, 4096 + 64), dtype=torch.bfloat16)
+    pad[:, :4096] = x
+    outs = []
+    for xd in (x.cuda(), pad.cuda()[:, :4096]):
+        sync = torch.zeros(b.FUSED_SYNC_WORDS, dtype=torch.int32, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        outs.append(b.quantize_fused(xd, sync_words=sync, err_flag=err))
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+    for a, c in zip(*outs):
+        assert torch.equal(a, c)
