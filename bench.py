@@ -411,12 +411,16 @@ def quantizer_in_sequence(step, steps, sleep_cycles=int(4e7)):
     no launch waits for the host.  Each quantizer launch then starts after
     the previous dequantizer has finished (the event sits between them), so
     these durations include the launch's own ramp.  Returns (mean, median)
-    over the K launches, in ms."""
+    over the K launches, in ms, or (None, None) when torch offers no sleep
+    kernel to hold the stream with."""
+    hold = getattr(torch.cuda, "_sleep", None)
+    if hold is None:                          # no way to hold the stream: no bound
+        return None, None
     before = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     after = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     for rep in range(2):                      # the first pass warms up
         torch.cuda.synchronize()
-        torch.cuda._sleep(sleep_cycles)
+        hold(sleep_cycles)
         for i in range(steps):
             step.run(i, events=(before[i], after[i]))
         torch.cuda.synchronize()
@@ -717,7 +721,8 @@ def run_ours(args):
     roofline = roof("fused_quantize", "if4_quantize_fused (amax + scale + IF4 + NVFP4)")
     # the same kernel inside the step: two bounds on its share of a timed step
     roofline["in_step"] = {
-        "event_us_mean": seq_mean * 1e3, "event_us_median": seq_median * 1e3,
+        "event_us_mean": None if seq_mean is None else seq_mean * 1e3,
+        "event_us_median": None if seq_median is None else seq_median * 1e3,
         "event_note": "events on the stream around each quantizer launch of the timed steps "
                       "run again eagerly; includes the launch latency the events expose",
         "step_minus_dequantize_us": (ms - kern_ms["if4_dequantize"]) * 1e3,
