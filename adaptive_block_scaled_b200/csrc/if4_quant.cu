@@ -939,6 +939,27 @@ dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__
         ld_nc_v2(codes + (int64_t)g * 8, a0, a1);
         as = ld_nc_u8(scales + g);
     }
+    // Full rounds of a contiguous output while both loads of the round are
+    // in range: no per-group range checks (a0, a1, as hold group g at the top
+    // of every round).  With it the kernel takes 39 registers (six resident
+    // blocks per SM instead of eight) and runs 8 % faster on 134 MB tensors
+    // (about 14 groups per thread); held to 32 registers it gains nothing.
+    // Taken from six groups per thread on; at 4096 x 4096 (3-4 groups per
+    // thread) the checked loop below does all the work.
+    if (contig && ngroups / stride >= 6u) {
+        while ((uint64_t)g + 2ull * stride < ngroups) {
+            uint32_t gn = g + stride;
+            ld_nc_v2(codes + (int64_t)gn * 8, b0, b1);
+            bs = ld_nc_u8(scales + gn);
+            dequant_group<ODT, UNIT_TS, V8>(a0, a1, as, ts, lut_addr, y + (int64_t)g * (16 * OB));
+            g = gn;
+            gn = g + stride;
+            ld_nc_v2(codes + (int64_t)gn * 8, a0, a1);
+            as = ld_nc_u8(scales + gn);
+            dequant_group<ODT, UNIT_TS, V8>(b0, b1, bs, ts, lut_addr, y + (int64_t)g * (16 * OB));
+            g = gn;
+        }
+    }
     while (g < ngroups) {
         uint32_t gn = g + stride;
         bool more = gn < ngroups && gn > g;
