@@ -529,8 +529,9 @@ quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr,
     if (PF == 2 && g + stride < ngroups) load_group<DT, V8>(addr(g + stride), buf[1]);
     // Full rounds of a contiguous tensor, while every load of the round is in
     // range: no per-group range checks.  Worth 6-8 % for the IF4 encode (one
-    // group in flight); the two-buffer loop of the single-candidate modes is
-    // left as it is (it was no faster this way).
+    // group in flight); the two-buffer loop of the single-candidate modes, and
+    // the single launch's encode pass (which spilled with it), are left as
+    // they are (they were no faster this way).
     if (PF == 1 && contig) {
         while ((uint64_t)g + (uint64_t)(2 * PF) * stride < ngroups) {
 #pragma unroll
@@ -787,20 +788,6 @@ quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr
     }
     const float rts = __frcp_rn(ts);
     __syncthreads();
-    // full rounds of a contiguous tensor without per-group range checks, as
-    // in quantize_kernel, then the rest with them
-    if (contig) {
-        while ((uint64_t)g + 2ull * stride < ngroups) {
-#pragma unroll
-            for (int ph = 0; ph < 2; ++ph) {
-                load_group<DT, V8>(x + (int64_t)(g + stride) * GB, buf[ph ^ 1]);
-                quantize_one<DT, Q_IF4, RHT, NV>(buf[ph], g, x, ld_bytes, gpr_eff, ts, rts,
-                                                 inv_tab, nullptr, codes, scales, sm, signs,
-                                                 nv_codes, nv_scales);
-                g += stride;
-            }
-        }
-    }
     for (; g < ngroups;) {
 #pragma unroll
         for (int ph = 0; ph < 2; ++ph) {
