@@ -139,3 +139,48 @@ def test_rht_then_quantize_is_quantize_of_the_transform():
     r = oracle.quantize_tensor(oracle.rht(x, 0x5A5A))
     assert q["ts"] == r["ts"]
     assert np.array_equal(q["codes"], r["codes"]) and np.array_equal(q["scales"], r["scales"])
+
+
+def test_four_over_six_equal_errors_keep_six():
+    """Equal errors keep the amax/6 scale (reading R22).  ts = 1 and
+    x = [6, 3, -6, 0, ...] are exact under both candidate scales: E4M3 1.0
+    from amax/6 puts them on the grid as 6, 3, -6, and E4M3 1.5 from amax/4
+    scales them to 4, 2, -4, which decode back to 6, 3, -6.  Both errors are
+    zero, so the /6 scale (code 0x38) and its codes must be kept."""
+    x = np.zeros((1, 16), np.float32)
+    x[0, :3] = [6.0, 3.0, -6.0]
+    q = oracle.quantize(x, np.float32(1.0), mode=oracle.MODE_4OVER6)
+    assert q["e_fp"][0, 0] == 0.0 and q["e_int"][0, 0] == 0.0
+    assert int(q["scales"][0, 0]) == 0x38           # E4M3 1.0, not 1.5 (0x3C)
+    assert list(unpack(q["codes"][0])[:3]) == [0x7, 0x5, 0xF]
+
+
+def _rht_f32(x16, signs, order):
+    y = np.array([-v if (signs >> j) & 1 else v for j, v in enumerate(x16)], np.float32)
+    for h in order:
+        for i in range(16):
+            if not i & h:
+                a, b = y[i], y[i + h]
+                y[i], y[i + h] = np.float32(a + b), np.float32(a - b)
+    return (y * np.float32(0.25)).astype(np.float32)
+
+
+def test_rht_butterfly_stage_order():
+    """Reading R23 fixes the butterfly stages h = 1, 2, 4, 8 in that order.
+    The opposite order is the same transform in exact arithmetic but rounds
+    differently in binary32.  On seeded groups where the two orders give
+    different binary32 results, the oracle must give the stated order's."""
+    rng = np.random.default_rng(11)
+    signs = 0x6A1D
+    found = 0
+    for _ in range(2000):
+        x = (rng.standard_normal(16) * np.exp2(rng.integers(-3, 4, 16))).astype(np.float32)
+        fwd = _rht_f32(x, signs, (1, 2, 4, 8))
+        if np.array_equal(fwd, _rht_f32(x, signs, (8, 4, 2, 1))):
+            continue
+        got = oracle.rht(x[None, :], signs)[0]
+        assert np.array_equal(got.view(np.uint32), fwd.view(np.uint32)), x
+        found += 1
+        if found == 20:
+            break
+    assert found == 20
