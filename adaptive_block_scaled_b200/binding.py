@@ -56,6 +56,8 @@ def _load():
                                _vp],
         "if4_quantize_fused_rht": [_vp, _int, _i64, _i64, _i64, ctypes.c_uint32, _vp, _vp, _vp,
                                    _vp, _vp, _vp, _vp, _vp],
+        "if4_quantize_fused_dequant": [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp,
+                                       _vp, _vp, _vp, _vp],
         "if4_decode_f16": [_vp, _vp, _i64, _i64, _vp, _vp],
         "if4_gemm_f16": [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
         "if4_linear_workspace_bytes": [_i64, _i64, _i64],
@@ -322,6 +324,50 @@ def quantize_rht(x, signs, ts=None, err_flag=None, stream=None):
         ts_t, ts_mode = ts, TS_GIVEN
     if4_quantize_rht(x, signs, codes, scales, ts_t, ts_mode, err_flag, stream)
     return codes, scales, ts_t
+
+
+def if4_quantize_fused_dequant(x, codes, scales, nv_codes, nv_scales, ts, sync_words, y,
+                               err_flag=None, stream=None):
+    """The single launch that also writes y, the bf16 decode of its IF4 codes
+    (dense, 32-byte aligned)."""
+    rows, cols, ld = _matrix(x, "x")
+    _u8(codes, "codes", (rows, cols // 2))
+    _u8(scales, "scales", (rows, cols // 16))
+    if (nv_codes is None) != (nv_scales is None):
+        raise ValueError("nv_codes and nv_scales go together")
+    if nv_codes is not None:
+        _u8(nv_codes, "nv_codes", (rows, cols // 2))
+        _u8(nv_scales, "nv_scales", (rows, cols // 16))
+    if sync_words.dtype != torch.int32 or sync_words.numel() < FUSED_SYNC_WORDS:
+        raise ValueError(f"sync_words must be an int32 device tensor of at least "
+                         f"{FUSED_SYNC_WORDS} elements")
+    if y.dtype != torch.bfloat16 or tuple(y.shape) != (rows, cols) or not y.is_contiguous():
+        raise ValueError("y must be a dense bf16 tensor of the shape of x")
+    _check(lib.if4_quantize_fused_dequant(_ptr(x), _dtype(x, "x"), rows, cols, ld, _ptr(codes),
+                                          _ptr(scales), _ptr(nv_codes), _ptr(nv_scales),
+                                          _ptr(ts), _ptr(sync_words), _ptr(y), _ptr(err_flag),
+                                          _stream(stream)),
+           "if4_quantize_fused_dequant")
+
+
+def quantize_fused_dequant(x, with_nvfp4=True, sync_words=None, err_flag=None, stream=None):
+    """The quantize-then-dequantize round trip in one launch.  Returns
+    (codes, scales, ts, y) or (codes, scales, ts, nv_codes, nv_scales, y)."""
+    rows, cols, _ = _matrix(x, "x")
+    dev = x.device
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+    nv_codes = torch.empty_like(codes) if with_nvfp4 else None
+    nv_scales = torch.empty_like(scales) if with_nvfp4 else None
+    ts = torch.empty(1, dtype=torch.float32, device=dev)
+    y = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
+    if sync_words is None:
+        sync_words = torch.zeros(FUSED_SYNC_WORDS, dtype=torch.int32, device=dev)
+    if4_quantize_fused_dequant(x, codes, scales, nv_codes, nv_scales, ts, sync_words, y,
+                               err_flag, stream)
+    if with_nvfp4:
+        return codes, scales, ts, nv_codes, nv_scales, y
+    return codes, scales, ts, y
 
 
 def quantize_fused(x, with_nvfp4=True, sync_words=None, err_flag=None, stream=None, signs=None):

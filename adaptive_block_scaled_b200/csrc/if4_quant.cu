@@ -439,16 +439,117 @@ __device__ __forceinline__ GroupCode encode_if4(const f2_t (&xv)[8], float amax,
     });
 }
 
+// ------------------------------------------ group decode (dequantizer) ----
+
+template <int ODT>
+__device__ __forceinline__ uint32_t pack_out2(float a, float b)
+{
+    if constexpr (ODT == DT_BF16) return bf16x2_from_f32(a, b);
+    else return f16x2_from_f32(a, b);
+}
+
+// Decoded value of every code: lut[n] is the FP4 value of nibble n,
+// lut[16 + n] the INT4 value fl(6k/7) of nibble n (k its sign extension).
+// 32 floats, one per shared-memory bank, so any pattern of lookups by a warp
+// is conflict-free.
+__device__ __forceinline__ float code_value(uint32_t i)
+{
+    if (i < 16) {
+        const uint32_t h = f16x2_from_e2m1x2(i);      // nibble in bits 0-3
+        return f16lo_to_f32(h);
+    }
+    const float k = (float)((int)((i - 16) ^ 8u) - 8);
+    return __fmul_rn(k, c67());
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+// 8 decoded values (not yet scaled) of the 8 nibbles of w; base is the
+// shared address of lut or lut + 16 floats.
+__device__ __forceinline__ void decode_word(uint32_t w, uint32_t base, float (&q)[8])
+{
+    q[0] = lds_f32(base + ((w << 2) & 0x3Cu));
+#pragma unroll
+    for (int i = 1; i < 8; ++i) q[i] = lds_f32(base + ((w >> (4 * i - 2)) & 0x3Cu));
+}
+
+// Decode one group (code words w0, w1, scale byte sb) and store its 16
+// outputs at p.
+template <int ODT, bool UNIT_TS, bool V8 = false>
+__device__ __forceinline__ void dequant_group(uint32_t w0, uint32_t w1, uint32_t sb, float ts,
+                                              uint32_t lut_addr, char *p)
+{
+    const float e4 = f32_from_e4m3(sb);
+    const float eff = UNIT_TS ? e4 : __fmul_rn(e4, ts);
+    const uint32_t base = lut_addr + ((sb >> 1) & 0x40u);        // INT4 half for bit 7
+    float qa[8], qb[8];
+    decode_word(w0, base, qa);
+    decode_word(w1, base, qb);
+    const f2_t EFF = f2_pack(eff, eff);
+    f2_t ya[4], yb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        ya[j] = f2_mul(f2_pack(qa[2 * j], qa[2 * j + 1]), EFF);
+        yb[j] = f2_mul(f2_pack(qb[2 * j], qb[2 * j + 1]), EFF);
+    }
+    if constexpr (ODT == DT_F32) {
+        uint32_t a[8], b[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float lo, hi;
+            f2_unpack(ya[j], lo, hi);
+            a[2 * j] = __float_as_uint(lo);
+            a[2 * j + 1] = __float_as_uint(hi);
+            f2_unpack(yb[j], lo, hi);
+            b[2 * j] = __float_as_uint(lo);
+            b[2 * j + 1] = __float_as_uint(hi);
+        }
+        if constexpr (V8) {
+            st_v8(p, a);
+            st_v8(p + 32, b);
+        } else {
+            st_v4(p, a[0], a[1], a[2], a[3]);
+            st_v4(p + 16, a[4], a[5], a[6], a[7]);
+            st_v4(p + 32, b[0], b[1], b[2], b[3]);
+            st_v4(p + 48, b[4], b[5], b[6], b[7]);
+        }
+    } else {
+        uint32_t o[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float lo, hi;
+            f2_unpack(ya[j], lo, hi);
+            o[j] = pack_out2<ODT>(lo, hi);
+            f2_unpack(yb[j], lo, hi);
+            o[4 + j] = pack_out2<ODT>(lo, hi);
+        }
+        // one 256-bit store fills a whole 32-byte sector; two 128-bit
+        // stores would each write half of every sector they touch
+        if constexpr (V8) {
+            st_v8(p, o);
+        } else {
+            st_v4(p, o[0], o[1], o[2], o[3]);
+            st_v4(p + 16, o[4], o[5], o[6], o[7]);
+        }
+    }
+}
+
 // Encode group g from its raw bits r and store its codes and scale byte.
 // Returns true when an input element is Inf or NaN.
-template <int DT, int MODE, bool RHT, bool NV = false>
+template <int DT, int MODE, bool RHT, bool NV = false, bool DQ = false>
 __device__ __forceinline__ bool quantize_one(const Raw<DT> &r, uint32_t g, const char *x,
                                              int64_t ld_bytes, uint32_t gpr, float ts, float rts,
                                              const float *inv_tab, const float *eff_tab,
                                              uint8_t *codes, uint8_t *scales,
                                              const SignMasks &sm, uint32_t signs,
                                              uint8_t *nv_codes = nullptr,
-                                             uint8_t *nv_scales = nullptr)
+                                             uint8_t *nv_scales = nullptr,
+                                             char *y = nullptr, uint32_t lut_addr = 0u)
 {
     constexpr int GB = 16 * elem_bytes<DT>();
     f2_t xv[8];
@@ -483,6 +584,12 @@ __device__ __forceinline__ bool quantize_one(const Raw<DT> &r, uint32_t g, const
         // the NVFP4 comparator: the FP4 candidate under the same block scale
         st_v2(nv_codes + (int64_t)g * 8, out.f0, out.f1);
         st_u8(nv_scales + g, out.scale & 0x7Fu);
+    }
+    if constexpr (DQ) {
+        // the round trip: this group's IF4 codes decoded as the dequantizer
+        // decodes them, bf16 into a dense 32-byte aligned y
+        dequant_group<DT_BF16, false, true>(out.c0, out.c1, out.scale, ts, lut_addr,
+                                            y + (int64_t)g * 32);
     }
     return nonfinite;
 }
@@ -713,13 +820,16 @@ __device__ __noinline__ bool grid_tensor_scale(uint32_t *sync, uint32_t gen0,
     return true;
 }
 
-template <int DT, bool V8, bool RHT, bool NV>
+// DQ: also write the round trip, the IF4 codes decoded to bf16 y (dense,
+// 32-byte aligned), as the dequantizer would decode them.
+template <int DT, bool V8, bool RHT, bool NV, bool DQ = false>
 __global__ void __launch_bounds__(256, DT == DT_F32 ? 3 : 4)
 quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr,
                       uint32_t ngroups, int contig, uint8_t *__restrict__ codes,
                       uint8_t *__restrict__ scales, uint8_t *__restrict__ nv_codes,
                       uint8_t *__restrict__ nv_scales, float *ts_out, uint32_t *sync, int *err,
-                      const __grid_constant__ SignMasks sm, uint32_t signs)
+                      const __grid_constant__ SignMasks sm, uint32_t signs,
+                      char *__restrict__ y)
 {
     // wait for the previous kernel in the stream (programmatic launch)
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -786,6 +896,9 @@ quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr
         const float eff = __fmul_rn(f32_from_e4m3(threadIdx.x), ts);
         inv_tab[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __frcp_rn(eff);
     }
+    __shared__ __align__(128) float lut[DQ ? 32 : 1];
+    if (DQ && threadIdx.x < 32) lut[threadIdx.x] = code_value(threadIdx.x);
+    const uint32_t lut_addr = (uint32_t)__cvta_generic_to_shared(lut);
     const float rts = __frcp_rn(ts);
     __syncthreads();
     for (; g < ngroups;) {
@@ -793,114 +906,16 @@ quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr
         for (int ph = 0; ph < 2; ++ph) {
             const uint32_t gn = g + stride;
             if (gn < ngroups) load_group<DT, V8>(addr(gn), buf[ph ^ 1]);
-            quantize_one<DT, Q_IF4, RHT, NV>(buf[ph], g, x, ld_bytes, gpr_eff, ts, rts, inv_tab,
-                                             nullptr, codes, scales, sm, signs, nv_codes,
-                                             nv_scales);
+            quantize_one<DT, Q_IF4, RHT, NV, DQ>(buf[ph], g, x, ld_bytes, gpr_eff, ts, rts,
+                                                 inv_tab, nullptr, codes, scales, sm, signs,
+                                                 nv_codes, nv_scales, y, lut_addr);
             g = gn;
             if (g >= ngroups) break;
         }
     }
 }
 
-// ------------------------------------------------ dequantize, fp16 decode --
-
-template <int ODT>
-__device__ __forceinline__ uint32_t pack_out2(float a, float b)
-{
-    if constexpr (ODT == DT_BF16) return bf16x2_from_f32(a, b);
-    else return f16x2_from_f32(a, b);
-}
-
-// Decoded value of every code: lut[n] is the FP4 value of nibble n,
-// lut[16 + n] the INT4 value fl(6k/7) of nibble n (k its sign extension).
-// 32 floats, one per shared-memory bank, so any pattern of lookups by a warp
-// is conflict-free.
-__device__ __forceinline__ float code_value(uint32_t i)
-{
-    if (i < 16) {
-        const uint32_t h = f16x2_from_e2m1x2(i);      // nibble in bits 0-3
-        return f16lo_to_f32(h);
-    }
-    const float k = (float)((int)((i - 16) ^ 8u) - 8);
-    return __fmul_rn(k, c67());
-}
-
-__device__ __forceinline__ float lds_f32(uint32_t addr)
-{
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-    return v;
-}
-
-// 8 decoded values (not yet scaled) of the 8 nibbles of w; base is the
-// shared address of lut or lut + 16 floats.
-__device__ __forceinline__ void decode_word(uint32_t w, uint32_t base, float (&q)[8])
-{
-    q[0] = lds_f32(base + ((w << 2) & 0x3Cu));
-#pragma unroll
-    for (int i = 1; i < 8; ++i) q[i] = lds_f32(base + ((w >> (4 * i - 2)) & 0x3Cu));
-}
-
-// Decode one group (code words w0, w1, scale byte sb) and store its 16
-// outputs at p.
-template <int ODT, bool UNIT_TS, bool V8 = false>
-__device__ __forceinline__ void dequant_group(uint32_t w0, uint32_t w1, uint32_t sb, float ts,
-                                              uint32_t lut_addr, char *p)
-{
-    const float e4 = f32_from_e4m3(sb);
-    const float eff = UNIT_TS ? e4 : __fmul_rn(e4, ts);
-    const uint32_t base = lut_addr + ((sb >> 1) & 0x40u);        // INT4 half for bit 7
-    float qa[8], qb[8];
-    decode_word(w0, base, qa);
-    decode_word(w1, base, qb);
-    const f2_t EFF = f2_pack(eff, eff);
-    f2_t ya[4], yb[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        ya[j] = f2_mul(f2_pack(qa[2 * j], qa[2 * j + 1]), EFF);
-        yb[j] = f2_mul(f2_pack(qb[2 * j], qb[2 * j + 1]), EFF);
-    }
-    if constexpr (ODT == DT_F32) {
-        uint32_t a[8], b[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float lo, hi;
-            f2_unpack(ya[j], lo, hi);
-            a[2 * j] = __float_as_uint(lo);
-            a[2 * j + 1] = __float_as_uint(hi);
-            f2_unpack(yb[j], lo, hi);
-            b[2 * j] = __float_as_uint(lo);
-            b[2 * j + 1] = __float_as_uint(hi);
-        }
-        if constexpr (V8) {
-            st_v8(p, a);
-            st_v8(p + 32, b);
-        } else {
-            st_v4(p, a[0], a[1], a[2], a[3]);
-            st_v4(p + 16, a[4], a[5], a[6], a[7]);
-            st_v4(p + 32, b[0], b[1], b[2], b[3]);
-            st_v4(p + 48, b[4], b[5], b[6], b[7]);
-        }
-    } else {
-        uint32_t o[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float lo, hi;
-            f2_unpack(ya[j], lo, hi);
-            o[j] = pack_out2<ODT>(lo, hi);
-            f2_unpack(yb[j], lo, hi);
-            o[4 + j] = pack_out2<ODT>(lo, hi);
-        }
-        // one 256-bit store fills a whole 32-byte sector; two 128-bit
-        // stores would each write half of every sector they touch
-        if constexpr (V8) {
-            st_v8(p, o);
-        } else {
-            st_v4(p, o[0], o[1], o[2], o[3]);
-            st_v4(p + 16, o[4], o[5], o[6], o[7]);
-        }
-    }
-}
+// ------------------------------------------------------------ dequantize --
 
 // ODT: output dtype.  UNIT_TS: leave the tensor scale out (the linear's
 // operand decode), else multiply by *ts.  One thread per group (lanes of a
@@ -1213,12 +1228,13 @@ int quantize_entry(const void *x, int x_dtype, int64_t rows, int64_t cols, int64
 
 // Single-launch quantizer: a cooperative launch of at most one wave, so
 // every block is resident when the blocks meet at the grid barrier.
-template <int DT, bool V8, bool RHT, bool NV>
+template <int DT, bool V8, bool RHT, bool NV, bool DQ = false>
 int launch_fused(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
                  uint8_t *nv_codes, uint8_t *nv_scales, float *ts, uint32_t *sync, int *err,
-                 cudaStream_t st, const DeviceInfo &d, const SignMasks &sm, uint32_t signs)
+                 cudaStream_t st, const DeviceInfo &d, const SignMasks &sm, uint32_t signs,
+                 void *y = nullptr)
 {
-    auto k = quantize_fused_kernel<DT, V8, RHT, NV>;
+    auto k = quantize_fused_kernel<DT, V8, RHT, NV, DQ>;
     static const int occ = resident_blocks(k, 256);
     const uint32_t grid = grid_for(occ, d, s.ngroups, 256);
     cudaLaunchConfig_t cfg = {};
@@ -1235,7 +1251,7 @@ int launch_fused(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
     cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, k, static_cast<const char *>(x), s.ld_bytes, s.gpr, s.ngroups,
                            s.contig ? 1 : 0, codes, scales, nv_codes, nv_scales, ts, sync, err, sm,
-                           signs) != cudaSuccess)
+                           signs, static_cast<char *>(y)) != cudaSuccess)
         return IF4_ERR_CUDA;
     return launch_status();
 }
@@ -1243,9 +1259,27 @@ int launch_fused(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
 template <int DT, bool RHT>
 int dispatch_fused_dt(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
                       uint8_t *nv_codes, uint8_t *nv_scales, float *ts, uint32_t *sync, int *err,
-                      cudaStream_t st, const DeviceInfo &d, const SignMasks &sm, uint32_t signs)
+                      cudaStream_t st, const DeviceInfo &d, const SignMasks &sm, uint32_t signs,
+                      void *y)
 {
     const bool nv = nv_codes != nullptr;
+    if constexpr (!RHT) {
+        if (y != nullptr) {
+            if (s.v8)
+                return nv ? launch_fused<DT, true, false, true, true>(
+                                s, x, codes, scales, nv_codes, nv_scales, ts, sync, err, st, d, sm,
+                                signs, y)
+                          : launch_fused<DT, true, false, false, true>(
+                                s, x, codes, scales, nv_codes, nv_scales, ts, sync, err, st, d, sm,
+                                signs, y);
+            return nv ? launch_fused<DT, false, false, true, true>(
+                            s, x, codes, scales, nv_codes, nv_scales, ts, sync, err, st, d, sm,
+                            signs, y)
+                      : launch_fused<DT, false, false, false, true>(
+                            s, x, codes, scales, nv_codes, nv_scales, ts, sync, err, st, d, sm,
+                            signs, y);
+        }
+    }
     if (s.v8)
         return nv ? launch_fused<DT, true, RHT, true>(s, x, codes, scales, nv_codes, nv_scales, ts,
                                                       sync, err, st, d, sm, signs)
@@ -1276,7 +1310,8 @@ int launch_dequant(const Shape &s, const uint8_t *codes, const uint8_t *scales, 
 template <bool RHT>
 int fused_entry(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
                 uint8_t *codes, uint8_t *scales, uint8_t *nv_codes, uint8_t *nv_scales, float *ts,
-                uint32_t *sync_words, int *err_flag, void *stream, uint32_t signs)
+                uint32_t *sync_words, int *err_flag, void *stream, uint32_t signs,
+                void *y = nullptr)
 {
     Shape s;
     int rc = check_tensor(x, x_dtype, rows, cols, ld_x, s);
@@ -1301,13 +1336,13 @@ int fused_entry(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t 
     switch (x_dtype) {
     case IF4_F32:
         return dispatch_fused_dt<DT_F32, RHT>(s, x, codes, scales, nv_codes, nv_scales, ts,
-                                                sync_words, err_flag, st, d, sm, signs);
+                                                sync_words, err_flag, st, d, sm, signs, y);
     case IF4_BF16:
         return dispatch_fused_dt<DT_BF16, RHT>(s, x, codes, scales, nv_codes, nv_scales, ts,
-                                                 sync_words, err_flag, st, d, sm, signs);
+                                                 sync_words, err_flag, st, d, sm, signs, y);
     default:
         return dispatch_fused_dt<DT_F16, RHT>(s, x, codes, scales, nv_codes, nv_scales, ts,
-                                                sync_words, err_flag, st, d, sm, signs);
+                                                sync_words, err_flag, st, d, sm, signs, y);
     }
 }
 
@@ -1410,6 +1445,17 @@ int if4_quantize_fused(const void *x, int x_dtype, int64_t rows, int64_t cols, i
 {
     return fused_entry<false>(x, x_dtype, rows, cols, ld_x, codes, scales, nv_codes, nv_scales, ts,
                               sync_words, err_flag, stream, 0u);
+}
+
+int if4_quantize_fused_dequant(const void *x, int x_dtype, int64_t rows, int64_t cols,
+                               int64_t ld_x, uint8_t *codes, uint8_t *scales, uint8_t *nv_codes,
+                               uint8_t *nv_scales, float *ts, uint32_t *sync_words, void *y,
+                               int *err_flag, void *stream)
+{
+    if (rows > 0 && cols > 0 && y == nullptr) return IF4_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(y) % 32 != 0) return IF4_ERR_ALIGN;
+    return fused_entry<false>(x, x_dtype, rows, cols, ld_x, codes, scales, nv_codes, nv_scales, ts,
+                              sync_words, err_flag, stream, 0u, y);
 }
 
 int if4_quantize_fused_rht(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,

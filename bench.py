@@ -53,7 +53,8 @@ def parse():
     p.add_argument("--kernel-only", default=None,
                    choices=["amax", "if4_quantize", "if4_dequantize", "nvfp4_quantize", "gemm",
                             "nvint4_quantize", "nvfp4_4over6_quantize", "if4_quantize_rht",
-                            "if4_decode_f16", "fused_quantize", "fused_quantize_rht"],
+                            "if4_decode_f16", "fused_quantize", "fused_quantize_rht",
+                            "fused_quantize_dequant"],
                    help="launch only this kernel, warmup+steps times (for ncu captures)")
     return p.parse_args()
 
@@ -279,9 +280,9 @@ class Step:
             )
             self.sets.append(s)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.kernels = ["fused_quantize", "amax", "scale", "if4_quantize", "if4_dequantize",
-                        "nvfp4_quantize"]
-        self.launches_per_step = 2
+        self.kernels = ["fused_quantize_dequant", "fused_quantize", "amax", "scale",
+                        "if4_quantize", "if4_dequantize", "nvfp4_quantize"]
+        self.launches_per_step = 1
 
     def bytes_per_set(self):
         s = self.sets[0]
@@ -311,6 +312,10 @@ class Step:
         if name == "if4_decode_f16":
             b.if4_decode_f16(s["codes"], s["scales"], s["y"].view(torch.float16))
             return
+        if name == "fused_quantize_dequant":
+            b.if4_quantize_fused_dequant(s["x"], s["codes"], s["scales"], s["ncodes"],
+                                         s["nscales"], s["ts"], s["sync"], s["y"], self.err)
+            return
         if name == "fused_quantize":
             b.if4_quantize_fused(s["x"], s["codes"], s["scales"], s["ncodes"], s["nscales"],
                                  s["ts"], s["sync"], self.err)
@@ -328,17 +333,24 @@ class Step:
             raise ValueError(name)
 
     def run(self, i, events=None):
-        """One step on buffer set i: the single-launch quantizer (tensor amax,
-        tensor scale, IF4 codes and the NVFP4 comparator), then the IF4
-        dequantizer to bf16.  events: optional pair recorded right before
-        and right after the quantizer launch."""
+        """One step on buffer set i, one launch: tensor amax, tensor scale,
+        IF4 codes, the NVFP4 comparator and the IF4 round trip (the codes
+        decoded to bf16 in the same launch).  events: optional pair recorded
+        right before and right after the launch."""
         b, s = self.b, self.sets[i % len(self.sets)]
         if events is not None:
             events[0].record()
-        b.if4_quantize_fused(s["x"], s["codes"], s["scales"], s["ncodes"], s["nscales"], s["ts"],
-                             s["sync"], self.err)
+        b.if4_quantize_fused_dequant(s["x"], s["codes"], s["scales"], s["ncodes"], s["nscales"],
+                                     s["ts"], s["sync"], s["y"], self.err)
         if events is not None:
             events[1].record()
+
+    def run_two_launch(self, i):
+        """The same step as two launches: the single-launch quantizer, then
+        the IF4 dequantizer reading the codes back."""
+        b, s = self.b, self.sets[i % len(self.sets)]
+        b.if4_quantize_fused(s["x"], s["codes"], s["scales"], s["ncodes"], s["nscales"], s["ts"],
+                             s["sync"], self.err)
         b.if4_dequantize(s["codes"], s["scales"], s["ts"], s["y"])
 
     def run_unfused(self, i, events=None, side=None):
@@ -433,7 +445,8 @@ def kernel_table(ms, n_elem, in_bytes, pk):
     dq_bytes = n_elem // 2 + n_elem // 16 + 2 * n_elem
     # the single-launch quantizer: x once, IF4 and NVFP4 codes and scales
     fused_bytes = in_bytes + 2 * (n_elem // 2 + n_elem // 16)
-    nbytes = {"fused_quantize": fused_bytes, "fused_quantize_rht": fused_bytes,
+    nbytes = {"fused_quantize_dequant": fused_bytes + 2 * n_elem,
+              "fused_quantize": fused_bytes, "fused_quantize_rht": fused_bytes,
               "amax": in_bytes, "scale": 8,
               "if4_quantize": q_bytes, "if4_dequantize": dq_bytes,
               "nvfp4_quantize": q_bytes, "nvint4_quantize": q_bytes,
@@ -488,7 +501,7 @@ def quality_report(x_cpu, step):
 
 def measure_e2e(x_cpu, steps, warmup):
     """The same step through the C ABI from pinned host memory: per step, the
-    H2D copy of the input, the two launches, and the D2H copy of every result
+    H2D copy of the input, the step's launch, and the D2H copy of every result
     (IF4 codes, scales and tensor scale, the bf16 dequantized tensor, NVFP4
     codes and scales), all inside the timed region.  Consecutive steps
     alternate between two streams with their own buffers, so one step's
@@ -515,9 +528,8 @@ def measure_e2e(x_cpu, steps, warmup):
         with torch.cuda.stream(L["stream"]):
             d = L["d"]
             L["x"].copy_(h_x, non_blocking=True)
-            b.if4_quantize_fused(L["x"], d["codes"], d["scales"], d["ncodes"], d["nscales"],
-                                 d["ts"], L["sync"], err)
-            b.if4_dequantize(d["codes"], d["scales"], d["ts"], d["y"])
+            b.if4_quantize_fused_dequant(L["x"], d["codes"], d["scales"], d["ncodes"],
+                                         d["nscales"], d["ts"], L["sync"], d["y"], err)
             for k in L["h"]:
                 L["h"][k].copy_(d[k], non_blocking=True)
 
@@ -679,6 +691,17 @@ def run_ours(args):
     # the same step as five launches (NVFP4 on a parallel graph branch), for
     # comparison
     side = torch.cuda.Stream()
+    # the same step as two launches (quantizer, then dequantizer)
+    twarm = capture(step.run_two_launch, sets)
+    ttimed = capture(step.run_two_launch, args.steps)
+    twarm.replay()
+    torch.cuda.synchronize()
+    start.record()
+    ttimed.replay()
+    stop.record()
+    torch.cuda.synchronize()
+    ms_two_launch = start.elapsed_time(stop) / args.steps
+    del twarm, ttimed
     uwarm = capture(step.run_unfused, sets, side=side)
     utimed = capture(step.run_unfused, args.steps, side=side)
     uwarm.replay()
@@ -718,16 +741,18 @@ def run_ours(args):
 
     # the dominant kernel of the step is the single-launch quantizer; the
     # IF4 quantizer alone (tensor scale given) is reported beside it
-    roofline = roof("fused_quantize", "if4_quantize_fused (amax + scale + IF4 + NVFP4)")
-    # the same kernel inside the step: two bounds on its share of a timed step
+    roofline = roof("fused_quantize_dequant",
+                    "if4_quantize_fused_dequant (amax + scale + IF4 + NVFP4 + bf16 round trip)")
+    # the same kernel inside the step (the step is this one launch): the
+    # timed step itself, and events around each launch of the steps run again
     roofline["in_step"] = {
+        "step_us": ms * 1e3,
+        "frac_at_step": kernels["fused_quantize_dequant"]["bytes"] / (ms * 1e-3) / 1e9
+        / pk["hbm_gbs"],
         "event_us_mean": None if seq_mean is None else seq_mean * 1e3,
         "event_us_median": None if seq_median is None else seq_median * 1e3,
-        "event_note": "events on the stream around each quantizer launch of the timed steps "
-                      "run again eagerly; includes the launch latency the events expose",
-        "step_minus_dequantize_us": (ms - kern_ms["if4_dequantize"]) * 1e3,
-        "frac_at_step_minus_dequantize": kernels["fused_quantize"]["bytes"]
-        / ((ms - kern_ms["if4_dequantize"]) * 1e-3) / 1e9 / pk["hbm_gbs"]}
+        "event_note": "events on the stream around each launch of the timed steps run again "
+                      "eagerly; includes the launch latency the events expose"}
     roofline_if4 = roof("if4_quantize", "if4_quantize (tensor scale given)")
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -741,9 +766,10 @@ def run_ours(args):
                              f"(inputs {sets * in_bytes / 1e6:.0f} MB > 3x126 MB L2)",
                        "launch": "the timed steps as one CUDA graph; per-kernel times from "
                                  "one graph per kernel of at least 32 launches over all sets",
-                       "step": "single-launch quantizer (amax, scale, IF4 quantize, NVFP4 "
-                               "quantize), then IF4 dequantize (bf16)"},
+                       "step": "one launch: amax, scale, IF4 quantize, NVFP4 quantize and the "
+                               "IF4 round trip (codes decoded to bf16 in the same launch)"},
             "gpu_launches": step.launches_per_step * args.steps,
+            "ms_per_step_two_launch": ms_two_launch,
             "ms_per_step_unfused": ms_unfused,
             "kernels": kernels, "kernels_outside_step": extra, "roofline": roofline,
             "roofline_if4_quantize": roofline_if4}
@@ -795,7 +821,7 @@ def run_kernel_only(args):
     b.if4_quantize(s["x"], s["codes"], s["scales"], s["ts"], b.TS_GIVEN, step.err)
     torch.cuda.synchronize()
     calls = {name: (lambda name=name: step.run_one(name, 0))
-             for name in Step.EXTRA + ["fused_quantize"]}
+             for name in Step.EXTRA + ["fused_quantize", "fused_quantize_dequant"]}
     calls.update({
         "amax": lambda: b.if4_tensor_amax(s["x"], s["amax"], step.err),
         "if4_quantize": lambda: b.if4_quantize(s["x"], s["codes"], s["scales"], s["ts"],

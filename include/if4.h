@@ -173,6 +173,27 @@ int if4_quantize_fused(const void *x, int x_dtype, int64_t rows, int64_t cols, i
                        float *ts, uint32_t *sync_words, int *err_flag, void *stream);
 
 /*
+ * The single launch with the round trip: everything if4_quantize_fused does,
+ * and also y, the IF4 codes it writes decoded exactly as if4_dequantize
+ * decodes them to bf16: y = bf16_RNE(fl(q * fl(E4M3(sb) * ts))), byte-
+ * identical to if4_dequantize(codes, scales, ts, ..., IF4_BF16) afterwards
+ * ("Adaptive Block-Scaled Data Types", gist.science section 2, "Metodo 6/7",
+ * and the companion's "MAC Unit: Decoding Two Formats from One Sign Bit").
+ * The quantize-then-dequantize round trip of one tensor in one launch; the
+ * codes are decoded while they are still in registers.
+ *
+ * y: bf16 [rows, cols], dense (row stride cols), base 32-byte aligned, owned
+ * by the caller, not overlapping x or the other outputs.  Other arguments and
+ * rules as if4_quantize_fused.  IF4_ERR_NULL for a null y of a non-empty
+ * tensor, IF4_ERR_ALIGN for a y that is not 32-byte aligned.  After
+ * IF4_DEV_TIMEOUT neither codes nor y were written.
+ */
+int if4_quantize_fused_dequant(const void *x, int x_dtype, int64_t rows, int64_t cols,
+                               int64_t ld_x, uint8_t *codes, uint8_t *scales, uint8_t *nv_codes,
+                               uint8_t *nv_scales, float *ts, uint32_t *sync_words, void *y,
+                               int *err_flag, void *stream);
+
+/*
  * The same single launch on the random-sign Hadamard transform of x (see
  * if4_quantize_rht): the amax, the tensor scale, the IF4 codes and the
  * NVFP4 comparator are those of the transformed tensor, equal to

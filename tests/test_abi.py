@@ -28,6 +28,8 @@ def lib():
     L.if4_quantize_fused.argtypes = [vp, i, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp]
     L.if4_quantize_fused_rht.argtypes = [vp, i, i64, i64, i64, ctypes.c_uint32, vp, vp, vp, vp,
                                          vp, vp, vp, vp]
+    L.if4_quantize_fused_dequant.argtypes = [vp, i, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp,
+                                             vp, vp]
     L.if4_linear_quantized.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, ctypes.c_size_t,
                                        vp, vp, vp, vp, vp, vp]
     L.if4_status_str.restype = ctypes.c_char_p
@@ -114,6 +116,13 @@ def test_fused_quantize_host_validation(lib):
     assert f(A, 1, 4, 32, 32, A, A, None, None, A + 2, A, None, None) == 4
     assert f(A, 1, 4, 32, 32, A, A, None, None, A, A + 4, None, None) == 4
     assert f(A, 1, 4, 32, 32, A, A, None, None, A, A + 128, None, None) == 4
+    h = lib.if4_quantize_fused_dequant
+    # null y of a non-empty tensor; y not 32-byte aligned; the rest as above
+    assert h(A, 1, 4, 32, 32, A, A, None, None, A, A, None, None, None) == 1
+    assert h(A, 1, 4, 32, 32, A, A, None, None, A, A, A + 16, None, None) == 4
+    assert h(A, 1, 4, 32, 32, A, A, None, None, None, A, A, None, None) == 1
+    assert h(A, 1, 4, 24, 24, A, A, None, None, A, A, A, None, None) == 2
+    assert h(A, 1, 4, 32, 32, A, A, None, None, A, A + 64, A, None, None) == 4
     g = lib.if4_quantize_fused_rht
     assert g(A, 1, 4, 32, 32, 0x1234, A, A, None, None, None, A, None, None) == 1
     assert g(A, 1, 4, 24, 24, 0x1234, A, A, None, None, A, A, None, None) == 2

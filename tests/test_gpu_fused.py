@@ -242,3 +242,43 @@ def test_fused_contiguous_and_strided_agree():
         assert int(err.item()) == 0
     for a, c in zip(*outs):
         assert torch.equal(a, c)
+
+
+@pytest.mark.parametrize("case", ["weight", "f32_ragged", "f16_small", "strided", "activation"])
+def test_fused_round_trip(case):
+    """if4_quantize_fused_dequant: codes, scales, ts and the NVFP4 output
+    byte-identical to if4_quantize_fused; y bit-identical to if4_dequantize
+    of those codes (bf16) and to the oracle's dequantization rounded to bf16."""
+    b = B()
+    g = torch.Generator().manual_seed(41)
+    if case == "weight":
+        x = workloads.llm_weight(2)
+        xd = x.cuda()
+    elif case == "f32_ragged":
+        x = torch.randn((333, 4096), generator=g) * 3
+        xd = x.cuda()
+    elif case == "f16_small":
+        x = torch.randn((7, 80), generator=g).half()
+        xd = x.cuda()
+    elif case == "strided":
+        base = workloads.llm_weight(1, rows=256, cols=1024 + 64)
+        xd = base.cuda()[:, 8:8 + 1024]
+        x = base[:, 8:8 + 1024].contiguous()
+    else:
+        x = workloads.activation_outliers(0)
+        xd = x.cuda()
+    sync = torch.zeros(b.FUSED_SYNC_WORDS, dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    codes, scales, ts, nc, ns, y = b.quantize_fused_dequant(xd, sync_words=sync, err_flag=err)
+    c2, s2, t2, n2, m2 = b.quantize_fused(xd)
+    y2 = b.dequantize(c2, s2, t2)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and sync[0].item() == 0 and sync[1].item() == 0
+    assert torch.equal(codes, c2) and torch.equal(scales, s2) and ts.item() == t2.item()
+    assert torch.equal(nc, n2) and torch.equal(ns, m2)
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    ref = oracle.quantize_tensor(x.float().numpy())
+    assert np.float32(ts.item()) == ref["ts"]
+    assert np.array_equal(codes.cpu().numpy(), ref["codes"])
+    want = torch.from_numpy(oracle.dequantize(ref["codes"], ref["scales"], ref["ts"]))
+    assert torch.equal(y.cpu().view(torch.int16), want.to(torch.bfloat16).view(torch.int16))
