@@ -180,3 +180,20 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
         sys.modules.pop("adaptive_block_scaled_b200.binding", None)
         if saved is not None:
             sys.modules["adaptive_block_scaled_b200.binding"] = saved
+
+
+def test_round_trip_binding_checks_y(lib):
+    """The binding of if4_quantize_fused_dequant rejects a y that is not a
+    dense bf16 tensor of the shape of x before calling the library."""
+    import torch
+    from adaptive_block_scaled_b200 import binding as b
+    x = torch.zeros((4, 32), dtype=torch.bfloat16)
+    codes = torch.zeros((4, 16), dtype=torch.uint8)
+    scales = torch.zeros((4, 2), dtype=torch.uint8)
+    ts = torch.zeros(1)
+    sync = torch.zeros(b.FUSED_SYNC_WORDS, dtype=torch.int32)
+    for y in (torch.zeros((4, 32)),                                  # float32
+              torch.zeros((4, 16), dtype=torch.bfloat16),            # wrong shape
+              torch.zeros((4, 64), dtype=torch.bfloat16)[:, ::2]):   # not dense
+        with pytest.raises(ValueError):
+            b.if4_quantize_fused_dequant(x, codes, scales, None, None, ts, sync, y)
