@@ -9,21 +9,24 @@
 // 6/7"; shd-paper.top technical framework, steps 1-5).  The arithmetic
 // contract is spelled out in include/if4.h.
 //
-// Work decomposition: the path is HBM-bound (2.5625 B per bf16 element for
-// quantize), so one thread owns one whole group: a 256-bit load brings its 16
-// bf16 values, every reduction (amax, both squared-error sums) stays in the
-// thread's registers, and the outputs are one 8-byte code store and one scale
-// byte.  Lanes of a warp own consecutive groups, so each warp-wide load or
-// store touches one contiguous span.  A grid-stride loop keeps the next
-// group's load in flight while the current one is computed.  The group
-// encoder itself (block scale, candidates, decision) is in if4_encode.cuh,
-// shared with the linear's IF4-output epilogue.
+// Work decomposition: the path moves 2.5625 B per bf16 element for quantize
+// (the single-candidate modes are HBM-bound; the IF4 encode, at about 200
+// instructions per group, is bound by instruction issue), so one thread owns
+// one whole group: a 256-bit load brings its 16 bf16 values, every reduction
+// (amax, both squared-error sums) stays in the thread's registers, and the
+// outputs are one 8-byte code store and one scale byte.  Lanes of a warp own
+// consecutive groups, so each warp-wide load or store touches one contiguous
+// span.  A grid-stride loop keeps the next group's load in flight while the
+// current one is computed, and runs full rounds of a contiguous tensor
+// without per-group range checks.  The group encoder itself (block scale,
+// candidates, decision) is in if4_encode.cuh, shared with the linear's
+// IF4-output epilogue.
 //
 // Kernels here: the tensor amax and tensor scale; the quantizer for IF4 and
 // its comparators (NVFP4, NVINT4, 4/6), optionally on the random-sign
 // Hadamard transform; the single-launch quantizer (amax, grid barrier, encode)
-// in one cooperative launch; the dequantizer and the fp16 operand decode of
-// the linear.
+// in one cooperative launch, optionally also writing the bf16 round trip of
+// its codes; the dequantizer and the fp16 operand decode of the linear.
 
 #include <cuda_runtime.h>
 
