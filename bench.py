@@ -2,18 +2,21 @@
 """Benchmark of the IF4 hot path on B200.
 
 One step = one pass of the whole quantization path over one tensor that is
-already resident in HBM:
+already resident in HBM, as one launch (if4_quantize_fused_dequant):
     tensor amax -> tensor scale -> IF4 quantize (block scale, FP4 and INT4
-    candidates, choice) -> IF4 dequantize to bf16 -> NVFP4 quantize with the
-    same tensor scale
-Default workload: the LLM weight matrix, bf16 4096 x 4096, Student-t(3)
-scaled to std 0.02, groups of 16 along K.  The IF4 x IF4 linear has its own
-workload and is reported under "linear" when its entry point is built.
+    candidates, choice) and NVFP4 quantize with the same tensor scale ->
+    the IF4 codes dequantized to bf16
+The same step as two launches (single-launch quantizer, then the
+dequantizer) and as five is timed beside it.  Default workload: the LLM
+weight matrix, bf16 4096 x 4096, Student-t(3) scaled to std 0.02, groups of
+16 along K.  The IF4 x IF4 linear has its own workload and is reported under
+"linear" when its entry point is built.
 
 value = elements / step time (Gelem/s), max over ranks; with N GPUs every
 rank quantizes its own tensor (independent problems, weak scaling, no data
-collective).  L2: the step rotates over buffer sets whose total exceeds twice
-the 126 MB L2, so no step reads what the previous one left in L2.
+collective).  L2: the step rotates over buffer sets whose inputs total more
+than three times the 126 MB L2, so no step reads what the previous one left
+in L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
