@@ -30,3 +30,26 @@ def test_algorithmic_bytes_per_element(elem_bytes):
         assert t[k]["bytes"] == pytest.approx(per_elem * n, rel=0, abs=0.5), k
         # 1 ms per launch: GB/s is bytes / 1e6
         assert t[k]["gbs"] == pytest.approx(t[k]["bytes"] / 1e6)
+
+
+def test_reference_arm_prints_the_contract_line():
+    """bench.py --impl reference (the oracle, on the host cores) prints one
+    JSON line with the contract's keys, its cpu_baseline and e2e describing
+    that run."""
+    import json
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "0"], capture_output=True, text=True,
+                         timeout=600, cwd=root, check=True).stdout
+    line = json.loads(out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["value"] > 0 and line["higher_is_better"] is True
+    assert line["n_gpus"] == 1 and line["steps"] == 1 and line["warmup"] == 0
+    assert line["config"]["workload"] == bench.WORKLOAD
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"]
+    assert cb["value"] == line["value"]
+    assert line["e2e"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
