@@ -141,3 +141,129 @@ def test_binary32_decision_outside_the_band_is_the_binary64_rule(kind):
         # band widths of it (where a band of 2^-30, or none, decides 3 of them
         # wrongly)
         assert near > 0 and close >= 50
+
+
+# ---------------------------------------------------------------- 4/6 ----
+#
+# The 4/6 comparator decides between the block scales of amax/6 and amax/4
+# from binary32 x-domain error sums, each difference one fused
+# fma(q, -eff, x); groups within the band 2^-18 S + 2^-19 X^2 + 2^-126
+# (X = 6 max(eff6, eff4)) are redecided by the binary64 rule.
+
+def _e4m3_values():
+    import torch
+    return torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).to(
+        torch.float64).numpy()
+
+
+_E4 = None
+
+
+def _e4m3(f):
+    global _E4
+    if _E4 is None:
+        _E4 = _e4m3_values()
+    f = min(f, 1e4)
+    d = np.abs(_E4 - f)
+    return min(range(127), key=lambda c: (d[c], c & 1))
+
+
+def _scales_46(x16, ts):
+    amax = max(abs(t) for t in x16)
+    sb6 = _e4m3(r32(r32(amax / 6.0) / ts))
+    sb4 = _e4m3(r32(r32(amax / 4.0) / ts))
+    eff6, eff4 = r32(_E4[sb6] * ts), r32(_E4[sb4] * ts)
+    return sb6, sb4, eff6, eff4
+
+
+def fast_decision_46(x16, ts):
+    sb6, sb4, eff6, eff4 = _scales_46(x16, ts)
+    inv6, inv4 = r32(1.0 / eff6), r32(1.0 / eff4)
+    e6 = [0.0, 0.0]
+    e4 = [0.0, 0.0]
+    for j in range(8):
+        for lane in (0, 1):
+            x = x16[2 * j + lane]
+            q6 = fp4_value(r32(x * inv6))
+            q4 = fp4_value(r32(x * inv4))
+            d6 = fma32(q6, -eff6, x)
+            d4 = fma32(q4, -eff4, x)
+            e6[lane] = fma32(d6, d6, e6[lane])
+            e4[lane] = fma32(d4, d4, e4[lane])
+    s6, s4 = r32(e6[0] + e6[1]), r32(e4[0] + e4[1])
+    d = r32(s6 - s4)
+    X = r32(6.0 * max(eff6, eff4))
+    band = fma32(r32(s6 + s4), 2.0 ** -18, fma32(r32(X * X), 2.0 ** -19, 2.0 ** -126))
+    return sb6 != sb4, d > 0.0, not abs(d) > band, d, band
+
+
+def exact_decision_46(x16, ts):
+    sb6, sb4, eff6, eff4 = _scales_46(x16, ts)
+    inv6, inv4 = r32(1.0 / eff6), r32(1.0 / eff4)
+    s6 = s4 = 0.0
+    for x in x16:
+        xh6 = r32(fp4_value(r32(x * inv6)) * eff6)
+        xh4 = r32(fp4_value(r32(x * inv4)) * eff4)
+        s6 = s6 + (x - xh6) ** 2
+        s4 = s4 + (x - xh4) ** 2
+    return s4 < s6
+
+
+def _fp4_values_vec(v):
+    """fp4_value over an array (nearest E2M1 magnitude, ties to the even code,
+    saturating at 6, sign of v)."""
+    a = np.minimum(np.abs(v), 6.0)
+    d = np.abs(E2M1[None, :] - a[:, None])
+    dmin = d.min(axis=1, keepdims=True)
+    tie_even = (d == dmin) & ((np.arange(8) % 2) == 0)[None, :]
+    pick = np.where(tie_even.any(axis=1), tie_even.argmax(axis=1), (d == dmin).argmax(axis=1))
+    q = E2M1[pick]
+    return np.where(np.signbit(v), -q, q)
+
+
+def near_tie_groups_46(n, seed):
+    """Groups whose 16th element (below the group maximum, so neither block
+    scale moves) is chosen from a fine grid to bring the two error sums as
+    close together as it can."""
+    rng = np.random.default_rng(seed)
+    ts = r32(2.0 ** -6)
+    out = []
+    for _ in range(n):
+        amax = r32(rng.uniform(0.5, 3.0))
+        base = [amax] + [r32(t) for t in rng.uniform(-1, 1, 14) * amax]
+        _, _, eff6, eff4 = _scales_46(base + [0.0], ts)
+        inv6, inv4 = r32(1.0 / eff6), r32(1.0 / eff4)
+        part = 0.0
+        for x in base:
+            part += (x - r32(fp4_value(r32(x * inv6)) * eff6)) ** 2
+            part -= (x - r32(fp4_value(r32(x * inv4)) * eff4)) ** 2
+        t = (np.linspace(-0.999, 0.999, 4001) * amax).astype(np.float32).astype(np.float64)
+        xh6 = (_fp4_values_vec((t * inv6).astype(np.float32).astype(np.float64)) * eff6)
+        xh4 = (_fp4_values_vec((t * inv4).astype(np.float32).astype(np.float64)) * eff4)
+        xh6 = xh6.astype(np.float32).astype(np.float64)
+        xh4 = xh4.astype(np.float32).astype(np.float64)
+        gaps = part + (t - xh6) ** 2 - (t - xh4) ** 2
+        for i in np.argsort(np.abs(gaps))[:3]:
+            out.append((base + [float(t[i])], ts))
+    return out
+
+
+def test_46_binary32_decision_outside_the_band_is_the_binary64_rule():
+    groups = near_tie_groups_46(100, 5)
+    rng = np.random.default_rng(13)
+    ts = r32(2.0 ** -6)
+    groups += [([r32(t) for t in rng.standard_normal(16) * rng.uniform(0.1, 3.0)], ts)
+               for _ in range(300)]
+    decided = near = close = 0
+    for x16, ts in groups:
+        differ, four, is_near, d, band = fast_decision_46(x16, ts)
+        if not differ:
+            continue                          # identical candidates: kept /6 either way
+        if is_near:
+            near += 1
+            continue
+        decided += 1
+        close += abs(d) < 10 * band
+        assert four == exact_decision_46(x16, ts), (x16, ts)
+    # the construction reaches the band and decides groups close to it
+    assert near > 0 and close >= 30
