@@ -267,3 +267,56 @@ def test_46_binary32_decision_outside_the_band_is_the_binary64_rule():
         assert four == exact_decision_46(x16, ts), (x16, ts)
     # the construction reaches the band and decides groups close to it
     assert near > 0 and close >= 30
+
+
+# --------------------------------------------------------- block scale ----
+#
+# The kernels compute the block scale fl(fl(amax/6)/ts) without dividing:
+# q = RN(amax * RN(1/6)), q = RN(q + RN(amax - 6q) * RN(1/6)) (two fused
+# multiply-adds), then the same with ts and RN(1/ts) (Markstein's method:
+# one correction of a quotient from the correctly rounded reciprocal).  The
+# claim is that this equals the two IEEE divisions whenever amax >= 2^-100
+# and the second quotient stays below 2^100 (outside that, the kernels
+# divide).
+
+def _fma32_vec(a, b, c):
+    """fl32(a*b + c) elementwise, one rounding (float64 arrays of binary32
+    values; the product is exact in binary64, TwoSum makes the sum exact)."""
+    p = a * b
+    s = p + c
+    bv = s - p
+    e = (p - (s - bv)) + (c - bv)
+    r = s.astype(np.float32).astype(np.float64)
+    towards = np.where(s > r, np.inf, -np.inf).astype(np.float32)
+    other = np.nextafter(r.astype(np.float32), towards).astype(np.float64)
+    mid = (r + other) / 2.0
+    fix = (s == mid) & (e != 0) & ((e > 0) == (other > r))
+    return np.where(fix, other, r)
+
+
+def test_block_scale_quotients_equal_the_ieee_divisions():
+    rng = np.random.default_rng(17)
+    n = 1_000_000
+    amax = (rng.uniform(1, 2, n) * np.exp2(rng.integers(-100, 100, n))).astype(np.float32)
+    ts = (rng.uniform(1, 2, n) * np.exp2(rng.integers(-117, 117, n))).astype(np.float32)
+    # a share of exact cases: amax a multiple of 6 ts
+    k = n // 10
+    ts[:k] = np.float32(2.0) ** rng.integers(-60, 60, k).astype(np.float32)
+    amax[:k] = (rng.integers(1, 448, k) * 6 * ts[:k].astype(np.float64)).astype(np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        _check_block_scale(amax, ts, n)
+
+
+def _check_block_scale(amax, ts, n):
+    a, t = amax.astype(np.float64), ts.astype(np.float64)
+    r6 = float(np.float32(1.0) / np.float32(6.0))
+    rts = (np.float32(1.0) / ts).astype(np.float64)
+    q = (a * r6).astype(np.float32).astype(np.float64)
+    q = _fma32_vec(_fma32_vec(-q, np.full(n, 6.0), a), np.full(n, r6), q)
+    s = (q * rts).astype(np.float32).astype(np.float64)
+    got = _fma32_vec(_fma32_vec(-s, t, q), rts, s)
+    want = ((amax / np.float32(6.0)) / ts).astype(np.float64)     # IEEE binary32 divisions
+    valid = (amax >= np.float32(2.0 ** -100)) & (s < 2.0 ** 100) & (want >= 2.0 ** -126)
+    assert valid.sum() > n // 2
+    bad = valid & (got != want)
+    assert not bad.any(), (amax[bad][:5], ts[bad][:5])
