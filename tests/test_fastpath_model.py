@@ -320,3 +320,51 @@ def _check_block_scale(amax, ts, n):
     assert valid.sum() > n // 2
     bad = valid & (got != want)
     assert not bad.any(), (amax[bad][:5], ts[bad][:5])
+
+
+# ---------------------------------------------------- coinciding candidates --
+#
+# Before the binary64 rule, the kernels test on the two code words whether
+# every element's FP4 and INT4 candidates have the same value (the grids share
+# only 0 and +-6), which makes the group an exact tie that keeps FP4.  The bit
+# expression below is the kernels' test; it is checked here against the
+# decoded values.
+
+def coincide_bits(fp4, int4):
+    m = fp4 & 0x77777777
+    is6 = m & (m >> 1) & (m >> 2) & 0x11111111
+    nz = (m | (m >> 1) | (m >> 2)) & 0x11111111
+    sgn = (fp4 >> 3) & 0x11111111
+    want = ((is6 * 0xF) & 0xFFFFFFFF) & (0x77777777 ^ ((sgn * 0xE) & 0xFFFFFFFF))
+    return (nz & ~is6 & 0xFFFFFFFF) == 0 and int4 == want
+
+
+def _fp4_nibble_value(n):
+    mag = E2M1[n & 7]
+    return -mag if n & 8 else mag
+
+
+def _int4_nibble_value(n):
+    k = n - 16 if n & 8 else n
+    return r32(k * 6.0 / 7.0)
+
+
+def test_coinciding_candidates_bit_test_matches_the_values():
+    ints = [n for n in range(16) if n != 8]          # 0x8 (k = -8) is never written
+    # one element (the others 0 on both grids), at every nibble position
+    for pos in range(8):
+        for f in range(16):
+            for i in ints:
+                same = _fp4_nibble_value(f) == _int4_nibble_value(i)
+                assert coincide_bits(f << (4 * pos), i << (4 * pos)) == same, (pos, f, i)
+    # whole words: coincide iff every element does
+    rng = np.random.default_rng(23)
+    pairs = [(f, i) for f in range(16) for i in ints]
+    equal = [(f, i) for f, i in pairs if _fp4_nibble_value(f) == _int4_nibble_value(i)]
+    for trial in range(20000):
+        pool = equal if trial % 2 else pairs          # half the words from equal pairs only
+        picks = [pool[j] for j in rng.integers(0, len(pool), 8)]
+        fw = sum(f << (4 * p) for p, (f, _) in enumerate(picks))
+        iw = sum(i << (4 * p) for p, (_, i) in enumerate(picks))
+        same = all(_fp4_nibble_value(f) == _int4_nibble_value(i) for f, i in picks)
+        assert coincide_bits(fw, iw) == same, (hex(fw), hex(iw))
