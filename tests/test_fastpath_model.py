@@ -368,3 +368,20 @@ def test_coinciding_candidates_bit_test_matches_the_values():
         iw = sum(i << (4 * p) for p, (_, i) in enumerate(picks))
         same = all(_fp4_nibble_value(f) == _int4_nibble_value(i) for f, i in picks)
         assert coincide_bits(fw, iw) == same, (hex(fw), hex(iw))
+
+
+# ------------------------------------------------------------ INT4 packing --
+#
+# The kernels get k + 8 in the low bits of the binary32 r = 1.5 * 2^23 + 8 +
+# k (one fused multiply-add), combine an element pair as the integer
+# bits(r_odd) * 16 + bits(r_even), keep byte 0, and turn the offset-8 nibbles
+# into two's complement with XOR 0x88.
+
+def test_int4_nibble_packing_identity():
+    m8 = F32(12582912.0 + 8.0)                   # 1.5 * 2^23 + 8
+    for ke in range(-7, 8):
+        for ko in range(-7, 8):
+            re = int(np.array([m8 + F32(ke)], np.float32).view(np.uint32)[0])
+            ro = int(np.array([m8 + F32(ko)], np.float32).view(np.uint32)[0])
+            byte0 = ((ro * 16 + re) & 0xFFFFFFFF) & 0xFF
+            assert byte0 ^ 0x88 == ((ko & 0xF) << 4) | (ke & 0xF), (ke, ko)
