@@ -53,3 +53,26 @@ def test_reference_arm_prints_the_contract_line():
     assert cb["value"] == line["value"]
     assert line["e2e"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_clock_summary_reads_reasons_and_the_clock_under_load():
+    """The nvidia-smi samples the bench takes during the timed region: the
+    median SM clock of the samples under load, the maximum clock, and every
+    throttle reason seen active ("Not Active" is not a reason; malformed
+    lines are skipped)."""
+    c = bench.ClockSampler(0)
+    c.lines = [
+        "0, 1965, 1965, 120.5, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n",
+        "0, 1965, 1965, 612.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n",
+        "0, 1890, 1965, 655.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n",
+        "0, 1950, 1965, 640.0, 0x0000000000000008, Active, Not Active, Not Active, Not Active\n",
+        "garbage line\n",
+        "0, [N/A], 1965, 600.0, 0x0, Not Active, Not Active, Not Active, Not Active\n",
+    ]
+    s = c.summary()
+    assert s["samples"] == 4 and s["samples_under_load"] == 3
+    assert s["sm_mhz"] == 1950.0 and s["sm_max_mhz"] == 1965.0
+    assert s["power_w_max"] == 655.1
+    assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    c.lines = []
+    assert c.summary() is None
