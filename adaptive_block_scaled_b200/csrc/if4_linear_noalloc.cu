@@ -23,7 +23,12 @@
 //     the caller must order them, e.g. by issuing them on one stream;
 //   * the first call on each device looks up the array's device address
 //     (cudaGetSymbolAddress, with that device current) and caches it, so that
-//     first call should come before any stream capture the caller starts.
+//     first call should come before any stream capture the caller starts;
+//   * the cached address belongs to the device's primary context.  A
+//     cudaDeviceReset ends that context and with it the array; the cache
+//     cannot see that, so after a reset a process must not call
+//     if4_linear_noalloc on that device again (if4_linear, with a workspace
+//     from the caller, is unaffected).
 
 #include <cuda_runtime.h>
 
@@ -68,13 +73,16 @@ extern "C" int if4_linear_noalloc(const uint8_t *a_codes, const uint8_t *a_scale
                                   int64_t N, int64_t K, void *c, int *err_flag, void *stream)
 {
     const size_t need = if4_linear_workspace_bytes(M, N, K);
-    if (need > (size_t)IF4_LINEAR_NOALLOC_MAX_BYTES) return IF4_ERR_WORKSPACE;
     void *scratch = nullptr;
-    if (need != 0) {
+    // A problem too large for the array gets no scratch: if4_linear then
+    // checks the other arguments first and refuses it with
+    // IF4_ERR_WORKSPACE, so the errors come in the same order as from
+    // if4_linear itself.  Invalid sizes (need == 0) are reported by the same
+    // checks.
+    if (need != 0 && need <= (size_t)IF4_LINEAR_NOALLOC_MAX_BYTES) {
         const int rc = scratch_address(&scratch);
         if (rc != IF4_OK) return rc;
     }
-    // invalid sizes (need == 0) are reported by if4_linear's own checks
     return if4_linear(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, M, N, K, scratch,
-                      (size_t)IF4_LINEAR_NOALLOC_MAX_BYTES, c, err_flag, stream);
+                      scratch ? (size_t)IF4_LINEAR_NOALLOC_MAX_BYTES : 0u, c, err_flag, stream);
 }

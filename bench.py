@@ -7,10 +7,18 @@ already resident in HBM, as one launch (if4_quantize_fused_dequant):
     candidates, choice) and NVFP4 quantize with the same tensor scale ->
     the IF4 codes dequantized to bf16
 The same step as two launches (single-launch quantizer, then the
-dequantizer) and as five is timed beside it.  Default workload: the LLM
-weight matrix, bf16 4096 x 4096, Student-t(3) scaled to std 0.02, groups of
-16 along K.  The IF4 x IF4 linear has its own workload and is reported under
-"linear" when its entry point is built.
+dequantizer) and as five is timed beside it.  Default workload: the
+activation tensor, bf16 8192 tokens x 8192 hidden, N(0, 1) with 1 % of the
+channels (fixed by the seed) scaled by 20, groups of 16 along the hidden
+dimension: the largest of the quantizer workloads (67 M elements, with the
+gradient tensor) and the one whose outlier groups put the most groups near
+an FP4/INT4 tie.  The other quantizer workloads (the 256 x 1024 float32
+tensor, the 4096 x 4096 weight, the 16384 x 4096 Hadamard-transformed
+gradient) get their own kernel tables and, like the headline, a parity and
+quality block: every group's codes and scale byte against the CPU oracle
+(mismatches counted), the oracle's near ties counted, and the MSE of IF4 and
+its comparators.  The IF4 x IF4 linear has its own workload and is reported
+under "linear".
 
 value = elements / step time (Gelem/s), max over ranks; with N GPUs every
 rank quantizes its own tensor (independent problems, weak scaling, no data
@@ -36,7 +44,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "IF4 quantize Gelem/s & HBM GB/s vs ~8 TB/s peak (1 B200); MSE vs NVFP4"
 UNIT = "Gelem/s"
-WORKLOAD = "weight_bf16_4096x4096"
+WORKLOAD = "activation_bf16_8192x8192"
+# the quantizer workloads: each gets a parity and quality block
+QUANT_WORKLOADS = ("small_fp32_256x1024", "weight_bf16_4096x4096", "activation_bf16_8192x8192",
+                   "gradient_bf16_16384x4096")
 L2_BYTES = 126e6
 RHT_SIGNS = 0x6A3C          # one fixed random-sign vector for the transform
 
@@ -52,7 +63,9 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-linear", action="store_true")
     p.add_argument("--no-large", action="store_true",
-                   help="skip the per-kernel table of the two large workloads")
+                   help="skip the per-kernel tables of the other quantizer workloads")
+    p.add_argument("--no-quality", action="store_true",
+                   help="skip the per-workload parity and quality block")
     p.add_argument("--kernel-only", default=None,
                    choices=["amax", "if4_quantize", "if4_dequantize", "nvfp4_quantize", "gemm",
                             "nvint4_quantize", "nvfp4_4over6_quantize", "if4_quantize_rht",
@@ -69,6 +82,11 @@ def peaks():
         return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
                     bf16_tflops_sustained=d.get("bf16_tflops_sustained"), source="measured")
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def b_lib():
+    from adaptive_block_scaled_b200 import binding
+    return binding.lib
 
 
 def make_input(name, seed=0):
@@ -180,42 +198,51 @@ def barrier(world):
 
 # ----------------------------------------------------------- CPU oracle --
 
-def cpu_oracle_step(x_np):
+def cpu_oracle_step(x_np, threads=0):
+    """One step of the path on the oracle: tensor amax and scale, IF4
+    quantize, dequantize, NVFP4 quantize with the same tensor scale.
+    threads = 0: every host core (OpenMP over rows)."""
     import oracle
-    q = oracle.quantize_tensor(x_np)
-    oracle.dequantize(q["codes"], q["scales"], q["ts"])
-    n = oracle.quantize(x_np, q["ts"], mode=oracle.MODE_NVFP4)
+    q = oracle.quantize_tensor(x_np, threads=threads)
+    oracle.dequantize(q["codes"], q["scales"], q["ts"], threads=threads)
+    n = oracle.quantize(x_np, q["ts"], mode=oracle.MODE_NVFP4, threads=threads)
     return q, n
 
 
-def cpu_baseline(x_cpu, seconds):
-    """The oracle as it stands (C, OpenMP over rows, all host cores) on a
-    bounded row sample of the same workload; elements/s of the whole step."""
+def oracle_rate(x_np, seconds, threads):
+    """Elements/s of the oracle's step on the first rows of x_np, as many
+    rows as take about `seconds` (sized by a probe of 64 rows)."""
+    rows = x_np.shape[0]
+    probe = np.ascontiguousarray(x_np[:min(rows, 64)])
+    t0 = time.perf_counter()
+    cpu_oracle_step(probe, threads)
+    per_row = (time.perf_counter() - t0) / probe.shape[0]
+    sample_rows = int(max(1, min(rows, seconds / max(per_row, 1e-9))))
+    sample = np.ascontiguousarray(x_np[:sample_rows])
+    t0 = time.perf_counter()
+    q, _ = cpu_oracle_step(sample, threads)
+    dt = time.perf_counter() - t0
+    return sample.size / dt / 1e9, sample_rows, dt, int(q["near"].sum())
+
+
+def cpu_baseline(x_cpu, seconds, workload):
+    """The oracle as it stands (C, OpenMP over rows) timed on a bounded row
+    sample of the same workload, on every host core and on one core;
+    elements/s of the whole step."""
     import oracle
     x_np = x_cpu.float().numpy()
     rows = x_np.shape[0]
-    sample_rows = max(1, min(rows, 256))
-    t0 = time.perf_counter()
-    cpu_oracle_step(x_np[:sample_rows])
-    dt = time.perf_counter() - t0
-    per_row = dt / sample_rows
-    sample_rows = int(max(1, min(rows, seconds / max(per_row, 1e-9))))
-    sample = np.ascontiguousarray(x_np[:sample_rows])
-    reps, elapsed, near = 0, 0.0, 0
-    while elapsed < seconds or reps == 0:
-        t0 = time.perf_counter()
-        q, _ = cpu_oracle_step(sample)
-        elapsed += time.perf_counter() - t0
-        reps += 1
-        near = int(q["near"].sum())
-        if reps >= 50:
-            break
-    elems = sample.size * reps
-    return {"value": elems / elapsed / 1e9, "unit": UNIT, "cores": oracle.max_threads(),
-            "kind": "oracle",
-            "sample": f"first {sample_rows} of {rows} rows of {WORKLOAD}, {reps} passes of "
-                      f"amax+scale+IF4 quantize+dequantize+NVFP4 quantize ({elapsed:.1f} s)",
-            "near_ties_in_sample": near}
+    cores = oracle.max_threads()
+    v_all, r_all, t_all, near = oracle_rate(x_np, seconds, 0)
+    v_one, r_one, t_one, _ = oracle_rate(x_np, seconds, 1)
+    what = "amax+scale+IF4 quantize+dequantize+NVFP4 quantize"
+    return {"value": v_all, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"first {r_all} of {rows} rows of {workload}, one pass of {what} "
+                      f"({t_all:.1f} s, {cores} threads)",
+            "near_ties_in_sample": near,
+            "one_core": {"value": v_one, "unit": UNIT, "cores": 1,
+                         "sample": f"first {r_one} of {rows} rows of {workload}, one pass of "
+                                   f"{what} ({t_one:.1f} s, 1 thread)"}}
 
 
 def run_reference(args):
@@ -242,19 +269,31 @@ def run_reference(args):
         times.append(time.perf_counter() - t0)
     step = sum(times) / len(times)
     value = sample.size / step / 1e9
+    sample_desc = (f"first {sample_rows} of {rows} rows of {args.workload} per step "
+                   f"(amax+scale+IF4 quantize+dequantize+NVFP4 quantize)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": args.workload, "rows_sampled": sample_rows,
-                       "cols": int(x_np.shape[1]), "l2": "host CPU"},
+            "config": bench_config(args.workload, x, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle",
-                             "cores": oracle.max_threads(),
-                             "sample": f"first {sample_rows} rows of {args.workload} per step"},
+                             "cores": oracle.max_threads(), "sample": sample_desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
+
+
+def bench_config(workload, x_cpu, world):
+    """The `config` object of the JSON line; the same for both arms."""
+    rows, cols = x_cpu.shape
+    return {"workload": workload, "rows": int(rows), "cols": int(cols),
+            "input_dtype": str(x_cpu.dtype).replace("torch.", ""), "group": 16,
+            "parallelism": f"independent tensors x{world}",
+            "l2": "inputs larger than L2: rotating buffer sets whose inputs total more than "
+                  "3x the 126 MB L2",
+            "step": "amax, scale, IF4 quantize, NVFP4 quantize and the IF4 round trip "
+                    "(codes decoded to bf16)"}
 
 
 # ---------------------------------------------------------- our kernels --
@@ -464,42 +503,103 @@ def kernel_table(ms, n_elem, in_bytes, pk):
     return table
 
 
-def large_workloads(pk, names=("activation_bf16_8192x8192", "gradient_bf16_16384x4096")):
-    """Per-kernel times on the large workloads (more than L2 per launch)."""
+def other_workloads(pk, headline):
+    """Per-kernel tables of the other bf16 quantizer workloads (the weight,
+    activation and gradient tensors, whichever is not the headline)."""
     out = {}
-    for wname in names:
+    for wname in ("weight_bf16_4096x4096", "activation_bf16_8192x8192",
+                  "gradient_bf16_16384x4096"):
+        if wname == headline:
+            continue
         x_cpu = make_input(wname)
         n_elem, in_bytes = x_cpu.numel(), x_cpu.numel() * x_cpu.element_size()
-        step = Step(x_cpu, sets=3)
-        for i in range(3):
+        sets = max(4, int(np.ceil(3 * L2_BYTES / in_bytes)) + 1)
+        step = Step(x_cpu, sets=sets)
+        for i in range(sets):
             step.run(i)
         torch.cuda.synchronize()
         ms = kernel_times(step, step.kernels + Step.EXTRA, 10)
         out[wname] = kernel_table(ms, n_elem, in_bytes, pk)
-        out[wname]["quality"] = quality_report(x_cpu, step)
         del step
         torch.cuda.empty_cache()
     return out
 
 
-def quality_report(x_cpu, step):
-    """MSE against the input (x domain, float64 on the host) of IF4 and of
-    the comparators on the same tensor and tensor scale, from GPU outputs
-    (quantized and dequantized by the library, outside the timed region);
-    the IF4 INT4-group fraction."""
+def _group_mismatches(codes_gpu, scales_gpu, codes_ref, scales_ref):
+    """Groups whose 8 code bytes or scale byte differ."""
+    c = codes_gpu.reshape(-1, 8) != codes_ref.reshape(-1, 8)
+    s = scales_gpu.reshape(-1) != scales_ref.reshape(-1)
+    return int(np.count_nonzero(c.any(axis=1) | s))
+
+
+def parity_quality(name, x_cpu=None):
+    """Parity and quality of one quantizer workload, outside any timed
+    region: the library's IF4 quantizer (tensor scale computed) and its
+    comparators (NVFP4, NVINT4, 4/6 under that tensor scale) against the CPU
+    oracle on the same input, group by group (code bytes and scale byte);
+    the oracle's near ties (candidate errors within 1e-6 relative, or a zero
+    block scale), counted; the dequantized IF4 values against the oracle's,
+    element by element; the MSE of each format in the x domain (float64, from
+    the library's dequantized output) and the IF4 INT4-group fraction."""
+    import oracle
     from adaptive_block_scaled_b200 import binding as b
-    s = step.sets[0]
-    x = x_cpu.float().numpy().astype(np.float64)
-    out = {}
-    for mode in ("if4", "nvfp4", "nvint4", "4over6"):
-        c, sc, _ = b.quantize(s["x"], mode, ts=s["ts"].clone())
-        y = b.dequantize(c, sc, s["ts"], dtype=torch.float32).cpu().numpy().astype(np.float64)
-        out["mse_" + mode] = float(np.mean((x - y) ** 2))
-        if mode == "if4":
-            out["int4_group_fraction"] = float(np.mean(sc.cpu().numpy() >> 7))
+    if x_cpu is None:
+        x_cpu = make_input(name)
+    x_np = np.ascontiguousarray(x_cpu.float().numpy())
+    x64 = x_np.astype(np.float64)
+    dev = torch.device("cuda")
+    xd = x_cpu.to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ref = oracle.quantize_tensor(x_np)
+    c, sc, ts = b.quantize(xd, "if4", err_flag=err)
+    y = b.dequantize(c, sc, ts, dtype=torch.float32).cpu().numpy()
+    c_np, sc_np = c.cpu().numpy(), sc.cpu().numpy()
+    y_ref = oracle.dequantize(ref["codes"], ref["scales"], ref["ts"])
+    out = {"groups": int(sc_np.size),
+           "near_ties": int(ref["near"].sum()),
+           "ts_bit_identical": bool(np.float32(ts.item()) == ref["ts"]),
+           "mismatched_groups": {"if4": _group_mismatches(c_np, sc_np, ref["codes"],
+                                                          ref["scales"])},
+           "dequantize_mismatched_elements": int(np.count_nonzero(
+               y.view(np.uint32) != y_ref.view(np.uint32))),
+           "int4_group_fraction": float(np.mean(sc_np >> 7)),
+           "mse_if4": float(np.mean((x64 - y) ** 2))}
+    for mode, omode in (("nvfp4", oracle.MODE_NVFP4), ("nvint4", oracle.MODE_NVINT4),
+                        ("4over6", oracle.MODE_4OVER6)):
+        cm, scm, _ = b.quantize(xd, mode, ts=ts.clone(), err_flag=err)
+        rm = oracle.quantize(x_np, ref["ts"], mode=omode)
+        out["mismatched_groups"][mode] = _group_mismatches(cm.cpu().numpy(), scm.cpu().numpy(),
+                                                           rm["codes"], rm["scales"])
+        ym = b.dequantize(cm, scm, ts, dtype=torch.float32).cpu().numpy()
+        out["mse_" + mode] = float(np.mean((x64 - ym) ** 2))
+    torch.cuda.synchronize()
+    out["device_error_flag"] = int(err.item())
     nv = out["mse_nvfp4"]
     out["mse_reduction_vs_nvfp4_pct"] = 100.0 * (1.0 - out["mse_if4"] / nv) if nv > 0 else 0.0
     return out
+
+
+def step_outputs_vs_oracle(x_cpu, s):
+    """The timed step's own outputs (buffer set s: IF4 codes and scales,
+    tensor scale, NVFP4 codes and scales, bf16 round trip) against the
+    oracle on the same input."""
+    import oracle
+    x_np = np.ascontiguousarray(x_cpu.float().numpy())
+    ref = oracle.quantize_tensor(x_np)
+    nref = oracle.quantize(x_np, ref["ts"], mode=oracle.MODE_NVFP4)
+    y_ref = torch.from_numpy(oracle.dequantize(ref["codes"], ref["scales"], ref["ts"]))
+    y_ref = y_ref.to(torch.bfloat16).view(torch.int16).numpy()
+    return {"groups": int(ref["scales"].size),
+            "near_ties": int(ref["near"].sum()),
+            "ts_bit_identical": bool(np.float32(s["ts"].item()) == ref["ts"]),
+            "if4_mismatched_groups": _group_mismatches(s["codes"].cpu().numpy(),
+                                                       s["scales"].cpu().numpy(),
+                                                       ref["codes"], ref["scales"]),
+            "nvfp4_mismatched_groups": _group_mismatches(s["ncodes"].cpu().numpy(),
+                                                         s["nscales"].cpu().numpy(),
+                                                         nref["codes"], nref["scales"]),
+            "y_mismatched_elements": int(np.count_nonzero(
+                s["y"].cpu().view(torch.int16).numpy() != y_ref))}
 
 
 def measure_e2e(x_cpu, steps, warmup):
@@ -723,7 +823,6 @@ def run_ours(args):
     graphs_keep = timed
 
     value = world * n_elem / (ms * 1e-3) / 1e9
-    q_bytes = in_bytes + n_elem // 2 + n_elem // 16
     kernels = kernel_table(kern_ms, n_elem, in_bytes, pk)
     extra = kernel_table(kernel_times(step, Step.EXTRA, 5), n_elem, in_bytes, pk)
 
@@ -731,7 +830,7 @@ def run_ours(args):
         k = kernels[name]
         r = {"bound": "hbm", "kernel": label, "achieved": k["gbs"], "peak": pk["hbm_gbs"],
              "unit": "GB/s", "frac": k["gbs"] / pk["hbm_gbs"],
-             "peak_source": f"{pk['source']} hbm_gbs (copy bandwidth, read+write; of measured)",
+             "peak_source": f"{pk['source']} hbm_gbs (copy bandwidth, read+write; of {pk['source']})",
              "algorithmic_bytes_per_launch": k["bytes"], "traffic": None,
              "timing": "CUDA events around a graph of at least 32 back-to-back launches over "
                        "the buffer sets, on the launching stream; mean per launch"}
@@ -758,19 +857,16 @@ def run_ours(args):
                       "eagerly; includes the launch latency the events expose"}
     roofline_if4 = roof("if4_quantize", "if4_quantize (tensor scale given)")
 
+    config = bench_config(args.workload, x_cpu, world)
+    config.update({"buffer_sets": sets,
+                   "l2_detail": f"rotating {sets} buffer sets, {sets * per_set / 1e6:.0f} MB "
+                                f"(inputs {sets * in_bytes / 1e6:.0f} MB > 3x126 MB L2)",
+                   "launch": "the timed steps as one CUDA graph; per-kernel times from one graph "
+                             "per kernel of at least 32 launches over all sets"})
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic",
-            "config": {"workload": args.workload, "rows": int(x_cpu.shape[0]),
-                       "cols": int(x_cpu.shape[1]), "input_dtype": str(x_cpu.dtype).replace("torch.", ""),
-                       "group": 16, "parallelism": f"independent tensors x{world}",
-                       "l2": f"rotating {sets} buffer sets, {sets * per_set / 1e6:.0f} MB "
-                             f"(inputs {sets * in_bytes / 1e6:.0f} MB > 3x126 MB L2)",
-                       "launch": "the timed steps as one CUDA graph; per-kernel times from "
-                                 "one graph per kernel of at least 32 launches over all sets",
-                       "step": "one launch: amax, scale, IF4 quantize, NVFP4 quantize and the "
-                               "IF4 round trip (codes decoded to bf16 in the same launch)"},
+            "data": "synthetic", "config": config,
             "gpu_launches": step.launches_per_step * args.steps,
             "ms_per_step_two_launch": ms_two_launch,
             "ms_per_step_unfused": ms_unfused,
@@ -778,18 +874,29 @@ def run_ours(args):
             "roofline_if4_quantize": roofline_if4}
     if rank == 0:
         line["clocks"] = clk.summary()
-        line["quality"] = quality_report(x_cpu, step)
+        # the step's own outputs (buffer set 0, last written by the timed
+        # steps or the per-kernel graphs that ran the same launch) against
+        # the oracle: rerun the step on set 0 so it holds the step's results
+        step.run(0)
+        torch.cuda.synchronize()
+        line["step_outputs_vs_oracle"] = step_outputs_vs_oracle(x_cpu, step.sets[0])
         line["e2e"] = measure_e2e(x_cpu, max(5, args.steps // 5), 2)
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(x_cpu, args.cpu_seconds)
+            line["cpu_baseline"] = cpu_baseline(x_cpu, args.cpu_seconds, args.workload)
+    del step, graphs_keep
+    torch.cuda.empty_cache()
+    if rank == 0:
+        # parity and quality of every quantizer workload (the headline's own
+        # tensor included), outside the timed region: N = 1 only
+        if world == 1 and not args.no_quality:
+            line["quality"] = {w: parity_quality(w, x_cpu if w == args.workload else None)
+                               for w in QUANT_WORKLOADS}
         # single-GPU reports: only at N = 1, so that with N > 1 the other
         # ranks do not wait long at the final barrier
-        if not args.no_linear and world == 1 and hasattr(step.b.lib, "if4_linear"):
+        if not args.no_linear and world == 1 and hasattr(b_lib(), "if4_linear"):
             line["linear"] = linear_report(pk)
         if not args.no_large and world == 1:
-            del step, graphs_keep
-            torch.cuda.empty_cache()
-            line["large_workloads"] = large_workloads(pk)
+            line["other_workloads"] = other_workloads(pk, args.workload)
         print(json.dumps(line), flush=True)
     barrier(world)
     if world > 1:

@@ -90,7 +90,8 @@ enum {
 enum {
     IF4_DEV_NONFINITE = 1,   /* an input element is Inf or NaN: outputs unspecified */
     IF4_DEV_BAD_SCALE = 2,   /* a given ts is not finite or outside [2^-117, 2^117] */
-    IF4_DEV_TIMEOUT = 4      /* a pipeline wait in the linear ran out of its bound  */
+    IF4_DEV_TIMEOUT = 4      /* a bounded wait (the linear's pipeline, the single-launch
+                                quantizer's grid barrier) ran out: outputs unspecified */
 };
 
 /* Largest supported tensor: rows * cols / 16 < 2^31 groups. */
@@ -159,9 +160,11 @@ int if4_quantize_rht(const void *x, int x_dtype, int64_t rows, int64_t cols, int
  * and word 33 keeps the last ts; they may hold any value.  The rest is
  * unused.  So one allocation serves any number
  * of calls that run one after another; calls that may run at the same time
- * (other streams) need their own.  After a call that set IF4_DEV_TIMEOUT (a
- * block waited more than 1 s at the grid barrier; no codes were written)
- * the words must be zeroed again.
+ * (other streams) need their own.  A call that set IF4_DEV_TIMEOUT (a
+ * block waited more than 1 s at the grid barrier) leaves codes, scales, ts
+ * and y unspecified: blocks that gave up wrote nothing, but a block that
+ * arrived last, or was still waiting, may have encoded its groups.  Zero the
+ * words and call again.
  *
  * nv_codes / nv_scales: both NULL (IF4 only) or both given.  err_flag may be
  * NULL; IF4_DEV_NONFINITE and IF4_DEV_TIMEOUT are reported there.  Other
@@ -186,7 +189,8 @@ int if4_quantize_fused(const void *x, int x_dtype, int64_t rows, int64_t cols, i
  * by the caller, not overlapping x or the other outputs.  Other arguments and
  * rules as if4_quantize_fused.  IF4_ERR_NULL for a null y of a non-empty
  * tensor, IF4_ERR_ALIGN for a y that is not 32-byte aligned.  After
- * IF4_DEV_TIMEOUT neither codes nor y were written.
+ * IF4_DEV_TIMEOUT codes, scales, ts and y are unspecified, as for
+ * if4_quantize_fused.
  */
 int if4_quantize_fused_dequant(const void *x, int x_dtype, int64_t rows, int64_t cols,
                                int64_t ld_x, uint8_t *codes, uint8_t *scales, uint8_t *nv_codes,
@@ -302,9 +306,10 @@ int if4_linear_quantized(const uint8_t *a_codes, const uint8_t *a_scales, const 
                          void *c, uint8_t *c_codes, uint8_t *c_scales, const float *c_ts,
                          int *err_flag, void *stream);
 
-/* Size of the scratch array behind if4_linear_noalloc (32 MiB per device). */
+/* Number of uint32 sync words if4_quantize_fused and its variants need. */
 #define IF4_FUSED_SYNC_WORDS 64u
 
+/* Size of the scratch array behind if4_linear_noalloc (32 MiB per device). */
 #define IF4_LINEAR_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
 
 /*
@@ -322,7 +327,11 @@ int if4_linear_quantized(const uint8_t *a_codes, const uint8_t *a_scales, const 
  * calls whose work overlaps on the GPU race and corrupt each other, so order
  * them (e.g. one stream).  The first call on each device looks up the
  * array's address with that device current; make that first call before any
- * stream capture.
+ * stream capture.  That address belongs to the device's primary context:
+ * after a cudaDeviceReset of the device, do not call if4_linear_noalloc on it
+ * again in the same process.  Errors come in the order of if4_linear's: a
+ * problem too large for the array returns IF4_ERR_WORKSPACE only when every
+ * other argument is valid.
  */
 int if4_linear_noalloc(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_ts,
                        const uint8_t *b_codes, const uint8_t *b_scales, const float *b_ts,

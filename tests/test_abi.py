@@ -32,6 +32,7 @@ def lib():
                                              vp, vp]
     L.if4_linear_quantized.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, ctypes.c_size_t,
                                        vp, vp, vp, vp, vp, vp]
+    L.if4_linear_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
     L.if4_status_str.restype = ctypes.c_char_p
     return L
 
@@ -141,6 +142,20 @@ def test_linear_quantized_host_validation(lib):
     assert f(A, A, A, A, A, A, 128, 256, 64, A, W, None, A + 8, A, A, A, None) == 4
     assert f(A, A, A, A, A, A, 128, 256, 64, A, W, None, A, A, A + 2, A, None) == 4
     assert f(A, A, A, A, A, A, 128, 256, 64, A, 16, None, A, A, A, A, None) == 6
+
+
+def test_linear_noalloc_error_order(lib):
+    """The allocation-free linear reports errors in if4_linear's order: a
+    problem too large for its scratch array is refused with
+    IF4_ERR_WORKSPACE only when every other argument is valid."""
+    f = lib.if4_linear_noalloc
+    big = (4096, 4096, 4096)        # 64 MiB of decoded operands > the 32 MiB array
+    assert f(A, A, A, A, A, A, *big, A, A, None) == 6
+    assert f(None, A, A, A, A, A, *big, A, A, None) == 1
+    assert f(A, A, A, A, A, A, *big, A, None, None) == 1      # err_flag
+    assert f(A, A, A, A, A, A, 4096, 4096, 4104, A, A, None) == 2
+    assert f(A, A, A, A, A, A, *big, A + 8, A, None) == 4     # c misaligned
+    assert f(A, A, A, A, A, A, 0, 4096, 4096, A, A, None) == 2
 
 
 def test_dequantize_and_decode_host_validation(lib):

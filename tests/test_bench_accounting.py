@@ -48,6 +48,9 @@ def test_reference_arm_prints_the_contract_line():
     assert line["value"] > 0 and line["higher_is_better"] is True
     assert line["n_gpus"] == 1 and line["steps"] == 1 and line["warmup"] == 0
     assert line["config"]["workload"] == bench.WORKLOAD
+    # the same config object as the GPU arm's (its extra keys aside)
+    x = bench.make_input(bench.WORKLOAD)
+    assert line["config"] == bench.bench_config(bench.WORKLOAD, x, 1)
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"]
     assert cb["value"] == line["value"]
@@ -76,3 +79,30 @@ def test_clock_summary_reads_reasons_and_the_clock_under_load():
     assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]
     c.lines = []
     assert c.summary() is None
+
+
+def test_cpu_baseline_times_every_core_and_one_core():
+    """The oracle's timing on the host: all cores and one core, each on a
+    stated row sample of the given workload."""
+    import torch
+    x = torch.randn(64, 256, generator=torch.Generator().manual_seed(0))
+    cb = bench.cpu_baseline(x, 0.05, "test_64x256")
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
+    assert "test_64x256" in cb["sample"]
+    one = cb["one_core"]
+    assert one["cores"] == 1 and one["value"] > 0 and "1 thread" in one["sample"]
+
+
+def test_group_mismatch_count():
+    """A group counts once whether its code bytes, its scale byte or both
+    differ."""
+    import numpy as np
+    c = np.zeros((4, 16), np.uint8)
+    s = np.zeros((4, 2), np.uint8)
+    c2, s2 = c.copy(), s.copy()
+    c2[0, 3] = 1            # group 0 (codes)
+    s2[1, 1] = 0x80         # group 3 (scale)
+    c2[2, 0] = 1            # group 4 (codes) ...
+    s2[2, 0] = 1            # ... and its scale: still one group
+    assert bench._group_mismatches(c2, s2, c, s) == 3
+    assert bench._group_mismatches(c, s, c, s) == 0

@@ -307,6 +307,42 @@ def test_block_scale_quotients_equal_the_ieee_divisions():
         _check_block_scale(amax, ts, n)
 
 
+def _markstein_div6(amax):
+    """The kernels' first quotient: q = fl(a * fl(1/6)), then one correction
+    q + fl(a - 6q) * fl(1/6) by fused multiply-adds (float64 arrays of
+    binary32 values)."""
+    a = amax.astype(np.float64)
+    n = a.size
+    r6 = float(np.float32(1.0) / np.float32(6.0))
+    q = (a * r6).astype(np.float32).astype(np.float64)
+    return _fma32_vec(_fma32_vec(-q, np.full(n, 6.0), a), np.full(n, r6), q)
+
+
+def test_amax_over_6_quotient_every_mantissa_and_exponent():
+    """fl(amax / 6) by the two-step quotient equals the IEEE division for
+    every one of the 2^23 binary32 values in [1, 2), and for 4096 mantissas
+    (the 2048 smallest and largest, random ones filling the rest to 4096)
+    of every binade from 2^-100 (below it the kernels divide) to the largest
+    finite float.  Away from under- and overflow, every step of both sides
+    scales exactly with a power of two, so the first binade covers every
+    mantissa of every binade; the sampled binades check the ends."""
+    one_binade = (np.arange(1 << 23, dtype=np.uint32) | np.uint32(127 << 23)).view(np.float32)
+    got = _markstein_div6(one_binade)
+    want = (one_binade / np.float32(6.0)).astype(np.float64)
+    assert np.array_equal(got, want)
+    rng = np.random.default_rng(29)
+    mant = np.concatenate([np.arange(1024), (1 << 23) - 1 - np.arange(1024),
+                           rng.integers(0, 1 << 23, 2048)]).astype(np.uint32)
+    exps = np.arange(27, 255, dtype=np.uint32)          # 2^-100 .. 2^127
+    bits = (exps[:, None] << np.uint32(23)) | mant[None, :]
+    amax = bits.ravel().view(np.float32)
+    with np.errstate(over="ignore"):
+        got = _markstein_div6(amax)
+        want = (amax / np.float32(6.0)).astype(np.float64)
+    bad = got != want
+    assert not bad.any(), amax[bad][:5]
+
+
 def _check_block_scale(amax, ts, n):
     a, t = amax.astype(np.float64), ts.astype(np.float64)
     r6 = float(np.float32(1.0) / np.float32(6.0))
