@@ -44,6 +44,73 @@ __device__ __forceinline__ uint32_t ld_nc_u8(const void *p)
     return v;
 }
 
+// --------------------------------------------- L2 eviction priority ----
+// A cache policy (createpolicy) passed with a load or store sets the L2
+// eviction priority of the lines it touches: evict_first lines are replaced
+// before normal ones, evict_last lines after them.
+
+__device__ __forceinline__ uint64_t l2_evict_first()
+{
+    uint64_t p;
+    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t l2_evict_normal()
+{
+    uint64_t p;
+    asm("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t l2_evict_last()
+{
+    uint64_t p;
+    asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void ld_nc_v8_pol(const void *p, uint32_t (&r)[8], uint64_t pol)
+{
+    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], %9;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]),
+          "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+        : "l"(p), "l"(pol));
+}
+
+__device__ __forceinline__ void ld_nc_v4_pol(const void *p, uint32_t &a, uint32_t &b, uint32_t &c,
+                                             uint32_t &d, uint64_t pol)
+{
+    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.b32 {%0,%1,%2,%3}, [%4], %5;"
+        : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "l"(p), "l"(pol));
+}
+
+__device__ __forceinline__ void st_v8_pol(void *p, const uint32_t (&r)[8], uint64_t pol)
+{
+    asm volatile("st.global.L1::no_allocate.L2::cache_hint.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8}, %9;"
+                 :: "l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]),
+                    "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "l"(pol) : "memory");
+}
+
+__device__ __forceinline__ void st_v4_pol(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                          uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1,%2,%3,%4}, %5;"
+                 :: "l"(p), "r"(a), "r"(b), "r"(c), "r"(d), "l"(pol) : "memory");
+}
+
+__device__ __forceinline__ void st_v2_pol(void *p, uint32_t a, uint32_t b, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.v2.b32 [%0], {%1,%2}, %3;"
+                 :: "l"(p), "r"(a), "r"(b), "l"(pol) : "memory");
+}
+
+__device__ __forceinline__ void st_u8_pol(void *p, uint32_t v, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.u8 [%0], %1, %2;"
+                 :: "l"(p), "h"((uint16_t)v), "l"(pol) : "memory");
+}
+
 __device__ __forceinline__ void st_v8(void *p, const uint32_t (&r)[8])
 {
     asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"

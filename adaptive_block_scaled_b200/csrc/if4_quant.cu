@@ -76,6 +76,33 @@ __device__ __forceinline__ void load_group(const char *p, Raw<DT> &r)
     }
 }
 
+// The same loads with an L2 cache policy.
+template <int DT, bool V8>
+__device__ __forceinline__ void load_group_pol(const char *p, Raw<DT> &r, uint64_t pol)
+{
+    if constexpr (DT == DT_F32) {
+        if constexpr (V8) {
+            uint32_t a[8], b[8];
+            ld_nc_v8_pol(p, a, pol);
+            ld_nc_v8_pol(p + 32, b, pol);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) { r.w[i] = a[i]; r.w[8 + i] = b[i]; }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                ld_nc_v4_pol(p + 16 * q, r.w[4 * q], r.w[4 * q + 1], r.w[4 * q + 2], r.w[4 * q + 3],
+                             pol);
+        }
+    } else {
+        if constexpr (V8) {
+            ld_nc_v8_pol(p, r.w, pol);
+        } else {
+            ld_nc_v4_pol(p, r.w[0], r.w[1], r.w[2], r.w[3], pol);
+            ld_nc_v4_pol(p + 16, r.w[4], r.w[5], r.w[6], r.w[7], pol);
+        }
+    }
+}
+
 // Unpack to 8 float pairs (element 2j low, 2j+1 high) and the group's max |x|
 // as float bits; *nonfinite is set for Inf/NaN.
 template <int DT>
@@ -483,9 +510,10 @@ __device__ __forceinline__ void decode_word(uint32_t w, uint32_t base, float (&q
 
 // Decode one group (code words w0, w1, scale byte sb) and store its 16
 // outputs at p.
-template <int ODT, bool UNIT_TS, bool V8 = false>
+// POL: the 16-bit outputs are stored with the L2 cache policy pol.
+template <int ODT, bool UNIT_TS, bool V8 = false, bool POL = false>
 __device__ __forceinline__ void dequant_group(uint32_t w0, uint32_t w1, uint32_t sb, float ts,
-                                              uint32_t lut_addr, char *p)
+                                              uint32_t lut_addr, char *p, uint64_t pol = 0)
 {
     const float e4 = f32_from_e4m3(sb);
     const float eff = UNIT_TS ? e4 : __fmul_rn(e4, ts);
@@ -533,8 +561,13 @@ __device__ __forceinline__ void dequant_group(uint32_t w0, uint32_t w1, uint32_t
         }
         // one 256-bit store fills a whole 32-byte sector; two 128-bit
         // stores would each write half of every sector they touch
-        if constexpr (V8) {
+        if constexpr (V8 && POL) {
+            st_v8_pol(p, o, pol);
+        } else if constexpr (V8) {
             st_v8(p, o);
+        } else if constexpr (POL) {
+            st_v4_pol(p, o[0], o[1], o[2], o[3], pol);
+            st_v4_pol(p + 16, o[4], o[5], o[6], o[7], pol);
         } else {
             st_v4(p, o[0], o[1], o[2], o[3]);
             st_v4(p + 16, o[4], o[5], o[6], o[7]);
@@ -543,8 +576,9 @@ __device__ __forceinline__ void dequant_group(uint32_t w0, uint32_t w1, uint32_t
 }
 
 // Encode group g from its raw bits r and store its codes and scale byte.
-// Returns true when an input element is Inf or NaN.
-template <int DT, int MODE, bool RHT, bool NV = false, bool DQ = false>
+// Returns true when an input element is Inf or NaN.  POL: every store
+// carries the L2 cache policy pol.
+template <int DT, int MODE, bool RHT, bool NV = false, bool DQ = false, bool POL = false>
 __device__ __forceinline__ bool quantize_one(const Raw<DT> &r, uint32_t g, const char *x,
                                              int64_t ld_bytes, uint32_t gpr, float ts, float rts,
                                              const float *inv_tab, const float *eff_tab,
@@ -552,7 +586,8 @@ __device__ __forceinline__ bool quantize_one(const Raw<DT> &r, uint32_t g, const
                                              const SignMasks &sm, uint32_t signs,
                                              uint8_t *nv_codes = nullptr,
                                              uint8_t *nv_scales = nullptr,
-                                             char *y = nullptr, uint32_t lut_addr = 0u)
+                                             char *y = nullptr, uint32_t lut_addr = 0u,
+                                             uint64_t pol = 0)
 {
     constexpr int GB = 16 * elem_bytes<DT>();
     f2_t xv[8];
@@ -581,18 +616,28 @@ __device__ __forceinline__ bool quantize_one(const Raw<DT> &r, uint32_t g, const
             out = encode_group<MODE, false>(xv, sb, inv, nullptr);
         if (sb == 0) out.c0 = out.c1 = out.scale = 0u;
     }
-    st_v2(codes + (int64_t)g * 8, out.c0, out.c1);
-    st_u8(scales + g, out.scale);
+    if constexpr (POL) {
+        st_v2_pol(codes + (int64_t)g * 8, out.c0, out.c1, pol);
+        st_u8_pol(scales + g, out.scale, pol);
+    } else {
+        st_v2(codes + (int64_t)g * 8, out.c0, out.c1);
+        st_u8(scales + g, out.scale);
+    }
     if constexpr (NV && MODE == Q_IF4) {
         // the NVFP4 comparator: the FP4 candidate under the same block scale
-        st_v2(nv_codes + (int64_t)g * 8, out.f0, out.f1);
-        st_u8(nv_scales + g, out.scale & 0x7Fu);
+        if constexpr (POL) {
+            st_v2_pol(nv_codes + (int64_t)g * 8, out.f0, out.f1, pol);
+            st_u8_pol(nv_scales + g, out.scale & 0x7Fu, pol);
+        } else {
+            st_v2(nv_codes + (int64_t)g * 8, out.f0, out.f1);
+            st_u8(nv_scales + g, out.scale & 0x7Fu);
+        }
     }
     if constexpr (DQ) {
         // the round trip: this group's IF4 codes decoded as the dequantizer
         // decodes them, bf16 into a dense 32-byte aligned y
-        dequant_group<DT_BF16, false, true>(out.c0, out.c1, out.scale, ts, lut_addr,
-                                            y + (int64_t)g * 32);
+        dequant_group<DT_BF16, false, true, POL>(out.c0, out.c1, out.scale, ts, lut_addr,
+                                                 y + (int64_t)g * 32, pol);
     }
     return nonfinite;
 }
@@ -832,7 +877,7 @@ quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr
                       uint8_t *__restrict__ scales, uint8_t *__restrict__ nv_codes,
                       uint8_t *__restrict__ nv_scales, float *ts_out, uint32_t *sync, int *err,
                       const __grid_constant__ SignMasks sm, uint32_t signs,
-                      char *__restrict__ y)
+                      char *__restrict__ y, uint32_t keep_from, int use_l2_policy)
 {
     // wait for the previous kernel in the stream (programmatic launch)
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -849,15 +894,26 @@ quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr
     const uint32_t stride = gridDim.x * blockDim.x;
     const uint32_t g_first = blockIdx.x * blockDim.x + threadIdx.x;
 
+    // L2 eviction priorities for a tensor larger than L2 can usefully keep
+    // (use_l2_policy): pass 1 reads the groups from keep_from on, the last it
+    // reads, with evict_last and the others with evict_first, so that at the
+    // barrier L2 holds the tensor's tail; pass 2 walks the tensor backwards,
+    // starting on that tail, and reads and writes with evict_first, so the
+    // stream of outputs replaces lines already used rather than the tail
+    // still to come.  Otherwise every access has the normal priority.
     // pass 1: max |x| (of the transform, with RHT), six loads in flight
     uint32_t m = 0;
     constexpr int U = (DT == DT_F32 || RHT) ? 3 : 6;
+    {
+    const uint64_t pol_first = use_l2_policy ? l2_evict_first() : l2_evict_normal();
+    const uint64_t pol_last = use_l2_policy ? l2_evict_last() : l2_evict_normal();
     for (uint64_t g0 = g_first; g0 < ngroups; g0 += (uint64_t)U * stride) {
         Raw<DT> r[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const uint64_t g = g0 + (uint64_t)u * stride;
-            if (g < ngroups) load_group<DT, V8>(addr((uint32_t)g), r[u]);
+            if (g < ngroups)
+                load_group_pol<DT, V8>(addr((uint32_t)g), r[u], g >= keep_from ? pol_last : pol_first);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u)
@@ -871,14 +927,18 @@ quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr
                 }
             }
     }
+    }
     m = __reduce_max_sync(0xFFFFFFFFu, m);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (lane == 0) warp_max[warp] = m;
-    // the encode pass's first group does not depend on ts: its load is in
-    // flight while the block waits at the grid barrier
+    const uint64_t pol_first = use_l2_policy ? l2_evict_first() : l2_evict_normal();
+    // pass 2 takes the j-th group of pass 1's order from the end: group
+    // ngroups - 1 - j.  Its first group does not depend on ts: that load is
+    // in flight while the block waits at the grid barrier.
+    auto rev = [&](uint32_t j) -> uint32_t { return ngroups - 1u - j; };
     Raw<DT> buf[2];
     uint32_t g = g_first;
-    if (g < ngroups) load_group<DT, V8>(addr(g), buf[0]);
+    if (g < ngroups) load_group_pol<DT, V8>(addr(rev(g)), buf[0], pol_first);
     __syncthreads();
     if (threadIdx.x == 0) {
         uint32_t b = 0;
@@ -908,10 +968,11 @@ quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr
 #pragma unroll
         for (int ph = 0; ph < 2; ++ph) {
             const uint32_t gn = g + stride;
-            if (gn < ngroups) load_group<DT, V8>(addr(gn), buf[ph ^ 1]);
-            quantize_one<DT, Q_IF4, RHT, NV, DQ>(buf[ph], g, x, ld_bytes, gpr_eff, ts, rts,
-                                                 inv_tab, nullptr, codes, scales, sm, signs,
-                                                 nv_codes, nv_scales, y, lut_addr);
+            if (gn < ngroups) load_group_pol<DT, V8>(addr(rev(gn)), buf[ph ^ 1], pol_first);
+            quantize_one<DT, Q_IF4, RHT, NV, DQ, true>(buf[ph], rev(g), x, ld_bytes, gpr_eff, ts,
+                                                       rts, inv_tab, nullptr, codes, scales, sm,
+                                                       signs, nv_codes, nv_scales, y, lut_addr,
+                                                       pol_first);
             g = gn;
             if (g >= ngroups) break;
         }
@@ -1229,6 +1290,14 @@ int quantize_entry(const void *x, int x_dtype, int64_t rows, int64_t cols, int64
                                      ts_mode == IF4_TS_GIVEN ? 1 : 0, st, d, signs);
 }
 
+// The single-launch quantizer's L2 eviction priorities (see the kernel):
+// used for inputs larger than 64 MB, keeping the last 48 MB in L2 for the
+// encode pass.  On the 134 MB activation tensor the keep size was swept from
+// 32 to 112 MB: 48 MB was fastest, and it cut the launch's DRAM reads from
+// 267 to 218 MB.
+constexpr uint64_t kL2PolicyMinBytes = 64ull << 20;
+constexpr uint64_t kL2KeepBytes = 48ull << 20;
+
 // Single-launch quantizer: a cooperative launch of at most one wave, so
 // every block is resident when the blocks meet at the grid barrier.
 template <int DT, bool V8, bool RHT, bool NV, bool DQ = false>
@@ -1252,9 +1321,15 @@ int launch_fused(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
+    // L2 eviction priorities for inputs above kL2PolicyMinBytes: the last
+    // kL2KeepBytes of the tensor are kept for the encode pass
+    const uint64_t in_bytes = (uint64_t)s.ngroups * (uint64_t)(16 * elem_bytes<DT>());
+    const bool use_pol = in_bytes > kL2PolicyMinBytes;
+    const uint64_t keep_groups = kL2KeepBytes / (uint64_t)(16 * elem_bytes<DT>());
+    const uint32_t keep_from = keep_groups >= s.ngroups ? 0u : (uint32_t)(s.ngroups - keep_groups);
     if (cudaLaunchKernelEx(&cfg, k, static_cast<const char *>(x), s.ld_bytes, s.gpr, s.ngroups,
                            s.contig ? 1 : 0, codes, scales, nv_codes, nv_scales, ts, sync, err, sm,
-                           signs, static_cast<char *>(y)) != cudaSuccess)
+                           signs, static_cast<char *>(y), keep_from, use_pol ? 1 : 0) != cudaSuccess)
         return IF4_ERR_CUDA;
     return launch_status();
 }
