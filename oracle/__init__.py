@@ -1,7 +1,9 @@
 """IF4 CPU oracle -- TEST INFRASTRUCTURE ONLY.
 
 Plain, slow, obviously-correct statement of what the IF4 quantizer computes,
-written from the pages on "Adaptive Block-Scaled Data Types".  The scalar
+written from the pages on "Adaptive Block-Scaled Data Types", and of the same
+adaptive choice at 6 and 3 bits (IF6, IF3; their grids are readings, not fixed
+by the pages).  The scalar
 arithmetic lives in ``if4_oracle.c`` (binary32 values, binary64 error sums);
 this module only marshals numpy arrays and adds the reductions that are plain
 library calls (means, the float64 matrix product for the linear).
@@ -68,6 +70,29 @@ def lib():
         L.orc_rht.argtypes = [_f32p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                               ctypes.c_uint32, _f32p, ctypes.c_int]
         L.orc_rht.restype = None
+        for name in ("orc_e2m3_code", "orc_int6_code", "orc_e2m0_code", "orc_int3_code"):
+            fn = getattr(L, name)
+            fn.argtypes = [ctypes.c_float]
+            fn.restype = ctypes.c_uint8
+        for name in ("orc_e2m3_value", "orc_int6_value", "orc_e2m0_value", "orc_int3_value"):
+            fn = getattr(L, name)
+            fn.argtypes = [ctypes.c_uint8]
+            fn.restype = ctypes.c_float
+        for name in ("orc_e2m3_code_array", "orc_int6_code_array", "orc_e2m0_code_array",
+                     "orc_int3_code_array"):
+            fn = getattr(L, name)
+            fn.argtypes = [_f32p, ctypes.c_int64, _u8p]
+            fn.restype = None
+        L.orc_tensor_scale_w.argtypes = [ctypes.c_float, ctypes.c_int]
+        L.orc_tensor_scale_w.restype = ctypes.c_float
+        L.orc_quantize_w.argtypes = [_f32p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                     ctypes.c_float, ctypes.c_int, ctypes.c_int, _u8p, _u8p,
+                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.c_int]
+        L.orc_quantize_w.restype = None
+        L.orc_dequantize_w.argtypes = [_u8p, _u8p, ctypes.c_float, ctypes.c_int64,
+                                       ctypes.c_int64, ctypes.c_int, _f32p, ctypes.c_int]
+        L.orc_dequantize_w.restype = None
         L.orc_max_threads.argtypes = []
         L.orc_max_threads.restype = ctypes.c_int
         _LIB = L
@@ -218,6 +243,113 @@ def linear(a_hat, b_hat, rows=None, cols=None):
     if cols is not None:
         b = b[np.asarray(cols)]
     return a @ b.T
+
+
+# --------------------------------------------------- other widths: IF6, IF3 --
+#
+# The same adaptive choice at 6 and 3 bits.  The pages name IF6 and IF3 but
+# fix neither grid; see if4_oracle.c for the readings (FP6 = E2M3 against a
+# 31-level INT6 reaching 7.5; FP3 = E2M0 {0, 1, 2, 4} against a 3-level INT3
+# reaching 4).  Codes: element i at bits [w*i, w*i + w) of the group's
+# little-endian bytes (12 per group for IF6, 6 for IF3).
+
+W_IF, W_FP, W_INT = 0, 1, 2
+
+
+def e2m3_code(v: float) -> int:
+    return int(lib().orc_e2m3_code(float(np.float32(v))))
+
+
+def e2m3_value(c: int) -> float:
+    return float(lib().orc_e2m3_value(int(c) & 0x3F))
+
+
+def int6_code(v: float) -> int:
+    return int(lib().orc_int6_code(float(np.float32(v))))
+
+
+def int6_value(c: int) -> float:
+    return float(lib().orc_int6_value(int(c) & 0x3F))
+
+
+def e2m0_code(v: float) -> int:
+    return int(lib().orc_e2m0_code(float(np.float32(v))))
+
+
+def e2m0_value(c: int) -> float:
+    return float(lib().orc_e2m0_value(int(c) & 0x7))
+
+
+def int3_code(v: float) -> int:
+    return int(lib().orc_int3_code(float(np.float32(v))))
+
+
+def int3_value(c: int) -> float:
+    return float(lib().orc_int3_value(int(c) & 0x7))
+
+
+def e2m3_code_array(values):
+    return _array_fn("orc_e2m3_code_array", values)
+
+
+def int6_code_array(values):
+    return _array_fn("orc_int6_code_array", values)
+
+
+def e2m0_code_array(values):
+    return _array_fn("orc_e2m0_code_array", values)
+
+
+def int3_code_array(values):
+    return _array_fn("orc_int3_code_array", values)
+
+
+def tensor_scale_w(amax, bits: int) -> np.float32:
+    """ts = amax/(fpmax*448) (fpmax 7.5 for 6 bits, 4 for 3); 1 for amax 0."""
+    return np.float32(lib().orc_tensor_scale_w(float(np.float32(amax)), int(bits)))
+
+
+def quantize_w(x, ts, bits: int, mode: int = W_IF, threads: int = 0):
+    """Quantize a [rows, cols] float32 array to IF6 / IF3 (bits 6 or 3), or to
+    the FP-only or INT-only candidate (mode W_FP / W_INT).  Returns dict(codes
+    uint8 [rows, cols*bits/8], scales uint8 [rows, cols/16], e_fp, e_int,
+    near) as quantize()."""
+    if bits not in (3, 6):
+        raise ValueError("bits must be 3 or 6")
+    x = _as_f32_2d(x)
+    rows, cols = x.shape
+    codes = np.zeros((rows, cols * bits // 8), np.uint8)
+    scales = np.zeros((rows, cols // 16), np.uint8)
+    e_fp = np.zeros((rows, cols // 16), np.float64)
+    e_int = np.zeros((rows, cols // 16), np.float64)
+    near = np.zeros((rows, cols // 16), np.uint8)
+    lib().orc_quantize_w(x, rows, cols, cols, float(np.float32(ts)), int(bits), int(mode), codes,
+                         scales, e_fp.ctypes.data, e_int.ctypes.data, near.ctypes.data,
+                         int(threads) if threads else max_threads())
+    return dict(codes=codes, scales=scales, e_fp=e_fp, e_int=e_int, near=near)
+
+
+def quantize_tensor_w(x, bits: int, mode: int = W_IF, threads: int = 0):
+    """Tensor amax, the width's tensor scale, then quantize_w."""
+    amax = tensor_amax(x)
+    ts = tensor_scale_w(amax, bits)
+    out = quantize_w(x, ts, bits, mode, threads)
+    out["amax"] = amax
+    out["ts"] = ts
+    return out
+
+
+def dequantize_w(codes, scales, ts, bits: int, threads: int = 0):
+    """float32 [rows, cols] = fl(q * fl(E4(scale) * ts)) at width bits."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, cols = scales.shape[0], scales.shape[1] * 16
+    if codes.shape != (rows, cols * bits // 8):
+        raise ValueError("codes must be [rows, cols*bits/8]")
+    y = np.zeros((rows, cols), np.float32)
+    lib().orc_dequantize_w(codes, scales, float(np.float32(ts)), rows, cols, int(bits), y,
+                           int(threads) if threads else max_threads())
+    return y
 
 
 def mse(x, xhat) -> float:

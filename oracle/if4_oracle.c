@@ -44,9 +44,14 @@
  *   its error is strictly lower; a group whose block scale rounds to zero is
  *   stored as all-zero FP4; the even element of a pair goes in the low nibble.
  *
+ * The same adaptive choice at 6 and 3 bits (IF6, IF3) is at the end of this
+ * file.  The pages name both but give neither grid; the grids used there
+ * (FP6 = E2M3 against a 31-level INT6, FP3 = E2M0 against a 3-level INT3)
+ * are readings, not fixed by the pages.
+ *
  * Parity pins: every function here is checked by the non-GPU tests against
- * brute force over the grids, a library float8 cast, closed-form values and
- * hand-worked groups; none is "parity unpinned".
+ * brute force over the grids, a library float8 cast, exact rationals,
+ * closed-form values and hand-worked groups; none is "parity unpinned".
  */
 #include <math.h>
 #include <stdint.h>
@@ -354,6 +359,241 @@ void orc_dequantize(const uint8_t *codes, const uint8_t *scales, float ts, int64
     (void)nthreads;
 }
 
+/* ------------------------------------------- other widths: IF6 and IF3 ---
+ *
+ * The pages apply the same adaptive choice at 3 and 6 bits (abstract: "the
+ * same insight ... for other bit-widths, including IF3 and IF6"; companion
+ * "It Generalizes: IF3 and IF6"; gist.science section 2 "Extensoes") but give
+ * neither grid.  Readings (each also listed in the design notes):
+ *   IF6: FP candidate E2M3 (sign, two exponent bits with bias 1, three
+ *        mantissa bits; magnitudes m/8 for exponent field 0, else
+ *        (1 + m/8) 2^(e-1); largest 7.5), INT candidate k in [-31, 31]
+ *        decoded as fl(15k/62) and chosen as the round-to-nearest-even of the
+ *        exact product v * fl(62/15), so both grids reach 7.5, as FP4 and the
+ *        7/6-scaled INT4 both reach 6.
+ *   IF3: FP candidate E2M0 (sign, two exponent bits, no mantissa: magnitudes
+ *        0, 1, 2, 4), INT candidate k in [-3, 3] decoded as fl(4k/3) and
+ *        chosen as the round-to-nearest-even of v * 3/4; both reach 4.
+ *   Both: the block scale is E4M3 of (amax/fpmax)/ts, the tensor scale
+ *        amax_T/(fpmax * 448), ties between equal candidate errors keep FP,
+ *        bit 7 of the scale byte set for INT, FP ties to the even code,
+ *        saturating; an FP zero keeps the sign of v; INT codes two's
+ *        complement.  Element i's code occupies bits [w*i, w*i + w) of the
+ *        group's little-endian code bytes (12 bytes per group for IF6, 6 for
+ *        IF3), so IF6 stores 6.5 and IF3 3.5 bits per value. */
+
+enum { ORC_W_IF = 0, ORC_W_FP = 1, ORC_W_INT = 2 };
+
+/* 6-bit E2M3 code of v: bit 5 = sign of v, bits 0-4 = magnitude code
+ * (exponent << 3 | mantissa), round to nearest with ties to the even code,
+ * saturating at 7.5.  The scalings by 8, 4 and 2 are exact. */
+uint8_t orc_e2m3_code(float v)
+{
+    uint8_t sign = signbit(v) ? 0x20 : 0;
+    double a = fabs((double)v);
+    int c;
+    if (!(a <= 7.5)) c = 31;                       /* above 7.5 (or NaN) */
+    else if (a < 1.0) c = (int)rint(a * 8.0);      /* step 1/8: codes 0..8 */
+    else if (a < 2.0) c = (int)rint(a * 8.0);      /* step 1/8: codes 8..16 */
+    else if (a < 4.0) c = (int)rint(a * 4.0) + 8;  /* step 1/4: codes 16..24 */
+    else c = (int)rint(a * 2.0) + 16;              /* step 1/2: codes 24..31 */
+    return (uint8_t)(sign | c);
+}
+
+float orc_e2m3_value(uint8_t code)
+{
+    int e = (code >> 3) & 3, m = code & 7;
+    double mag = e == 0 ? m / 8.0 : ldexp(1.0 + m / 8.0, e - 1);
+    return (float)((code & 0x20) ? -mag : mag);
+}
+
+/* k = RNE(v * fl(62/15)), the product exact in binary64, clamped to
+ * [-31, 31]; 6-bit two's complement. */
+uint8_t orc_int6_code(float v)
+{
+    const float c = 62.0f / 15.0f;
+    double k = rint((double)v * (double)c);
+    if (!(k >= -31.0)) k = -31.0;
+    if (k > 31.0) k = 31.0;
+    return (uint8_t)(((int)k) & 0x3F);
+}
+
+float orc_int6_value(uint8_t code)
+{
+    int k = (code & 0x20) ? (int)(code & 0x3F) - 64 : (int)(code & 0x3F);
+    return (float)(15 * k) / 62.0f;
+}
+
+/* 3-bit E2M0 code: bit 2 = sign of v, bits 0-1 = magnitude code of 0, 1, 2,
+ * 4; ties to the even code (0.5 -> 0, 1.5 -> 2, 3 -> 2), saturating at 4. */
+uint8_t orc_e2m0_code(float v)
+{
+    uint8_t sign = signbit(v) ? 4 : 0;
+    double a = fabs((double)v);
+    int c;
+    if (!(a <= 3.0)) c = 3;
+    else if (a >= 1.5) c = 2;
+    else if (a > 0.5) c = 1;
+    else c = 0;
+    return (uint8_t)(sign | c);
+}
+
+float orc_e2m0_value(uint8_t code)
+{
+    static const float mag[4] = {0.0f, 1.0f, 2.0f, 4.0f};
+    float m = mag[code & 3];
+    return (code & 4) ? -m : m;
+}
+
+/* k = RNE(v * 3/4) clamped to [-3, 3]; 3-bit two's complement. */
+uint8_t orc_int3_code(float v)
+{
+    double k = rint((double)v * 0.75);
+    if (!(k >= -3.0)) k = -3.0;
+    if (k > 3.0) k = 3.0;
+    return (uint8_t)(((int)k) & 0x7);
+}
+
+float orc_int3_value(uint8_t code)
+{
+    int k = (code & 4) ? (int)(code & 7) - 8 : (int)(code & 7);
+    return (float)(4 * k) / 3.0f;
+}
+
+static float width_fpmax(int bits) { return bits == 6 ? 7.5f : 4.0f; }
+
+/* Tensor scale of the width-`bits` format: amax/(fpmax * 448), 1 for a zero
+ * tensor, floored at 2^-117 as for IF4. */
+float orc_tensor_scale_w(float amax, int bits)
+{
+    const float floor_ts = 0x1p-117f;
+    if (amax == 0.0f) return 1.0f;
+    float ts = amax / (width_fpmax(bits) * 448.0f);
+    return ts < floor_ts ? floor_ts : ts;
+}
+
+static void put_code(uint8_t *bytes, int bits, int i, uint8_t code)
+{
+    for (int b = 0; b < bits; ++b)
+        if ((code >> b) & 1) {
+            int pos = bits * i + b;
+            bytes[pos >> 3] |= (uint8_t)(1u << (pos & 7));
+        }
+}
+
+static uint8_t get_code(const uint8_t *bytes, int bits, int i)
+{
+    uint8_t c = 0;
+    for (int b = 0; b < bits; ++b) {
+        int pos = bits * i + b;
+        c |= (uint8_t)(((bytes[pos >> 3] >> (pos & 7)) & 1u) << b);
+    }
+    return c;
+}
+
+/* One group of 16 at width `bits` (6 or 3): code bytes (2 * bits of them),
+ * returns the scale byte; the binary64 squared errors of both candidates in
+ * the scaled domain and the near-tie flag as for IF4. */
+static uint8_t quantize_group_w(const float *x, float ts, int bits, int mode, uint8_t *codes,
+                                double *e_fp_out, double *e_int_out, uint8_t *near_out)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    memset(codes, 0, (size_t)(2 * bits));
+    uint8_t sb = orc_e4m3_encode((amax / width_fpmax(bits)) / ts);
+    if (sb == 0) {
+        *e_fp_out = 0.0;
+        *e_int_out = 0.0;
+        *near_out = 1;
+        return 0x00;
+    }
+    float eff = orc_e4m3_value(sb) * ts;
+    float inv = 1.0f / eff;
+    uint8_t cf[16], ci[16];
+    double e_fp = 0.0, e_int = 0.0;
+    for (int i = 0; i < 16; ++i) {
+        float v = x[i] * inv;
+        float qf, qi;
+        if (bits == 6) {
+            cf[i] = orc_e2m3_code(v);
+            ci[i] = orc_int6_code(v);
+            qf = orc_e2m3_value(cf[i]);
+            qi = orc_int6_value(ci[i]);
+        } else {
+            cf[i] = orc_e2m0_code(v);
+            ci[i] = orc_int3_code(v);
+            qf = orc_e2m0_value(cf[i]);
+            qi = orc_int3_value(ci[i]);
+        }
+        double df = (double)v - (double)qf;
+        double di = (double)v - (double)qi;
+        e_fp = e_fp + df * df;
+        e_int = e_int + di * di;
+    }
+    int use_int = (mode == ORC_W_INT) || ((mode == ORC_W_IF) && (e_int < e_fp));
+    const uint8_t *c = use_int ? ci : cf;
+    for (int i = 0; i < 16; ++i) put_code(codes, bits, i, c[i]);
+    double hi = e_fp > e_int ? e_fp : e_int;
+    *e_fp_out = e_fp;
+    *e_int_out = e_int;
+    *near_out = (uint8_t)(fabs(e_fp - e_int) <= 1e-6 * hi);
+    return (uint8_t)(sb | (use_int ? 0x80 : 0x00));
+}
+
+/* x: float [rows, ld], cols % 16 == 0.  codes: [rows, cols * bits / 8],
+ * scales: [rows, cols/16].  mode: ORC_W_IF, ORC_W_FP or ORC_W_INT. */
+void orc_quantize_w(const float *x, int64_t rows, int64_t cols, int64_t ld, float ts, int bits,
+                    int mode, uint8_t *codes, uint8_t *scales, double *e_fp, double *e_int,
+                    uint8_t *near, int nthreads)
+{
+    int64_t gpr = cols / 16, cb = 2 * bits;
+#ifdef _OPENMP
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+#endif
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < gpr; ++g) {
+            double ef, ei;
+            uint8_t nt;
+            int64_t gi = r * gpr + g;
+            scales[gi] = quantize_group_w(x + r * ld + g * 16, ts, bits, mode,
+                                          codes + r * gpr * cb + g * cb, &ef, &ei, &nt);
+            if (e_fp) e_fp[gi] = ef;
+            if (e_int) e_int[gi] = ei;
+            if (near) near[gi] = nt;
+        }
+    }
+    (void)nthreads;
+}
+
+/* y[r, c] = fl(q * fl(E4(sb) * ts)), q decoded as FP or INT by bit 7. */
+void orc_dequantize_w(const uint8_t *codes, const uint8_t *scales, float ts, int64_t rows,
+                      int64_t cols, int bits, float *y, int nthreads)
+{
+    int64_t gpr = cols / 16, cb = 2 * bits;
+#ifdef _OPENMP
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+#endif
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < gpr; ++g) {
+            uint8_t sb = scales[r * gpr + g];
+            float eff = orc_e4m3_value(sb) * ts;
+            const uint8_t *gc = codes + r * gpr * cb + g * cb;
+            for (int i = 0; i < 16; ++i) {
+                uint8_t c = get_code(gc, bits, i);
+                float q = bits == 6 ? ((sb & 0x80) ? orc_int6_value(c) : orc_e2m3_value(c))
+                                    : ((sb & 0x80) ? orc_int3_value(c) : orc_e2m0_value(c));
+                y[r * cols + g * 16 + i] = q * eff;
+            }
+        }
+    }
+    (void)nthreads;
+}
+
 int orc_max_threads(void)
 {
 #ifdef _OPENMP
@@ -379,4 +619,24 @@ void orc_e2m1_nibble_array(const float *v, int64_t n, uint8_t *out)
 void orc_int4_nibble_array(const float *v, int64_t n, uint8_t *out)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = orc_int4_nibble(v[i]);
+}
+
+void orc_e2m3_code_array(const float *v, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_e2m3_code(v[i]);
+}
+
+void orc_int6_code_array(const float *v, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_int6_code(v[i]);
+}
+
+void orc_e2m0_code_array(const float *v, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_e2m0_code(v[i]);
+}
+
+void orc_int3_code_array(const float *v, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_int3_code(v[i]);
 }
