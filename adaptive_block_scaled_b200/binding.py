@@ -66,6 +66,10 @@ def _load():
         "if4_linear_noalloc": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
         "if4_linear_quantized": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
                                  ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp, _vp],
+        "if6_quantize": [_vp, _int, _i64, _i64, _i64, _int, _vp, _vp, _vp, _int, _vp, _vp],
+        "if3_quantize": [_vp, _int, _i64, _i64, _i64, _int, _vp, _vp, _vp, _int, _vp, _vp],
+        "if6_dequantize": [_vp, _vp, _vp, _i64, _i64, _vp, _int, _i64, _vp],
+        "if3_dequantize": [_vp, _vp, _vp, _i64, _i64, _vp, _int, _i64, _vp],
         "if4_status_str": [_int],
         "if4_version": [],
     }
@@ -286,6 +290,64 @@ def if4_linear_quantized(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, works
                                     workspace.numel() * workspace.element_size(), _ptr(c),
                                     _ptr(c_codes), _ptr(c_scales), _ptr(c_ts), _ptr(err_flag),
                                     _stream(stream)), "if4_linear_quantized")
+
+
+# ------------------------------------------------------- IF6 and IF3 ---
+
+W_ADAPTIVE, W_FP_ONLY, W_INT_ONLY = 0, 1, 2
+
+
+def _width_fns(bits):
+    if bits == 6:
+        return lib.if6_quantize, lib.if6_dequantize, "if6"
+    if bits == 3:
+        return lib.if3_quantize, lib.if3_dequantize, "if3"
+    raise ValueError("bits must be 6 or 3")
+
+
+def ifw_quantize(x, bits, mode, codes, scales, ts, ts_mode=TS_COMPUTE, err_flag=None,
+                 stream=None):
+    """if6_quantize / if3_quantize: codes uint8 [rows, cols*bits/8]."""
+    qfn, _, name = _width_fns(bits)
+    rows, cols, ld = _matrix(x, "x")
+    _u8(codes, "codes", (rows, cols * bits // 8))
+    _u8(scales, "scales", (rows, cols // 16))
+    if ts.dtype != torch.float32 or ts.numel() < 1:
+        raise ValueError("ts must be a float32 device tensor")
+    _check(qfn(_ptr(x), _dtype(x, "x"), rows, cols, ld, int(mode), _ptr(codes), _ptr(scales),
+               _ptr(ts), int(ts_mode), _ptr(err_flag), _stream(stream)), name + "_quantize")
+
+
+def ifw_dequantize(codes, scales, ts, bits, y, stream=None):
+    """if6_dequantize / if3_dequantize into y [rows, cols] (f32, bf16 or f16)."""
+    _, dfn, name = _width_fns(bits)
+    rows, cols, ld = _matrix(y, "y")
+    _u8(codes, "codes", (rows, cols * bits // 8))
+    _u8(scales, "scales", (rows, cols // 16))
+    _check(dfn(_ptr(codes), _ptr(scales), _ptr(ts), rows, cols, _ptr(y), _dtype(y, "y"), ld,
+               _stream(stream)), name + "_dequantize")
+
+
+def quantize_w(x, bits, mode=W_ADAPTIVE, ts=None, err_flag=None, stream=None):
+    """IF6 (bits=6) or IF3 (bits=3) of a 2-D tensor, or the FP-only / INT-only
+    candidate (mode).  Returns (codes, scales, ts); ts=None computes it."""
+    rows, cols, _ = _matrix(x, "x")
+    dev = x.device
+    codes = torch.empty((rows, cols * bits // 8), dtype=torch.uint8, device=dev)
+    scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+    if ts is None:
+        ts_t, ts_mode = torch.empty(1, dtype=torch.float32, device=dev), TS_COMPUTE
+    else:
+        ts_t, ts_mode = ts, TS_GIVEN
+    ifw_quantize(x, bits, mode, codes, scales, ts_t, ts_mode, err_flag, stream)
+    return codes, scales, ts_t
+
+
+def dequantize_w(codes, scales, ts, bits, dtype=torch.bfloat16, stream=None):
+    rows, cols = scales.shape[0], scales.shape[1] * 16
+    y = torch.empty((rows, cols), dtype=dtype, device=codes.device)
+    ifw_dequantize(codes, scales, ts, bits, y, stream)
+    return y
 
 
 LINEAR_NOALLOC_MAX_BYTES = 32 * 1024 * 1024

@@ -27,6 +27,7 @@ SOURCES = [
     ("if4_quant.cu", ["-fmad=false"]),
     ("if4_linear.cu", ["-fmad=false"]),   # shares the IF4 encoder (no contraction)
     ("if4_linear_noalloc.cu", []),
+    ("ifw_quant.cu", ["-fmad=false"]),    # IF6 / IF3: the same arithmetic contract
 ]
 HEADERS = ["if4_device.cuh", "if4_encode.cuh", "exports.map"]
 

@@ -1,0 +1,508 @@
+// IF6 and IF3: the adaptive FP/INT choice of IF4 at 6 and 3 bits, on B200
+// (sm_100a), and their C ABI.
+//
+// "Adaptive Block-Scaled Data Types" applies the IF4 idea to other bit widths
+// and names IF3 and IF6 (abstract; companion "It Generalizes: IF3 and IF6";
+// gist.science section 2 "Extensoes") without printing either grid.  The
+// readings this file implements, the same as the CPU oracle's:
+//   IF6: FP6 = E2M3 (largest 7.5) against INT6 k in [-31, 31] decoded as
+//        fl(15k/62) and chosen as RNE(v * fl(62/15)); both grids reach 7.5.
+//   IF3: FP3 = E2M0, magnitudes 0, 1, 2, 4, against INT3 k in [-3, 3] decoded
+//        as fl(4k/3) and chosen as RNE(v * 3/4); both reach 4.
+// Everything else follows IF4: block scale E4M3 of (amax/fpmax)/ts, tensor
+// scale amax_T/(fpmax*448), v = x * fl(1/fl(E4M3*ts)), the lower squared
+// error in the scaled domain wins with ties to FP, bit 7 of the scale byte
+// marks INT, an FP zero keeps the sign of v, INT codes are two's complement,
+// and element i's code sits at bits [w*i, w*i + w) of the group's
+// little-endian code bytes (12 per group for IF6, 6 for IF3).
+//
+// Design: one thread per group of 16 (a grid-stride loop with the next
+// group's load in flight), the FP rounding done with exact power-of-two
+// scalings and one round-to-nearest-even, the INT integer with one fused
+// multiply-add (a single rounding of the exact product), the INT values from
+// a shared table of correctly rounded quotients, and the decision from the
+// two binary64 error sums in element order, the rule itself.  These formats
+// are not on the bench's step, so the kernels favour plainness over the IF4
+// fast path's binary32 decision.
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/if4.h"
+#include "if4_device.cuh"
+
+using namespace if4dev;
+
+namespace {
+
+enum { W_IF = IF4_W_ADAPTIVE, W_FP = IF4_W_FP_ONLY, W_INT = IF4_W_INT_ONLY };
+
+template <int BITS>
+struct Width;
+
+template <>
+struct Width<6> {
+    static constexpr float fpmax = 7.5f;
+    static constexpr int kmax = 31;
+    static constexpr int code_bytes = 12;
+};
+
+template <>
+struct Width<3> {
+    static constexpr float fpmax = 4.0f;
+    static constexpr int kmax = 3;
+    static constexpr int code_bytes = 6;
+};
+
+constexpr float kMagic = 12582912.0f;           // 1.5 * 2^23
+
+// FP code of v: sign in the top bit of the width, magnitude code below.
+template <int BITS>
+__device__ __forceinline__ uint32_t fp_code(float v)
+{
+    const float a = fabsf(v);
+    uint32_t c;
+    if constexpr (BITS == 6) {
+        // E2M3: steps of 1/8 below 2, 1/4 below 4, 1/2 up to 7.5; the
+        // scalings by 8, 4 and 2 are exact, __float2int_rn is RNE
+        if (!(a <= 7.5f)) c = 31u;
+        else if (a < 2.0f) c = (uint32_t)__float2int_rn(__fmul_rn(a, 8.0f));
+        else if (a < 4.0f) c = (uint32_t)__float2int_rn(__fmul_rn(a, 4.0f)) + 8u;
+        else c = (uint32_t)__float2int_rn(__fmul_rn(a, 2.0f)) + 16u;
+        return c | (signbit(v) ? 0x20u : 0u);
+    } else {
+        // E2M0: 0, 1, 2, 4; ties to the even code (0.5 -> 0, 1.5 -> 2, 3 -> 2)
+        if (!(a <= 3.0f)) c = 3u;
+        else if (a >= 1.5f) c = 2u;
+        else if (a > 0.5f) c = 1u;
+        else c = 0u;
+        return c | (signbit(v) ? 4u : 0u);
+    }
+}
+
+// FP value of a code (exact in binary32).
+template <int BITS>
+__device__ __forceinline__ float fp_value(uint32_t code)
+{
+    float mag;
+    if constexpr (BITS == 6) {
+        const uint32_t e = (code >> 3) & 3u, m = code & 7u;
+        mag = e == 0 ? __fmul_rn((float)m, 0.125f)
+                     : ldexpf(__fadd_rn(1.0f, __fmul_rn((float)m, 0.125f)), (int)e - 1);
+        return (code & 0x20u) ? -mag : mag;
+    } else {
+        const uint32_t c = code & 3u;
+        mag = c == 0 ? 0.0f : (float)(1u << (c - 1));
+        return (code & 4u) ? -mag : mag;
+    }
+}
+
+// INT integer k = clamp(RNE(v * c), -kmax, kmax): one fused multiply-add
+// rounds the exact product once when |v| < 2^19 (the product then stays below
+// 2^22, where 1.5 * 2^23 + t keeps a unit ulp); beyond, k is clamped anyway.
+template <int BITS>
+__device__ __forceinline__ int int_k(float v, float c)
+{
+    constexpr int KM = Width<BITS>::kmax;
+    if (!(fabsf(v) < 0x1p19f)) return v < 0.0f ? -KM : KM;
+    const float r = __fmaf_rn(v, c, kMagic);
+    int k = (int)__fsub_rn(r, kMagic);
+    return k < -KM ? -KM : (k > KM ? KM : k);
+}
+
+template <int BITS>
+__device__ __forceinline__ uint32_t int_code(int k)
+{
+    return (uint32_t)k & ((1u << BITS) - 1u);
+}
+
+// Shared tables: the INT value of every code (index = code), filled with the
+// correctly rounded quotients 15k/62 or 4k/3.
+template <int BITS>
+__device__ __forceinline__ void fill_int_table(float *tab)
+{
+    constexpr int N = 1 << BITS;
+    for (int c = threadIdx.x; c < N; c += blockDim.x) {
+        const int k = (c & (N >> 1)) ? c - N : c;
+        tab[c] = BITS == 6 ? __fdiv_rn((float)(15 * k), 62.0f) : __fdiv_rn((float)(4 * k), 3.0f);
+    }
+}
+
+// 16 inputs of group g as floats.
+template <int DT>
+__device__ __forceinline__ void load16(const char *p, float (&x)[16])
+{
+    if constexpr (DT == IF4_F32) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t a, b, c, d;
+            ld_nc_v4(p + 16 * q, a, b, c, d);
+            x[4 * q] = __uint_as_float(a);
+            x[4 * q + 1] = __uint_as_float(b);
+            x[4 * q + 2] = __uint_as_float(c);
+            x[4 * q + 3] = __uint_as_float(d);
+        }
+    } else {
+        uint32_t w[8];
+        ld_nc_v4(p, w[0], w[1], w[2], w[3]);
+        ld_nc_v4(p + 16, w[4], w[5], w[6], w[7]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if constexpr (DT == IF4_BF16) {
+                x[2 * j] = __uint_as_float(w[j] << 16);
+                x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            } else {
+                x[2 * j] = f16lo_to_f32(w[j]);
+                x[2 * j + 1] = f16hi_to_f32(w[j]);
+            }
+        }
+    }
+}
+
+template <int DT>
+__host__ __device__ constexpr int ebytes() { return DT == IF4_F32 ? 4 : 2; }
+
+__device__ __forceinline__ const char *row_addr(const char *base, uint32_t g, uint32_t gpr,
+                                                int64_t ld_bytes, int gbytes)
+{
+    const uint32_t row = g / gpr;
+    return base + (int64_t)row * ld_bytes + (int64_t)(g - row * gpr) * gbytes;
+}
+
+// Store the 16 codes of a group, element i at bits [BITS*i, BITS*i + BITS).
+template <int BITS>
+__device__ __forceinline__ void store_codes(uint8_t *p, const uint32_t (&c)[16])
+{
+    uint64_t lo = 0, hi = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int pos = BITS * i;
+        if (pos + BITS <= 64) {
+            lo |= (uint64_t)c[i] << pos;
+        } else if (pos >= 64) {
+            hi |= (uint64_t)c[i] << (pos - 64);
+        } else {
+            lo |= (uint64_t)c[i] << pos;
+            hi |= (uint64_t)c[i] >> (64 - pos);
+        }
+    }
+    if constexpr (BITS == 6) {          // 12 bytes at a 4-byte aligned address
+        uint32_t *q = reinterpret_cast<uint32_t *>(p);
+        q[0] = (uint32_t)lo;
+        q[1] = (uint32_t)(lo >> 32);
+        q[2] = (uint32_t)hi;
+    } else {                            // 6 bytes at a 2-byte aligned address
+        uint16_t *q = reinterpret_cast<uint16_t *>(p);
+        q[0] = (uint16_t)lo;
+        q[1] = (uint16_t)(lo >> 16);
+        q[2] = (uint16_t)(lo >> 32);
+    }
+}
+
+template <int BITS>
+__device__ __forceinline__ void load_codes(const uint8_t *p, uint32_t (&c)[16])
+{
+    uint64_t lo, hi = 0;
+    if constexpr (BITS == 6) {
+        const uint32_t *q = reinterpret_cast<const uint32_t *>(p);
+        lo = (uint64_t)__ldg(q) | ((uint64_t)__ldg(q + 1) << 32);
+        hi = __ldg(q + 2);
+    } else {
+        const uint16_t *q = reinterpret_cast<const uint16_t *>(p);
+        lo = (uint64_t)__ldg(q) | ((uint64_t)__ldg(q + 1) << 16) | ((uint64_t)__ldg(q + 2) << 32);
+    }
+    constexpr uint64_t M = (1u << BITS) - 1u;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int pos = BITS * i;
+        if (pos + BITS <= 64) c[i] = (uint32_t)((lo >> pos) & M);
+        else if (pos >= 64) c[i] = (uint32_t)((hi >> (pos - 64)) & M);
+        else c[i] = (uint32_t)(((lo >> pos) | (hi << (64 - pos))) & M);
+    }
+}
+
+__device__ __forceinline__ bool ts_ok(float ts) { return ts >= 0x1p-117f && ts <= 0x1p117f; }
+
+// Quantizer: one group per thread per round of a grid-stride loop.
+template <int DT, int BITS>
+__global__ void __launch_bounds__(256)
+ifw_quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, uint32_t ngroups,
+                    int mode, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
+                    const float *__restrict__ ts_ptr, int *err, int check_ts)
+{
+    pdl_enter();
+    constexpr int GB = 16 * ebytes<DT>();
+    constexpr int CB = Width<BITS>::code_bytes;
+    __shared__ float int_tab[1 << BITS];
+    fill_int_table<BITS>(int_tab);
+    const float ts = *ts_ptr;
+    if (check_ts && blockIdx.x == 0 && threadIdx.x == 0 && !ts_ok(ts) && err)
+        atomicOr(err, IF4_DEV_BAD_SCALE);
+    const float c_int = BITS == 6 ? __fdiv_rn(62.0f, 15.0f) : 0.75f;
+    __syncthreads();
+    bool nonfinite = false;
+    const uint32_t stride = gridDim.x * blockDim.x;
+    for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < ngroups; g += stride) {
+        float xv[16];
+        load16<DT>(row_addr(x, g, gpr, ld_bytes, GB), xv);
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float a = fabsf(xv[i]);
+            nonfinite |= !(a <= 3.4028235e38f);
+            amax = a > amax ? a : amax;
+        }
+        const uint32_t sb =
+            e4m3_from_f32(__fdiv_rn(__fdiv_rn(amax, Width<BITS>::fpmax), ts)) & 0x7Fu;
+        uint32_t out[16];
+        uint32_t scale = 0;
+        if (sb == 0) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) out[i] = 0;
+        } else {
+            const float eff = __fmul_rn(f32_from_e4m3(sb), ts);
+            const float inv = __frcp_rn(eff);
+            uint32_t cf[16], ci[16];
+            double e_fp = 0.0, e_int = 0.0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float v = __fmul_rn(xv[i], inv);
+                cf[i] = fp_code<BITS>(v);
+                ci[i] = int_code<BITS>(int_k<BITS>(v, c_int));
+                const double df = __dsub_rn((double)v, (double)fp_value<BITS>(cf[i]));
+                const double di = __dsub_rn((double)v, (double)int_tab[ci[i]]);
+                e_fp = __dadd_rn(e_fp, __dmul_rn(df, df));
+                e_int = __dadd_rn(e_int, __dmul_rn(di, di));
+            }
+            const bool use_int = mode == W_INT || (mode == W_IF && e_int < e_fp);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) out[i] = use_int ? ci[i] : cf[i];
+            scale = sb | (use_int ? 0x80u : 0u);
+        }
+        store_codes<BITS>(codes + (int64_t)g * CB, out);
+        scales[g] = (uint8_t)scale;
+    }
+    if (nonfinite && err) atomicOr(err, IF4_DEV_NONFINITE);
+}
+
+// Dequantizer: y = fl(q * fl(E4M3 * ts)), rounded to the output type.
+template <int ODT, int BITS>
+__global__ void __launch_bounds__(256)
+ifw_dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+                      const float *__restrict__ ts_ptr, uint32_t gpr, uint32_t ngroups,
+                      char *__restrict__ y, int64_t ld_bytes)
+{
+    pdl_enter();
+    constexpr int CB = Width<BITS>::code_bytes;
+    constexpr int OB = ODT == IF4_F32 ? 4 : 2;
+    __shared__ float int_tab[1 << BITS];
+    __shared__ float fp_tab[1 << BITS];
+    fill_int_table<BITS>(int_tab);
+    for (int c = threadIdx.x; c < (1 << BITS); c += blockDim.x) fp_tab[c] = fp_value<BITS>(c);
+    const float ts = *ts_ptr;
+    __syncthreads();
+    const uint32_t stride = gridDim.x * blockDim.x;
+    for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < ngroups; g += stride) {
+        uint32_t c[16];
+        load_codes<BITS>(codes + (int64_t)g * CB, c);
+        const uint32_t sb = __ldg(scales + g);
+        const float eff = __fmul_rn(f32_from_e4m3(sb & 0x7Fu), ts);
+        const float *tab = (sb & 0x80u) ? int_tab : fp_tab;
+        float yv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) yv[i] = __fmul_rn(tab[c[i]], eff);
+        char *p = const_cast<char *>(row_addr(y, g, gpr, ld_bytes, 16 * OB));
+        if constexpr (ODT == IF4_F32) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                st_v4(p + 16 * q, __float_as_uint(yv[4 * q]), __float_as_uint(yv[4 * q + 1]),
+                      __float_as_uint(yv[4 * q + 2]), __float_as_uint(yv[4 * q + 3]));
+        } else {
+            uint32_t o[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                o[j] = ODT == IF4_BF16 ? bf16x2_from_f32(yv[2 * j], yv[2 * j + 1])
+                                       : f16x2_from_f32(yv[2 * j], yv[2 * j + 1]);
+            st_v4(p, o[0], o[1], o[2], o[3]);
+            st_v4(p + 16, o[4], o[5], o[6], o[7]);
+        }
+    }
+}
+
+// ts = amax / (fpmax * 448), 1 for amax == 0, floored at 2^-117; amax in *ts.
+template <int BITS>
+__global__ void ifw_tensor_scale_kernel(float *ts)
+{
+    pdl_enter();
+    const float a = *ts;
+    float t = 1.0f;
+    if (a != 0.0f) {
+        t = __fdiv_rn(a, Width<BITS>::fpmax * 448.0f);
+        if (t < 0x1p-117f) t = 0x1p-117f;
+    }
+    *ts = t;
+}
+
+// ------------------------------------------------------------ host side ----
+
+int elem_size(int dt) { return dt == IF4_F32 ? 4 : (dt == IF4_BF16 || dt == IF4_F16) ? 2 : 0; }
+
+struct Shape {
+    uint32_t gpr = 0, ngroups = 0;
+    int64_t ld_bytes = 0;
+};
+
+int check_tensor(const void *p, int dt, int64_t rows, int64_t cols, int64_t ld, Shape &s)
+{
+    const int es = elem_size(dt);
+    if (es == 0) return IF4_ERR_DTYPE;
+    if (rows < 0 || cols < 0 || cols % 16 != 0 || ld < cols) return IF4_ERR_SHAPE;
+    if (rows > 0 && (cols / 16) > 0 && rows > (int64_t)0x7FFFFFFF / (cols / 16)) return IF4_ERR_SHAPE;
+    if (rows > 0 && cols > 0 && p == nullptr) return IF4_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(p) % 16 != 0 || (ld * es) % 16 != 0) return IF4_ERR_ALIGN;
+    s.gpr = (uint32_t)(cols / 16);
+    s.ngroups = (uint32_t)(rows * (cols / 16));
+    s.ld_bytes = ld * es;
+    return IF4_OK;
+}
+
+int check_sm100()
+{
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return IF4_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return IF4_ERR_CUDA;
+    return major == 10 ? IF4_OK : IF4_ERR_DEVICE;
+}
+
+unsigned grid_size(uint32_t work)
+{
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const uint64_t want = ((uint64_t)work + 255) / 256;
+    const uint64_t cap = (uint64_t)sms * 8;
+    return (unsigned)(want < 1 ? 1 : (want < cap ? want : cap));
+}
+
+template <typename... KArgs, typename... Args>
+int launch(void (*k)(KArgs...), unsigned grid, cudaStream_t st, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k, args...) != cudaSuccess) return IF4_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? IF4_OK : IF4_ERR_CUDA;
+}
+
+template <int BITS>
+int quantize_w(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x, int mode,
+               uint8_t *codes, uint8_t *scales, float *ts, int ts_mode, int *err_flag,
+               void *stream)
+{
+    Shape s;
+    int rc = check_tensor(x, x_dtype, rows, cols, ld_x, s);
+    if (rc != IF4_OK) return rc;
+    if (mode != W_IF && mode != W_FP && mode != W_INT) return IF4_ERR_MODE;
+    if (ts_mode != IF4_TS_COMPUTE && ts_mode != IF4_TS_GIVEN) return IF4_ERR_MODE;
+    if (ts == nullptr) return IF4_ERR_NULL;
+    if (s.ngroups > 0 && (codes == nullptr || scales == nullptr)) return IF4_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(codes) % 4 != 0 || reinterpret_cast<uintptr_t>(ts) % 4 != 0)
+        return IF4_ERR_ALIGN;
+    rc = check_sm100();
+    if (rc != IF4_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (ts_mode == IF4_TS_COMPUTE) {
+        // max |x| into *ts (the IF4 amax pass), then the width's tensor scale
+        rc = if4_tensor_amax(x, x_dtype, rows, cols, ld_x, ts, err_flag, stream);
+        if (rc != IF4_OK) return rc;
+        rc = launch(ifw_tensor_scale_kernel<BITS>, 1, st, ts);
+        if (rc != IF4_OK) return rc;
+    }
+    if (s.ngroups == 0) return IF4_OK;
+    const unsigned grid = grid_size(s.ngroups);
+    const char *xc = static_cast<const char *>(x);
+    const int check = ts_mode == IF4_TS_GIVEN ? 1 : 0;
+    switch (x_dtype) {
+    case IF4_F32:
+        return launch(ifw_quantize_kernel<IF4_F32, BITS>, grid, st, xc, s.ld_bytes, s.gpr,
+                      s.ngroups, mode, codes, scales, (const float *)ts, err_flag, check);
+    case IF4_BF16:
+        return launch(ifw_quantize_kernel<IF4_BF16, BITS>, grid, st, xc, s.ld_bytes, s.gpr,
+                      s.ngroups, mode, codes, scales, (const float *)ts, err_flag, check);
+    default:
+        return launch(ifw_quantize_kernel<IF4_F16, BITS>, grid, st, xc, s.ld_bytes, s.gpr,
+                      s.ngroups, mode, codes, scales, (const float *)ts, err_flag, check);
+    }
+}
+
+template <int BITS>
+int dequantize_w(const uint8_t *codes, const uint8_t *scales, const float *ts, int64_t rows,
+                 int64_t cols, void *y, int y_dtype, int64_t ld_y, void *stream)
+{
+    Shape s;
+    int rc = check_tensor(y, y_dtype, rows, cols, ld_y, s);
+    if (rc != IF4_OK) return rc;
+    if (ts == nullptr) return IF4_ERR_NULL;
+    if (s.ngroups > 0 && (codes == nullptr || scales == nullptr)) return IF4_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(codes) % 4 != 0 || reinterpret_cast<uintptr_t>(ts) % 4 != 0)
+        return IF4_ERR_ALIGN;
+    rc = check_sm100();
+    if (rc != IF4_OK) return rc;
+    if (s.ngroups == 0) return IF4_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const unsigned grid = grid_size(s.ngroups);
+    char *yc = static_cast<char *>(y);
+    switch (y_dtype) {
+    case IF4_F32:
+        return launch(ifw_dequantize_kernel<IF4_F32, BITS>, grid, st, codes, scales, ts, s.gpr,
+                      s.ngroups, yc, s.ld_bytes);
+    case IF4_BF16:
+        return launch(ifw_dequantize_kernel<IF4_BF16, BITS>, grid, st, codes, scales, ts, s.gpr,
+                      s.ngroups, yc, s.ld_bytes);
+    default:
+        return launch(ifw_dequantize_kernel<IF4_F16, BITS>, grid, st, codes, scales, ts, s.gpr,
+                      s.ngroups, yc, s.ld_bytes);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int if6_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x, int mode,
+                 uint8_t *codes, uint8_t *scales, float *ts, int ts_mode, int *err_flag,
+                 void *stream)
+{
+    return quantize_w<6>(x, x_dtype, rows, cols, ld_x, mode, codes, scales, ts, ts_mode, err_flag,
+                         stream);
+}
+
+int if3_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x, int mode,
+                 uint8_t *codes, uint8_t *scales, float *ts, int ts_mode, int *err_flag,
+                 void *stream)
+{
+    return quantize_w<3>(x, x_dtype, rows, cols, ld_x, mode, codes, scales, ts, ts_mode, err_flag,
+                         stream);
+}
+
+int if6_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts, int64_t rows,
+                   int64_t cols, void *y, int y_dtype, int64_t ld_y, void *stream)
+{
+    return dequantize_w<6>(codes, scales, ts, rows, cols, y, y_dtype, ld_y, stream);
+}
+
+int if3_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts, int64_t rows,
+                   int64_t cols, void *y, int y_dtype, int64_t ld_y, void *stream)
+{
+    return dequantize_w<3>(codes, scales, ts, rows, cols, y, y_dtype, ld_y, stream);
+}
+
+}  // extern "C"

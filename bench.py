@@ -319,6 +319,12 @@ class Step:
                 nscales=torch.empty((self.rows, self.cols // 16), dtype=torch.uint8, device=dev),
                 sync=torch.zeros(64, dtype=torch.int32, device=dev),
                 ts_rht=torch.empty(1, dtype=torch.float32, device=dev),
+                codes6=torch.empty((self.rows, self.cols * 6 // 8), dtype=torch.uint8, device=dev),
+                codes3=torch.empty((self.rows, self.cols * 3 // 8), dtype=torch.uint8, device=dev),
+                scales6=torch.empty((self.rows, self.cols // 16), dtype=torch.uint8, device=dev),
+                scales3=torch.empty((self.rows, self.cols // 16), dtype=torch.uint8, device=dev),
+                ts6=torch.empty(1, dtype=torch.float32, device=dev),
+                ts3=torch.empty(1, dtype=torch.float32, device=dev),
             )
             self.sets.append(s)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -326,12 +332,22 @@ class Step:
                         "if4_quantize", "if4_dequantize", "nvfp4_quantize"]
         self.launches_per_step = 1
 
+    def init_widths(self):
+        """IF6 / IF3 tensor scales, codes and scales of every set (computed
+        once; their timed quantizers then take the tensor scale as given)."""
+        b = self.b
+        for s in self.sets:
+            for bits in (6, 3):
+                b.ifw_quantize(s["x"], bits, b.W_ADAPTIVE, s["codes%d" % bits],
+                               s["scales%d" % bits], s["ts%d" % bits], b.TS_COMPUTE, self.err)
+
     def bytes_per_set(self):
         s = self.sets[0]
         return sum(t.numel() * t.element_size() for t in s.values())
 
     EXTRA = ["nvint4_quantize", "nvfp4_4over6_quantize", "if4_quantize_rht", "if4_decode_f16",
-             "fused_quantize_rht"]
+             "fused_quantize_rht", "if6_quantize", "if6_dequantize", "if3_quantize",
+             "if3_dequantize"]
 
     def run_one(self, name, i):
         b, s = self.b, self.sets[i % len(self.sets)]
@@ -350,6 +366,17 @@ class Step:
             # the one the step and the quality report use
             b.if4_quantize_fused(s["x"], s["codes"], s["scales"], s["ncodes"], s["nscales"],
                                  s["ts_rht"], s["sync"], self.err, signs=RHT_SIGNS)
+            return
+        if name in ("if6_quantize", "if3_quantize"):
+            bits = 6 if name == "if6_quantize" else 3
+            # the width's own tensor scale, computed once before timing
+            b.ifw_quantize(s["x"], bits, b.W_ADAPTIVE, s["codes%d" % bits], s["scales%d" % bits],
+                           s["ts%d" % bits], b.TS_GIVEN, self.err)
+            return
+        if name in ("if6_dequantize", "if3_dequantize"):
+            bits = 6 if name == "if6_dequantize" else 3
+            b.ifw_dequantize(s["codes%d" % bits], s["scales%d" % bits], s["ts%d" % bits], bits,
+                             s["y"])
             return
         if name == "if4_decode_f16":
             b.if4_decode_f16(s["codes"], s["scales"], s["y"].view(torch.float16))
@@ -437,6 +464,8 @@ def kernel_times(step, names, reps, min_launches=32):
     out = {}
     sets = len(step.sets)
     n = sets * max(1, -(-min_launches // sets))
+    if any(k.startswith(("if6", "if3")) for k in names):
+        step.init_widths()
     for name in names:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
@@ -484,6 +513,7 @@ def quantizer_in_sequence(step, steps, sleep_cycles=int(4e7)):
 
 def kernel_table(ms, n_elem, in_bytes, pk):
     q_bytes = in_bytes + n_elem // 2 + n_elem // 16
+    w_bytes = {w: n_elem * w // 8 + n_elem // 16 for w in (6, 3)}     # IF6 / IF3 codes + scales
     dq_bytes = n_elem // 2 + n_elem // 16 + 2 * n_elem
     # the single-launch quantizer: x once, IF4 and NVFP4 codes and scales
     fused_bytes = in_bytes + 2 * (n_elem // 2 + n_elem // 16)
@@ -493,7 +523,9 @@ def kernel_table(ms, n_elem, in_bytes, pk):
               "if4_quantize": q_bytes, "if4_dequantize": dq_bytes,
               "nvfp4_quantize": q_bytes, "nvint4_quantize": q_bytes,
               "nvfp4_4over6_quantize": q_bytes, "if4_quantize_rht": q_bytes,
-              "if4_decode_f16": dq_bytes}
+              "if4_decode_f16": dq_bytes,
+              "if6_quantize": in_bytes + w_bytes[6], "if3_quantize": in_bytes + w_bytes[3],
+              "if6_dequantize": w_bytes[6] + 2 * n_elem, "if3_dequantize": w_bytes[3] + 2 * n_elem}
     table = {}
     for k, t in ms.items():
         b = nbytes[k]
@@ -540,7 +572,9 @@ def parity_quality(name, x_cpu=None):
     the oracle's near ties (candidate errors within 1e-6 relative, or a zero
     block scale), counted; the dequantized IF4 values against the oracle's,
     element by element; the MSE of each format in the x domain (float64, from
-    the library's dequantized output) and the IF4 INT4-group fraction."""
+    the library's dequantized output) and the IF4 INT4-group fraction; the
+    same for IF6 and IF3 (each with its own tensor scale) and their FP-only
+    formats."""
     import oracle
     from adaptive_block_scaled_b200 import binding as b
     if x_cpu is None:
@@ -572,6 +606,29 @@ def parity_quality(name, x_cpu=None):
                                                            rm["codes"], rm["scales"])
         ym = b.dequantize(cm, scm, ts, dtype=torch.float32).cpu().numpy()
         out["mse_" + mode] = float(np.mean((x64 - ym) ** 2))
+    # the same adaptive choice at 6 and 3 bits (IF6, IF3) and their FP-only
+    # formats, each against the oracle
+    for bits in (6, 3):
+        name = "if%d" % bits
+        rw = oracle.quantize_tensor_w(x_np, bits, oracle.W_IF)
+        cw, sw, tw = b.quantize_w(xd, bits, b.W_ADAPTIVE, err_flag=err)
+        cw_np, sw_np = cw.cpu().numpy(), sw.cpu().numpy()
+        bad = (cw_np.reshape(sw_np.size, -1) != rw["codes"].reshape(sw_np.size, -1)).any(axis=1)
+        out["mismatched_groups"][name] = int(np.count_nonzero(bad | (sw_np.reshape(-1) !=
+                                                                     rw["scales"].reshape(-1))))
+        out["near_ties_" + name] = int(rw["near"].sum())
+        out["ts_bit_identical_" + name] = bool(np.float32(tw.item()) == rw["ts"])
+        yw = b.dequantize_w(cw, sw, tw, bits, dtype=torch.float32).cpu().numpy()
+        out["mse_" + name] = float(np.mean((x64 - yw) ** 2))
+        out["int_group_fraction_" + name] = float(np.mean(sw_np >> 7))
+        fw = oracle.quantize_w(x_np, rw["ts"], bits, oracle.W_FP)
+        cf, sf, _ = b.quantize_w(xd, bits, b.W_FP_ONLY, ts=tw.clone(), err_flag=err)
+        cf_np, sf_np = cf.cpu().numpy(), sf.cpu().numpy()
+        badf = (cf_np.reshape(sf_np.size, -1) != fw["codes"].reshape(sf_np.size, -1)).any(axis=1)
+        out["mismatched_groups"]["fp%d" % bits] = int(np.count_nonzero(
+            badf | (sf_np.reshape(-1) != fw["scales"].reshape(-1))))
+        yf = b.dequantize_w(cf, sf, tw, bits, dtype=torch.float32).cpu().numpy()
+        out["mse_fp%d" % bits] = float(np.mean((x64 - yf) ** 2))
     torch.cuda.synchronize()
     out["device_error_flag"] = int(err.item())
     nv = out["mse_nvfp4"]

@@ -306,6 +306,57 @@ int if4_linear_quantized(const uint8_t *a_codes, const uint8_t *a_scales, const 
                          void *c, uint8_t *c_codes, uint8_t *c_scales, const float *c_ts,
                          int *err_flag, void *stream);
 
+/*
+ * IF6 and IF3: the same adaptive FP/INT choice at 6 and 3 bits per value.
+ * The pages name both formats and say the adaptive choice carries over to
+ * other bit widths ("Adaptive Block-Scaled Data Types", abstract; companion
+ * "It Generalizes: IF3 and IF6"; gist.science section 2, "Extensoes"), but
+ * print neither grid.  The grids below are this library's reading, not fixed
+ * by the pages:
+ *   IF6: FP6 = E2M3 (sign, 2 exponent bits with bias 1, 3 mantissa bits;
+ *        largest 7.5) against INT6 k in [-31, 31] decoded as fl(15k/62),
+ *        k = clamp(RNE(v * fl(62/15))); both grids end at 7.5.
+ *   IF3: FP3 = E2M0 (sign, magnitudes 0, 1, 2, 4) against INT3 k in [-3, 3]
+ *        decoded as fl(4k/3), k = clamp(RNE(v * 3/4)); both end at 4.
+ * Everything else is IF4's contract with fpmax (7.5 or 4) in place of 6:
+ * ts = amax_T/(fpmax*448) with IF4_TS_COMPUTE, sb = E4M3((amax_g/fpmax)/ts),
+ * v = x * fl(1/fl(E4M3(sb)*ts)), FP rounding to nearest with ties to the even
+ * code, saturating, an FP zero keeping the sign of v, INT codes in two's
+ * complement, the binary64 rule with ties to FP, bit 7 of the scale byte for
+ * INT, sb == 0 giving zero codes and byte 0x00.
+ *
+ * mode: IF4_W_ADAPTIVE (the lower-error candidate), IF4_W_FP_ONLY (the FP
+ * candidate everywhere, bit 7 clear: the fixed FP6/FP3 format at the same
+ * block scale) or IF4_W_INT_ONLY (the INT candidate everywhere, bit 7 set
+ * unless sb == 0).
+ *
+ * codes: uint8 [rows, cols*w/8] dense, w = 6 or 3: element i of a group is
+ * the w-bit field at bits [w*i, w*i + w) of the group's little-endian code
+ * bytes (12 bytes per group for IF6, 6 for IF3); 4-byte aligned base.
+ * scales: uint8 [rows, cols/16].  Storage: 6.5 and 3.5 bits per value.
+ * Other arguments, layouts and errors as if4_quantize (IF4_ERR_MODE also for
+ * an unknown mode).  These formats are off the bench's step; the kernels take
+ * the binary64 rule directly.
+ */
+enum { IF4_W_ADAPTIVE = 0, IF4_W_FP_ONLY = 1, IF4_W_INT_ONLY = 2 };
+
+int if6_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x, int mode,
+                 uint8_t *codes, uint8_t *scales, float *ts, int ts_mode, int *err_flag,
+                 void *stream);
+int if3_quantize(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x, int mode,
+                 uint8_t *codes, uint8_t *scales, float *ts, int ts_mode, int *err_flag,
+                 void *stream);
+
+/*
+ * Dequantize IF6 / IF3 (either mode's output): y = fl(q * fl(E4M3(sb & 0x7F)
+ * * ts)), q decoded as FP or INT by bit 7, rounded to y_dtype.  Layouts and
+ * errors as if4_dequantize; codes 4-byte aligned.
+ */
+int if6_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts, int64_t rows,
+                   int64_t cols, void *y, int y_dtype, int64_t ld_y, void *stream);
+int if3_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts, int64_t rows,
+                   int64_t cols, void *y, int y_dtype, int64_t ld_y, void *stream);
+
 /* Number of uint32 sync words if4_quantize_fused and its variants need. */
 #define IF4_FUSED_SYNC_WORDS 64u
 

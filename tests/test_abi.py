@@ -33,6 +33,9 @@ def lib():
     L.if4_linear_quantized.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, ctypes.c_size_t,
                                        vp, vp, vp, vp, vp, vp]
     L.if4_linear_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
+    for w in ("if6", "if3"):
+        getattr(L, w + "_quantize").argtypes = [vp, i, i64, i64, i64, i, vp, vp, vp, i, vp, vp]
+        getattr(L, w + "_dequantize").argtypes = [vp, vp, vp, i64, i64, vp, i, i64, vp]
     L.if4_status_str.restype = ctypes.c_char_p
     return L
 
@@ -65,7 +68,8 @@ def test_library_exports_every_declared_symbol(lib):
         assert n in exported, n
         assert hasattr(lib, n)
     # nothing but the C ABI leaks out (the static CUDA runtime stays local)
-    assert all(n.startswith(("if4_", "nvfp4_", "nvint4_")) for n in exported), sorted(exported)[:10]
+    assert all(n.startswith(("if4_", "if6_", "if3_", "nvfp4_", "nvint4_")) for n in exported), \
+        sorted(exported)[:10]
 
 
 def test_status_strings(lib):
@@ -156,6 +160,25 @@ def test_linear_noalloc_error_order(lib):
     assert f(A, A, A, A, A, A, 4096, 4096, 4104, A, A, None) == 2
     assert f(A, A, A, A, A, A, *big, A + 8, A, None) == 4     # c misaligned
     assert f(A, A, A, A, A, A, 0, 4096, 4096, A, A, None) == 2
+
+
+@pytest.mark.parametrize("w", ["if6", "if3"])
+def test_other_widths_host_validation(lib, w):
+    """IF6 / IF3 entry points reject invalid arguments before any launch."""
+    q = getattr(lib, w + "_quantize")
+    assert q(A, 1, 4, 24, 24, 0, A, A, A, 0, None, None) == 2          # cols % 16
+    assert q(A, 9, 4, 32, 32, 0, A, A, A, 0, None, None) == 3          # dtype
+    assert q(A, 1, 4, 32, 32, 3, A, A, A, 0, None, None) == 5          # mode
+    assert q(A, 1, 4, 32, 32, 0, A, A, A, 7, None, None) == 5          # ts_mode
+    assert q(A, 1, 4, 32, 32, 0, A, A, None, 0, None, None) == 1       # ts
+    assert q(A, 1, 4, 32, 32, 0, None, A, A, 0, None, None) == 1       # codes
+    assert q(A + 8, 1, 4, 32, 32, 0, A, A, A, 0, None, None) == 4      # x alignment
+    assert q(A, 1, 4, 32, 32, 0, A + 2, A, A, 0, None, None) == 4      # codes alignment
+    d = getattr(lib, w + "_dequantize")
+    assert d(None, A, A, 4, 32, A, 1, 32, None) == 1
+    assert d(A, A, A, 4, 40, A, 1, 40, None) == 2
+    assert d(A, A, A, 4, 32, A, 5, 32, None) == 3
+    assert d(A + 2, A, A, 4, 32, A, 1, 32, None) == 4
 
 
 def test_dequantize_and_decode_host_validation(lib):
