@@ -64,6 +64,7 @@ def _load():
         "if4_linear": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_size_t,
                        _vp, _vp, _vp],
         "if4_linear_noalloc": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
+        "if4_linear_fused": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
         "if4_linear_quantized": [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
                                  ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp, _vp],
         "if6_quantize": [_vp, _int, _i64, _i64, _i64, _int, _vp, _vp, _vp, _int, _vp, _vp],
@@ -254,6 +255,23 @@ def if4_linear(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, workspace, c, e
                           _ptr(b_scales), _ptr(b_ts), M, N, K, _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _ptr(c),
                           _ptr(err_flag), _stream(stream)), "if4_linear")
+
+
+def if4_linear_fused(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, c, err_flag,
+                     stream=None):
+    """The IF4 x IF4 linear with the operand decode inside the GEMM (no
+    workspace); the same C as if4_linear, bit for bit."""
+    M, N = c.shape
+    K = a_codes.shape[1] * 2
+    _u8(a_codes, "a_codes", (M, K // 2))
+    _u8(a_scales, "a_scales", (M, K // 16))
+    _u8(b_codes, "b_codes", (N, K // 2))
+    _u8(b_scales, "b_scales", (N, K // 16))
+    if c.dtype != torch.bfloat16 or not c.is_contiguous():
+        raise ValueError("c must be a contiguous bf16 tensor")
+    _check(lib.if4_linear_fused(_ptr(a_codes), _ptr(a_scales), _ptr(a_ts), _ptr(b_codes),
+                                _ptr(b_scales), _ptr(b_ts), M, N, K, _ptr(c), _ptr(err_flag),
+                                _stream(stream)), "if4_linear_fused")
 
 
 def if4_linear_noalloc(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, c, err_flag,

@@ -37,6 +37,13 @@ __device__ __forceinline__ uint32_t ld_nc_u32(const void *p)
     return v;
 }
 
+__device__ __forceinline__ uint32_t ld_nc_u16(const void *p)
+{
+    uint16_t v;
+    asm("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t ld_nc_u8(const void *p)
 {
     uint16_t v;

@@ -34,6 +34,7 @@
 #include <mutex>
 
 #include "../../include/if4.h"
+#include "if4_decode.cuh"
 #include "if4_encode.cuh"
 
 namespace {
@@ -724,6 +725,360 @@ gemm_f16_tcgen05_2sm(const __grid_constant__ CUtensorMap tmap_a,
     }
 }
 
+// ------------------------------------------- fused-decode CTA-pair GEMM ----
+//
+// The CTA-pair GEMM above with its TMA producer replaced by decoder warps,
+// so the IF4 operands are decoded inside the GEMM (the MAC of the companion
+// page "MAC Unit: Decoding Two Formats from One Sign Bit" routes each operand
+// through its group's decoder before the multiply) and no fp16 workspace is
+// needed.  The decoder threads of a CTA (TPR per row, 1 or 2) split its
+// operand slab (rows 0-127: A, 128-255: B) for every 64-wide K step: each
+// copies its part of a row's 32 code bytes, and the row's 4 scale bytes,
+// into a raw ring in shared memory with cp.async, two steps ahead (L2 serves
+// the re-reads across tiles), decodes them as if4_decode_f16 does (the
+// byte-permute decode, the same roundings, so the fp16 operands, and with the
+// same MMA order the product, equal if4_linear's bit for bit), and writes its
+// part of the row into the stage in the 128-byte swizzled layout the MMA
+// descriptors read (16-byte chunk j of row r at position j ^ (r & 7)).  A
+// proxy fence makes those generic stores visible to the tensor cores; then
+// one lane per warp arrives on the CTA's own decoder barrier, and one
+// forwarder thread per CTA relays the
+// completed stage to the leader CTA's MMA barrier (release.cluster).
+
+namespace fused {
+
+constexpr int DEC_WARP0 = 6;                          // after TMA-less warp 0, MMA, epilogue
+#ifndef IF4_FUSED_DEC_WARPS
+#define IF4_FUSED_DEC_WARPS 8
+#endif
+constexpr int DEC_WARPS = IF4_FUSED_DEC_WARPS;        // 8: a slab row per thread; 16: half
+constexpr int FNUM_THREADS = (DEC_WARP0 + DEC_WARPS) * 32;
+constexpr int TPR = DEC_WARPS * 32 / (2 * pair::PBM);  // decoder threads per slab row
+constexpr int GPT = 4 / TPR;                          // groups per thread per K step
+static_assert(TPR == 1 || TPR == 2, "one or two decoder threads per slab row");
+// Raw ring: per K step, the slab's code bytes as two 4 KB planes (16 bytes
+// of each row per plane, so a warp's 16-byte loads are conflict-free) and
+// the row's 4 scale bytes once per decoder thread.  Each decoder thread
+// fills and reads back its own part only, so cp.async's per-thread
+// wait_group is the only ordering needed.
+constexpr int RAW_STAGES = 3;
+constexpr int RAW_SCALE_OFF = 2 * 4096;
+constexpr int RAW_STAGE_BYTES = RAW_SCALE_OFF + TPR * 1024;
+constexpr int RAW_OFFSET = pair::PSTAGES * pair::PSTAGE_BYTES + 1024;   // after barriers, table
+constexpr int FSMEM_BYTES = RAW_OFFSET + RAW_STAGES * RAW_STAGE_BYTES + 1024;
+static_assert(FSMEM_BYTES <= 227 * 1024, "fused linear shared memory");
+
+// cp.async of 16 (or 4) bytes with zero fill of the bytes past src_bytes
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                 :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;"
+                 :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory");
+}
+
+__device__ __forceinline__ void lds_v4(uint32_t addr, uint32_t *w)
+{
+    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr) : "memory");
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// 16 fp16 values of one group (code words w0, w1, scale byte sb), scaled by
+// E4M3(sb) only, as if4_decode_f16 computes them: eight f16x2 words.
+__device__ __forceinline__ void decode_group_f16(uint32_t w0, uint32_t w1, uint32_t sb,
+                                                 uint32_t lut_addr, uint32_t (&o)[8])
+{
+    const float e4 = f32_from_e4m3(sb);
+    const uint32_t base = lut_addr + ((sb >> 1) & 0x40u);
+    float qa[8], qb[8];
+    decode_word(w0, base, qa);
+    decode_word(w1, base, qb);
+    const f2_t EFF = f2_pack(e4, e4);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float lo, hi;
+        f2_unpack(f2_mul(f2_pack(qa[2 * j], qa[2 * j + 1]), EFF), lo, hi);
+        o[j] = f16x2_from_f32(lo, hi);
+        f2_unpack(f2_mul(f2_pack(qb[2 * j], qb[2 * j + 1]), EFF), lo, hi);
+        o[4 + j] = f16x2_from_f32(lo, hi);
+    }
+}
+
+__device__ __forceinline__ void sts_v4(uint32_t addr, const uint32_t *w)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};"
+                 :: "r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
+}
+
+}  // namespace fused
+
+__global__ void __launch_bounds__(fused::FNUM_THREADS, 1)
+gemm_if4_fused_2sm(const uint8_t *__restrict__ a_codes, const uint8_t *__restrict__ a_scales,
+                   const uint8_t *__restrict__ b_codes, const uint8_t *__restrict__ b_scales,
+                   const float *__restrict__ a_ts, const float *__restrict__ b_ts,
+                   __nv_bfloat16 *__restrict__ c, int M, int N, int K, int *err)
+{
+    using namespace pair;
+    using namespace fused;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem_a = smem;
+    uint8_t *smem_b = smem + PSTAGES * PA_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + PSTAGES * PSTAGE_BYTES);
+    uint64_t *full = bars;                    // [PSTAGES], used in the leader
+    uint64_t *empty = bars + PSTAGES;          // [PSTAGES], both CTAs
+    uint64_t *acc_full = bars + 2 * PSTAGES;   // [2], both CTAs
+    uint64_t *acc_empty = acc_full + 2;       // [2], used in the leader
+    uint64_t *drain = acc_empty + 2;          // [1], leader
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    uint64_t *dec_full = drain + 2;           // [PSTAGES], both CTAs: this CTA's decoders
+    float *lut = reinterpret_cast<float *>(smem + PSTAGES * PSTAGE_BYTES + 256);
+    uint8_t *raw = smem + RAW_OFFSET;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cta_rank();
+    const bool leader = rank == 0;
+    const int m_tiles = (M + 2 * PBM - 1) / (2 * PBM);
+    const int n_tiles = (N + PBN - 1) / PBN;
+    const int tiles = m_tiles * n_tiles;
+    const int pair_id = blockIdx.x >> 1;
+    const int num_pairs = gridDim.x >> 1;
+    const int k_blocks = K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < PSTAGES; ++st) {
+            mbar_init(smem_u32(&full[st]), 2);           // one forwarder per CTA
+            mbar_init(smem_u32(&dec_full[st]), DEC_WARPS);
+            mbar_init(smem_u32(&empty[st]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&acc_full[b]), 1);
+            mbar_init(smem_u32(&acc_empty[b]), 2 * 4 * 32);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (threadIdx.x < 32) lut[threadIdx.x] = code_value(threadIdx.x);
+    if (warp == 1) {
+        __syncwarp();
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(tmem_slot)), "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                      // peer barriers initialised before any remote use
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    // programmatic launch: nothing above reads a kernel input
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    if (warp >= DEC_WARP0) {
+        // ------------------------------------------------------- decoders
+        // thread td owns part h = td / 256 (GPT of the 4 groups) of slab row
+        // td % 256 (rows 0-127 A, 128-255 B) in every K step
+        const int td = threadIdx.x - DEC_WARP0 * 32;
+        const int srow = td & 255, h = td >> 8;
+        const bool is_a = srow < PBM;
+        const int rloc = is_a ? srow : srow - PBM;              // row in this CTA's slab
+        const uint8_t *codes = is_a ? a_codes : b_codes;
+        const uint8_t *scales = is_a ? a_scales : b_scales;
+        const int rows_total = is_a ? M : N;
+        const uint32_t slab0 = smem_u32(is_a ? smem_a : smem_b) + (uint32_t)rloc * 128u;
+        const uint32_t sw = (uint32_t)(rloc & 7);
+        const uint32_t lut_addr = smem_u32(lut);
+        const uint32_t raw0 = smem_u32(raw);
+        // this thread's 16-byte code chunks c = h * (2 / TPR) + j (plane c, row
+        // srow) and its scale word
+        const uint32_t chunk0 = (uint32_t)h * (2u / TPR);
+        const uint32_t code_off = chunk0 * 4096u + (uint32_t)srow * 16u;
+        const uint32_t scale_off = RAW_SCALE_OFF + (uint32_t)td * 4u;
+        const int64_t code_stride = K / 2, scale_stride = K / 16;
+        const int my_tiles = pair_id < tiles ? (tiles - pair_id + num_pairs - 1) / num_pairs : 0;
+        const int64_t steps = (int64_t)my_tiles * k_blocks;
+        // Fetch side of the raw ring: copies step fi's code bytes of this
+        // thread's part and the row's 4 scale bytes (zero-filled past the
+        // matrix) into slot fslot, one commit group per step (an empty group
+        // past the end).
+        int ft = pair_id, fkb = 0, fslot = 0;
+        int64_t fi = 0;
+        auto fetch_next = [&]() {
+            if (fi < steps) {
+                const int row = (is_a ? (ft % m_tiles) * 2 * PBM + (int)rank * PBM
+                                      : (ft / m_tiles) * PBN + (int)rank * PBNH) + rloc;
+                const bool in = row < rows_total;
+                const int rr = in ? row : 0;
+                const uint8_t *src = codes + (int64_t)rr * code_stride + (int64_t)fkb * 32 +
+                                     16 * chunk0;
+                const uint32_t slot = raw0 + (uint32_t)fslot * RAW_STAGE_BYTES;
+#pragma unroll
+                for (int j = 0; j < 2 / TPR; ++j)
+                    cp_async16(slot + code_off + (uint32_t)j * 4096u, src + 16 * j, in ? 16u : 0u);
+                cp_async4(slot + scale_off,
+                          scales + (int64_t)rr * scale_stride + (int64_t)fkb * 4, in ? 4u : 0u);
+                if (++fkb == k_blocks) { fkb = 0; ft += num_pairs; }
+                ++fi;
+                if (++fslot == RAW_STAGES) fslot = 0;
+            }
+            cp_async_commit();
+        };
+#pragma unroll 1
+        for (int s = 0; s < RAW_STAGES - 1; ++s) fetch_next();
+        int stage = 0, rslot = 0;
+        uint32_t phase = 0;
+#pragma unroll 1
+        for (int64_t i = 0; i < steps; ++i) {
+            fetch_next();
+            cp_async_wait<RAW_STAGES - 1>();             // this thread's step i bytes landed
+            const uint32_t slot = raw0 + (uint32_t)rslot * RAW_STAGE_BYTES;
+            if (++rslot == RAW_STAGES) rslot = 0;
+            uint32_t w[2 * GPT];
+#pragma unroll
+            for (int j = 0; j < 2 / TPR; ++j) lds_v4(slot + code_off + (uint32_t)j * 4096u, w + 4 * j);
+            const uint32_t sc = lds_u32(slot + scale_off);
+            // the stage is free once the MMAs that read it have completed
+            bool freed = true;
+            if (lane == 0) freed = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag);
+            if (!__shfl_sync(0xFFFFFFFFu, freed ? 1 : 0, 0)) break;
+            const uint32_t dst = slab0 + (uint32_t)stage * (uint32_t)PA_BYTES;
+#pragma unroll
+            for (uint32_t j = 0; j < (uint32_t)GPT; ++j) {
+                const uint32_t g = (uint32_t)h * GPT + j;      // group in the 64-wide step
+                uint32_t o[8];
+                const uint32_t sb = (sc >> (8 * g)) & 0xFFu;
+                const float e4 = f32_from_e4m3(sb);
+                const uint32_t im = 0u - (sb >> 7);
+                const BytePlanes P = group_planes<false>(lut_addr + ((sb >> 1) & 0x40u), e4);
+                const uint32_t bad = decode_word16(w[2 * j], im, P, o) |
+                                     decode_word16(w[2 * j + 1], im, P, o + 4);
+                if (bad != 0u) decode_group_f16(w[2 * j], w[2 * j + 1], sb, lut_addr, o);
+                sts_v4(dst + (((2u * g) ^ sw) << 4), o);
+                sts_v4(dst + (((2u * g + 1u) ^ sw) << 4), o + 4);
+            }
+            // generic-proxy stores, then the MMA (async proxy) may read
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&dec_full[stage]));
+            if (++stage == PSTAGES) { stage = 0; phase ^= 1u; }
+        }
+        cp_async_wait<0>();                              // no copy in flight at exit
+    } else if (warp == 0 && lane == 0) {
+        // ------------------------------------------------------- forwarder
+        // Relays each stage from this CTA's decoders (CTA-scope barrier) to
+        // the leader's MMA barrier with one cluster-scope release, so the
+        // decoder threads, whose prefetches are in flight, never issue one.
+        const int my_tiles = pair_id < tiles ? (tiles - pair_id + num_pairs - 1) / num_pairs : 0;
+        const int64_t steps = (int64_t)my_tiles * k_blocks;
+        const uint32_t full_leader0 = map_to(smem_u32(&full[0]), 0);
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int64_t i = 0; i < steps; ++i) {
+            if (!mbar_wait(smem_u32(&dec_full[stage]), phase, abort_flag)) break;
+            arrive_remote(full_leader0 + (uint32_t)stage * 8u);
+            if (++stage == PSTAGES) { stage = 0; phase ^= 1u; }
+        }
+    } else if (warp == 1 && lane == 0 && leader) {
+        // ------------------------------------------- MMA issuer (leader)
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int t = pair_id; t < tiles && ok; t += num_pairs) {
+            if (!mbar_wait<true>(smem_u32(&acc_empty[acc]), acc_phase ^ 1u, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * PBN);
+            for (int kb = 0; kb < k_blocks; ++kb) {
+                // both CTAs' decoder warps arrive here with release.cluster
+                if (!mbar_wait<true>(smem_u32(&full[stage]), phase, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(smem_a + stage * PA_BYTES);
+                const uint32_t b0 = smem_u32(smem_b + stage * PB_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < BK / UMMA_K; ++kk)
+                    umma_f16_pair(d_tmem, smem_desc_sw128(a0 + kk * UMMA_K * 2),
+                                  smem_desc_sw128(b0 + kk * UMMA_K * 2), (kb | kk) != 0 ? 1u : 0u);
+                umma_commit_both(smem_u32(&empty[stage]));
+                if (++stage == PSTAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            umma_commit_both(smem_u32(&acc_full[acc]));
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                     :: "r"(smem_u32(drain)) : "memory");
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(smem_u32(drain), 0))
+            if (globaltimer() - t0 > WAIT_LIMIT_NS) break;
+    } else if (warp >= EPI_WARP0) {
+        // -------------------------------------------------------- epilogue
+        const int quarter = warp & 3;
+        const int row_in_cta = quarter * 32 + lane;
+        const float scale = __fmul_rn(*a_ts, *b_ts);
+        const OutQ oq{nullptr, nullptr, 1.0f, 1.0f, nullptr};
+        const uint32_t acc_empty_leader0 = map_to(smem_u32(&acc_empty[0]), 0);
+        const uint32_t acc_empty_leader1 = map_to(smem_u32(&acc_empty[1]), 0);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = pair_id; t < tiles; t += num_pairs) {
+            const int m0 = (t % m_tiles) * 2 * PBM + (int)rank * PBM;
+            const int n0 = (t / m_tiles) * PBN;
+            const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&acc_full[acc]), acc_phase,
+                                                              abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const int row = m0 + row_in_cta;
+#pragma unroll 1
+            for (int chunk = 0; chunk < PBN / 32; ++chunk) {
+                uint32_t r[32];
+                tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                              (uint32_t)(acc * PBN + chunk * 32), r);
+                store_chunk<false>(r, scale, row, M, N, n0 + chunk * 32, c, oq);
+            }
+            tc_fence_before();
+            arrive_remote(acc ? acc_empty_leader1 : acc_empty_leader0);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                      // the peer's MMAs and stores are done
+    if (threadIdx.x == 0 && *abort_flag && err) atomicOr(err, IF4_DEV_TIMEOUT);
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;"
+                     :: "r"(tmem_base), "r"(TMEM_COLS));
+    }
+}
+
 // ------------------------------------------------------------ host side ----
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -887,6 +1242,60 @@ int launch_gemm(const void *a, const void *b, const float *a_ts, const float *b_
     return launch_gemm_t<false>(a, b, a_ts, b_ts, M, N, K, o, err, st);
 }
 
+// The fused-decode linear: CTA pairs persistent over 256 x 256 tiles.
+int launch_fused(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *b_codes,
+                 const uint8_t *b_scales, const float *a_ts, const float *b_ts, int64_t M,
+                 int64_t N, int64_t K, void *c, int *err, cudaStream_t st)
+{
+    int sms = 0;
+    int rc = sm_count_checked(sms);
+    if (rc != IF4_OK) return rc;
+    if (sms < 2) return IF4_ERR_DEVICE;
+    auto kernel = gemm_if4_fused_2sm;
+    static std::once_flag attr_once;
+    static cudaError_t attr_rc = cudaSuccess;
+    std::call_once(attr_once, [&kernel] {
+        attr_rc = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       fused::FSMEM_BYTES);
+    });
+    if (attr_rc != cudaSuccess) return IF4_ERR_CUDA;
+    const int64_t tiles = ((M + 2 * pair::PBM - 1) / (2 * pair::PBM)) *
+                          ((N + pair::PBN - 1) / pair::PBN);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * (sms / 2)), 1, 1);
+    cfg.blockDim = dim3(fused::FNUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = fused::FSMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    static std::once_flag clusters_once;
+    static int resident_pairs = 0;
+    std::call_once(clusters_once, [&cfg, &kernel] {
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess)
+            resident_pairs = n;
+        else
+            (void)cudaGetLastError();
+    });
+    int64_t pairs = resident_pairs > 0 ? resident_pairs : sms / 2;
+    if (pairs > sms / 2) pairs = sms / 2;
+    if (tiles < pairs) pairs = tiles;
+    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kernel, a_codes, a_scales, b_codes, b_scales, a_ts, b_ts,
+                           static_cast<__nv_bfloat16 *>(c), (int)M, (int)N, (int)K, err) !=
+        cudaSuccess)
+        return IF4_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? IF4_OK : IF4_ERR_CUDA;
+}
+
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace
@@ -925,6 +1334,21 @@ int if4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_t
     rc = if4_decode_f16(b_codes, b_scales, N, K, wb, stream);
     if (rc != IF4_OK) return rc;
     return launch_gemm(wa, wb, a_ts, b_ts, M, N, K, c, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+int if4_linear_fused(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_ts,
+                     const uint8_t *b_codes, const uint8_t *b_scales, const float *b_ts, int64_t M,
+                     int64_t N, int64_t K, void *c, int *err_flag, void *stream)
+{
+    if (!a_codes || !a_scales || !b_codes || !b_scales) return IF4_ERR_NULL;
+    int rc = check_gemm_args(a_codes, b_codes, a_ts, b_ts, M, N, K, c, err_flag);
+    if (rc != IF4_OK) return rc;
+    if (K % 64 != 0) return IF4_ERR_SHAPE;
+    if (reinterpret_cast<uintptr_t>(a_codes) % 32 || reinterpret_cast<uintptr_t>(b_codes) % 32 ||
+        reinterpret_cast<uintptr_t>(a_scales) % 4 || reinterpret_cast<uintptr_t>(b_scales) % 4)
+        return IF4_ERR_ALIGN;
+    return launch_fused(a_codes, a_scales, b_codes, b_scales, a_ts, b_ts, M, N, K, c, err_flag,
+                        static_cast<cudaStream_t>(stream));
 }
 
 int if4_linear_quantized(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_ts,

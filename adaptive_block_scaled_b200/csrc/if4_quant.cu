@@ -37,6 +37,7 @@
 
 #include "../../include/if4.h"
 #include "if4_device.cuh"
+#include "if4_decode.cuh"
 #include "if4_encode.cuh"
 
 using namespace if4dev;
@@ -478,38 +479,10 @@ __device__ __forceinline__ uint32_t pack_out2(float a, float b)
     else return f16x2_from_f32(a, b);
 }
 
-// Decoded value of every code: lut[n] is the FP4 value of nibble n,
-// lut[16 + n] the INT4 value fl(6k/7) of nibble n (k its sign extension).
-// 32 floats, one per shared-memory bank, so any pattern of lookups by a warp
-// is conflict-free.
-__device__ __forceinline__ float code_value(uint32_t i)
-{
-    if (i < 16) {
-        const uint32_t h = f16x2_from_e2m1x2(i);      // nibble in bits 0-3
-        return f16lo_to_f32(h);
-    }
-    const float k = (float)((int)((i - 16) ^ 8u) - 8);
-    return __fmul_rn(k, c67());
-}
-
-__device__ __forceinline__ float lds_f32(uint32_t addr)
-{
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-    return v;
-}
-
-// 8 decoded values (not yet scaled) of the 8 nibbles of w; base is the
-// shared address of lut or lut + 16 floats.
-__device__ __forceinline__ void decode_word(uint32_t w, uint32_t base, float (&q)[8])
-{
-    q[0] = lds_f32(base + ((w << 2) & 0x3Cu));
-#pragma unroll
-    for (int i = 1; i < 8; ++i) q[i] = lds_f32(base + ((w >> (4 * i - 2)) & 0x3Cu));
-}
-
 // Decode one group (code words w0, w1, scale byte sb) and store its 16
-// outputs at p.
+// outputs at p: binary32 outputs by the per-element table; 16-bit outputs
+// by the byte-permute decode, and by the table when the group holds INT4
+// code 8 or eff is not finite with its sign bit clear (the same values).
 // POL: the 16-bit outputs are stored with the L2 cache policy pol.
 template <int ODT, bool UNIT_TS, bool V8 = false, bool POL = false>
 __device__ __forceinline__ void dequant_group(uint32_t w0, uint32_t w1, uint32_t sb, float ts,
@@ -518,17 +491,21 @@ __device__ __forceinline__ void dequant_group(uint32_t w0, uint32_t w1, uint32_t
     const float e4 = f32_from_e4m3(sb);
     const float eff = UNIT_TS ? e4 : __fmul_rn(e4, ts);
     const uint32_t base = lut_addr + ((sb >> 1) & 0x40u);        // INT4 half for bit 7
-    float qa[8], qb[8];
-    decode_word(w0, base, qa);
-    decode_word(w1, base, qb);
-    const f2_t EFF = f2_pack(eff, eff);
-    f2_t ya[4], yb[4];
+    // per-element table decode: values in binary32, then the output type
+    auto table_decode = [&](f2_t (&ya)[4], f2_t (&yb)[4]) {
+        float qa[8], qb[8];
+        decode_word(w0, base, qa);
+        decode_word(w1, base, qb);
+        const f2_t EFF = f2_pack(eff, eff);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        ya[j] = f2_mul(f2_pack(qa[2 * j], qa[2 * j + 1]), EFF);
-        yb[j] = f2_mul(f2_pack(qb[2 * j], qb[2 * j + 1]), EFF);
-    }
+        for (int j = 0; j < 4; ++j) {
+            ya[j] = f2_mul(f2_pack(qa[2 * j], qa[2 * j + 1]), EFF);
+            yb[j] = f2_mul(f2_pack(qb[2 * j], qb[2 * j + 1]), EFF);
+        }
+    };
     if constexpr (ODT == DT_F32) {
+        f2_t ya[4], yb[4];
+        table_decode(ya, yb);
         uint32_t a[8], b[8];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -551,13 +528,19 @@ __device__ __forceinline__ void dequant_group(uint32_t w0, uint32_t w1, uint32_t
         }
     } else {
         uint32_t o[8];
+        const uint32_t im = 0u - ((sb >> 7) & 1u);
+        const BytePlanes P = group_planes<ODT == DT_BF16>(base, eff);
+        const uint32_t bad = decode_word16(w0, im, P, o) | decode_word16(w1, im, P, o + 4);
+        if (bad != 0u || !permute_decode_ok(eff)) {
+            // per-element table decode, one pair at a time (few live values)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float lo, hi;
-            f2_unpack(ya[j], lo, hi);
-            o[j] = pack_out2<ODT>(lo, hi);
-            f2_unpack(yb[j], lo, hi);
-            o[4 + j] = pack_out2<ODT>(lo, hi);
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t w = i < 4 ? w0 : w1;
+                const int sh = 8 * (i & 3);
+                o[i] = pack_out2<ODT>(__fmul_rn(lds_f32(base + ((w >> sh << 2) & 0x3Cu)), eff),
+                                      __fmul_rn(lds_f32(base + ((w >> (sh + 4) << 2) & 0x3Cu)),
+                                                eff));
+            }
         }
         // one 256-bit store fills a whole 32-byte sector; two 128-bit
         // stores would each write half of every sector they touch

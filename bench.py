@@ -68,6 +68,7 @@ def parse():
                    help="skip the per-workload parity and quality block")
     p.add_argument("--kernel-only", default=None,
                    choices=["amax", "if4_quantize", "if4_dequantize", "nvfp4_quantize", "gemm",
+                            "linear_fused",
                             "nvint4_quantize", "nvfp4_4over6_quantize", "if4_quantize_rht",
                             "if4_decode_f16", "fused_quantize", "fused_quantize_rht",
                             "fused_quantize_dequant"],
@@ -785,6 +786,8 @@ def linear_report(pk, steps=20, warmup=3):
                                                c_codes, c_scales, c_ts, err_flag=err))
     t_sep = timed(lambda: (b.if4_linear(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], ws, c, err),
                            b.if4_quantize(c, c_codes, c_scales, c_ts, b.TS_GIVEN, err)))
+    # the decoders inside the GEMM (no workspace): the same C
+    t_fused = timed(lambda: b.if4_linear_fused(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], c, err))
     flops = 2.0 * M * N * K
     gemm_tf = flops / (t[2] * 1e-3) / 1e12
     total = sum(t)
@@ -793,6 +796,8 @@ def linear_report(pk, steps=20, warmup=3):
             "gemm_tflops": gemm_tf, "linear_tflops": flops / (total * 1e-3) / 1e12,
             "cublas_f16_ms": t_cublas, "cublas_f16_tflops": flops / (t_cublas * 1e-3) / 1e12,
             "linear_if4_out_ms": t_q, "linear_then_quantize_ms": t_sep,
+            "linear_fused_decode_ms": t_fused,
+            "linear_fused_decode_tflops": flops / (t_fused * 1e-3) / 1e12,
             "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": pk["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": gemm_tf / pk["bf16_tflops"],
                          "peak_source": f"{pk['source']} bf16_tflops (burst); fp16 dense rate = bf16"}}
@@ -964,7 +969,7 @@ def run_ours(args):
 def run_kernel_only(args):
     """Only the chosen kernel, on the chosen workload: the command ncu wraps."""
     from adaptive_block_scaled_b200 import binding as b
-    if args.kernel_only == "gemm":
+    if args.kernel_only in ("gemm", "linear_fused"):
         M, N, K = 8192, 4096, 4096
         a, bw = make_input("linear_8192x4096x4096")
         dev = torch.device("cuda")
@@ -973,9 +978,12 @@ def run_kernel_only(args):
         c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         err = torch.zeros(1, dtype=torch.int32, device=dev)
         for _ in range(args.warmup + args.steps):
-            b.if4_gemm_f16(wa, wb, aq[2], bq[2], c, err)
+            if args.kernel_only == "gemm":
+                b.if4_gemm_f16(wa, wb, aq[2], bq[2], c, err)
+            else:
+                b.if4_linear_fused(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], c, err)
         torch.cuda.synchronize()
-        print(json.dumps({"kernel_only": "gemm", "launches": args.warmup + args.steps,
+        print(json.dumps({"kernel_only": args.kernel_only, "launches": args.warmup + args.steps,
                           "err": int(err.item())}))
         if int(err.item()) != 0:
             sys.exit(1)

@@ -281,6 +281,25 @@ int if4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_t
                void *c, int *err_flag, void *stream);
 
 /*
+ * IF4 x IF4 linear with the decoders inside the GEMM: the same C as
+ * if4_linear, bit for bit, without a workspace.  The pages' MAC decodes each
+ * operand by its group's sign bit right before the multiply (companion, "MAC
+ * Unit: Decoding Two Formats from One Sign Bit"); here warps of the GEMM
+ * decode each 64-wide K step of both operands from the IF4 codes into the
+ * tensor cores' shared-memory operand stages, so the fp16 operands never
+ * exist in global memory.  Each operand row is decoded once per output tile
+ * that uses it, so the decode work is repeated N/256 times for A and M/256
+ * times for B (the separate decode of if4_linear runs once per element).
+ *
+ * K % 64 == 0; a_codes and b_codes 32-byte aligned, a_scales and b_scales
+ * 4-byte aligned (row strides K/2 and K/16 bytes); other rules, errors and
+ * err_flag as if4_linear (IF4_ERR_SHAPE for K % 64 != 0).
+ */
+int if4_linear_fused(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_ts,
+                     const uint8_t *b_codes, const uint8_t *b_scales, const float *b_ts,
+                     int64_t M, int64_t N, int64_t K, void *c, int *err_flag, void *stream);
+
+/*
  * IF4 x IF4 linear with an IF4 output: the product of if4_linear, rounded to
  * bf16 exactly as there, then quantized to IF4 along N (groups of 16
  * columns of each row of C) under the given tensor scale *c_ts, inside the

@@ -181,6 +181,16 @@ def test_other_widths_host_validation(lib, w):
     assert d(A + 2, A, A, 4, 32, A, 1, 32, None) == 4
 
 
+def test_linear_fused_host_validation(lib):
+    f = lib.if4_linear_fused
+    f.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int64] * 3 + [ctypes.c_void_p] * 3
+    assert f(None, A, A, A, A, A, 128, 256, 64, A, A, None) == 1
+    assert f(A, A, A, A, A, A, 128, 256, 80, A, A, None) == 2      # K % 64
+    assert f(A + 16, A, A, A, A, A, 128, 256, 64, A, A, None) == 4  # codes not 32-byte aligned
+    assert f(A, A + 2, A, A, A, A, 128, 256, 64, A, A, None) == 4   # scales not 4-byte aligned
+    assert f(A, A, A, A, A, A, 128, 252, 64, A, A, None) == 2      # N % 8
+
+
 def test_dequantize_and_decode_host_validation(lib):
     f = lib.if4_dequantize
     assert f(None, A, A, 4, 32, A, 1, 32, None) == 1

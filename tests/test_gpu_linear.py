@@ -226,3 +226,71 @@ def test_linear_quantized_output_full_workload():
     ref = oracle.quantize(c.float().cpu().numpy(), np.float32(c_ts.item()))
     assert np.array_equal(scales.cpu().numpy(), ref["scales"])
     assert np.array_equal(codes.cpu().numpy(), ref["codes"])
+
+
+# ------------------------------------------------ fused-decode linear ----
+
+def _linear_fused(aq, bq, M, N):
+    bb = B()
+    c = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bb.if4_linear_fused(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], c, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    return c
+
+
+@pytest.mark.parametrize("M,N,K", [(512, 512, 4096), (256, 256, 64), (200, 264, 1024),
+                                   (1, 8, 64), (777, 520, 2048), (1024, 1536, 512)])
+def test_fused_linear_equals_linear(M, N, K):
+    """The decoders inside the GEMM produce the same fp16 operands as
+    if4_decode_f16 and the MMAs accumulate in the same order, so C equals
+    if4_linear's bit for bit (and so is within the linear's 1e-2 of the
+    float64 product); shapes include partial tiles on both sides."""
+    a, b = workloads.linear_operands(4, M=M, N=N, K=K)
+    aq, bq = _quantized(a), _quantized(b)
+    want = _linear(aq, bq, M, N, K)
+    got = _linear_fused(aq, bq, M, N)
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16)), (M, N, K)
+    if M * N <= 512 * 512:
+        ref = oracle.linear(_dequant_ref(aq), _dequant_ref(bq))
+        assert _rel(got.float().cpu().numpy(), ref) <= 1e-2
+
+
+def test_fused_linear_full_workload():
+    M, N, K = 8192, 4096, 4096
+    a, b = workloads.linear_operands(0, M=M, N=N, K=K)
+    aq, bq = _quantized(a), _quantized(b)
+    want = _linear(aq, bq, M, N, K)
+    got = _linear_fused(aq, bq, M, N)
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+
+
+def test_fused_linear_arbitrary_code_bytes():
+    """Random code and scale bytes (INT4 code 8 included, which the encoder
+    never emits and the byte-permute decode hands to the per-element table):
+    the fused-decode linear still equals if4_linear bit for bit."""
+    M, N, K = 384, 520, 1024
+    rng = np.random.default_rng(11)
+
+    def operand(rows):
+        c = torch.from_numpy(rng.integers(0, 256, (rows, K // 2), dtype=np.uint8)).cuda()
+        s = torch.from_numpy(rng.integers(0, 256, (rows, K // 16), dtype=np.uint8)).cuda()
+        s[0, :] |= 0x80
+        c[0, :] = 0x88                  # a row of INT4 groups holding code 8 only
+        return c, s, torch.tensor([0.0125], dtype=torch.float32, device="cuda")
+
+    aq, bq = operand(M), operand(N)
+    want = _linear(aq, bq, M, N, K)
+    got = _linear_fused(aq, bq, M, N)
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+
+
+def test_fused_linear_rejects_k_not_multiple_of_64():
+    bb = B()
+    a, b = workloads.linear_operands(5, M=64, N=64, K=80)
+    aq, bq = _quantized(a), _quantized(b)
+    c = torch.empty((64, 64), dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(bb.IF4Error, match="shape"):
+        bb.if4_linear_fused(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], c, err)

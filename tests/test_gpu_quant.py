@@ -249,6 +249,55 @@ def test_decode_f16_matches_oracle():
     assert np.array_equal(d.view(np.uint16), ref.view(np.uint16))
 
 
+def _same_or_both_nan(got, want):
+    """Bit equality, except that any two NaNs match (payloads differ between
+    the GPU's and the host's invalid operations)."""
+    g, w = got.float().numpy(), want.float().numpy()
+    gb = got.view(torch.int16 if got.dtype != torch.float32 else torch.int32).numpy()
+    wb = want.view(torch.int16 if want.dtype != torch.float32 else torch.int32).numpy()
+    return bool(np.all((gb == wb) | (np.isnan(g) & np.isnan(w))))
+
+
+def _arbitrary_codes(seed, rows=64, cols=4096):
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 256, (rows, cols // 2), dtype=np.uint8)
+    scales = np.tile(np.arange(256, dtype=np.uint8), rows * cols // 16 // 256)
+    scales = rng.permutation(scales).reshape(rows, cols // 16)
+    codes[0, :] = 0x88                  # every nibble 8: INT4 k = -8, FP4 -0
+    return codes, scales
+
+
+@pytest.mark.parametrize("ts", [1.0, 0.3719, 3.0e-3, 211.5, 1.0e38, -0.5, -0.0, 0.0,
+                                float("inf"), float("nan")])
+def test_dequantize_every_scale_byte_arbitrary_codes(ts):
+    """Arbitrary code bytes (INT4 code 8 included, which the encoder never
+    emits) under every scale byte and degenerate tensor scales.  The 16-bit
+    outputs take the byte-permute decode, or the per-element table for INT4
+    code 8 and for a scale that is not finite with its sign bit clear; every
+    output equals the oracle's dequantization."""
+    b = B()
+    codes, scales = _arbitrary_codes(int(abs(ts) * 10) % 97 if np.isfinite(ts) else 5)
+    ts32 = np.float32(ts)
+    y_ref = oracle.dequantize(codes, scales, ts32)
+    c, s = torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda()
+    t = torch.tensor([ts32], dtype=torch.float32, device="cuda")
+    for dt in (torch.float32, torch.bfloat16, torch.float16):
+        y = b.dequantize(c, s, t, dtype=dt).cpu()
+        assert _same_or_both_nan(y, torch.from_numpy(y_ref).to(dt)), (ts, dt)
+
+
+def test_decode_f16_arbitrary_codes():
+    """As above for the linear's fp16 operand decode (scale bytes 0x7F and
+    0xFF are E4M3 NaN: their groups decode to NaN on both sides)."""
+    b = B()
+    codes, scales = _arbitrary_codes(9)
+    d = b.decode_f16(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda()).cpu()
+    ref = torch.from_numpy(oracle.decode_f16(codes, scales))
+    assert _same_or_both_nan(d, ref)
+    finite = np.isfinite(ref.numpy())
+    assert np.array_equal(d.numpy().view(np.uint16)[finite], ref.numpy().view(np.uint16)[finite])
+
+
 def test_tensor_amax_and_scale_entry_points():
     b = B()
     x = workloads.activation_outliers(1, tokens=512, hidden=1024)
