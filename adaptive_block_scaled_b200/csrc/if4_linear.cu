@@ -53,6 +53,10 @@ constexpr int EPI_WARP0 = 2;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
                            512 /*inverse block scales of the IF4 output*/;
 constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;   // 1 s per wait
+// mbarrier.try_wait suspends the thread until the phase completes or this
+// many ns pass, instead of returning at once; a waiting warp then takes no
+// issue slots from the warps beside it on its scheduler.
+constexpr int WAIT_HINT_NS = 20000;
 
 // instruction descriptor, kind::f16: D f32, A f16, B f16, both K-major,
 // N = 256, M = 128
@@ -93,9 +97,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+                 : "=r"(ok) : "r"(bar), "r"(parity), "n"(WAIT_HINT_NS) : "memory");
     return ok != 0;
 }
 
@@ -105,9 +109,9 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 {
     uint32_t ok;
     asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+                 : "=r"(ok) : "r"(bar), "r"(parity), "n"(WAIT_HINT_NS) : "memory");
     return ok != 0;
 }
 
@@ -731,41 +735,51 @@ gemm_f16_tcgen05_2sm(const __grid_constant__ CUtensorMap tmap_a,
 // so the IF4 operands are decoded inside the GEMM (the MAC of the companion
 // page "MAC Unit: Decoding Two Formats from One Sign Bit" routes each operand
 // through its group's decoder before the multiply) and no fp16 workspace is
-// needed.  The decoder threads of a CTA (TPR per row, 1 or 2) split its
-// operand slab (rows 0-127: A, 128-255: B) for every 64-wide K step: each
-// copies its part of a row's 32 code bytes, and the row's 4 scale bytes,
-// into a raw ring in shared memory with cp.async, two steps ahead (L2 serves
-// the re-reads across tiles), decodes them as if4_decode_f16 does (the
-// byte-permute decode, the same roundings, so the fp16 operands, and with the
-// same MMA order the product, equal if4_linear's bit for bit), and writes its
-// part of the row into the stage in the 128-byte swizzled layout the MMA
+// needed.  Two sets of decoder warps take the K steps in turn.  Within a
+// set, the decoder threads (TPR per row) split the CTA's operand slab (rows
+// 0-127: A, 128-255: B) of a 64-wide K step.  Each copies its part of a row's
+// 32 code bytes, and the row's 4 scale bytes, into its set's raw ring in
+// shared memory with cp.async, two of the set's steps ahead (L2 serves the
+// re-reads across tiles).  It decodes them as if4_decode_f16 does (the
+// byte-permute decode with the same roundings, so the fp16 operands, and with
+// the same MMA order the product, equal if4_linear's bit for bit), and writes
+// its part of the row into the stage in the 128-byte swizzled layout the MMA
 // descriptors read (16-byte chunk j of row r at position j ^ (r & 7)).  A
 // proxy fence makes those generic stores visible to the tensor cores; then
 // one lane per warp arrives on the CTA's own decoder barrier, and one
-// forwarder thread per CTA relays the
-// completed stage to the leader CTA's MMA barrier (release.cluster).
+// forwarder thread per CTA relays the completed stage to the leader CTA's MMA
+// barrier (release.cluster).
 
 namespace fused {
 
 constexpr int DEC_WARP0 = 6;                          // after TMA-less warp 0, MMA, epilogue
-#ifndef IF4_FUSED_DEC_WARPS
-#define IF4_FUSED_DEC_WARPS 8
-#endif
-constexpr int DEC_WARPS = IF4_FUSED_DEC_WARPS;        // 8: a slab row per thread; 16: half
+// Two sets of 8 decoder warps, each decoding whole slab rows of every other
+// K step.  Measured at 8192 x 4096 x 4096 (with the wait hint): one set of 8
+// warps 533 us; one set of 16 sharing rows, 522 us (without the hint); two
+// sets of 8, 418 us.  A K step's decode is latency-bound, so two steps in
+// flight help where more warps on the same step do not.
+constexpr int DEC_WARPS = 16;
 constexpr int FNUM_THREADS = (DEC_WARP0 + DEC_WARPS) * 32;
-constexpr int TPR = DEC_WARPS * 32 / (2 * pair::PBM);  // decoder threads per slab row
+// NPAR sets of decoder warps take the K steps in turn (set p: steps p,
+// p + NPAR, ...), so NPAR steps are decoded at once; within a set, TPR
+// threads share each slab row.
+constexpr int NPAR = 2;
+constexpr int TPR = DEC_WARPS * 32 / (2 * pair::PBM * NPAR);
+constexpr int SET_THREADS = 2 * pair::PBM * TPR;      // decoder threads per set
 constexpr int GPT = 4 / TPR;                          // groups per thread per K step
 static_assert(TPR == 1 || TPR == 2, "one or two decoder threads per slab row");
+static_assert(NPAR == 1 || NPAR == 2, "one or two sets of decoder warps");
+constexpr int FSTAGES = NPAR == 1 ? pair::PSTAGES : 5;  // operand stages (32 KB each)
 // Raw ring: per K step, the slab's code bytes as two 4 KB planes (16 bytes
 // of each row per plane, so a warp's 16-byte loads are conflict-free) and
 // the row's 4 scale bytes once per decoder thread.  Each decoder thread
 // fills and reads back its own part only, so cp.async's per-thread
-// wait_group is the only ordering needed.
+// wait_group is the only ordering needed.  One ring per set.
 constexpr int RAW_STAGES = 3;
 constexpr int RAW_SCALE_OFF = 2 * 4096;
 constexpr int RAW_STAGE_BYTES = RAW_SCALE_OFF + TPR * 1024;
-constexpr int RAW_OFFSET = pair::PSTAGES * pair::PSTAGE_BYTES + 1024;   // after barriers, table
-constexpr int FSMEM_BYTES = RAW_OFFSET + RAW_STAGES * RAW_STAGE_BYTES + 1024;
+constexpr int RAW_OFFSET = FSTAGES * pair::PSTAGE_BYTES + 1024;   // after barriers, table
+constexpr int FSMEM_BYTES = RAW_OFFSET + NPAR * RAW_STAGES * RAW_STAGE_BYTES + 1024;
 static_assert(FSMEM_BYTES <= 227 * 1024, "fused linear shared memory");
 
 // cp.async of 16 (or 4) bytes with zero fill of the bytes past src_bytes
@@ -846,17 +860,17 @@ gemm_if4_fused_2sm(const uint8_t *__restrict__ a_codes, const uint8_t *__restric
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *smem_a = smem;
-    uint8_t *smem_b = smem + PSTAGES * PA_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + PSTAGES * PSTAGE_BYTES);
-    uint64_t *full = bars;                    // [PSTAGES], used in the leader
-    uint64_t *empty = bars + PSTAGES;          // [PSTAGES], both CTAs
-    uint64_t *acc_full = bars + 2 * PSTAGES;   // [2], both CTAs
+    uint8_t *smem_b = smem + FSTAGES * PA_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + FSTAGES * PSTAGE_BYTES);
+    uint64_t *full = bars;                    // [FSTAGES], used in the leader
+    uint64_t *empty = bars + FSTAGES;          // [FSTAGES], both CTAs
+    uint64_t *acc_full = bars + 2 * FSTAGES;   // [2], both CTAs
     uint64_t *acc_empty = acc_full + 2;       // [2], used in the leader
     uint64_t *drain = acc_empty + 2;          // [1], leader
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    uint64_t *dec_full = drain + 2;           // [PSTAGES], both CTAs: this CTA's decoders
-    float *lut = reinterpret_cast<float *>(smem + PSTAGES * PSTAGE_BYTES + 256);
+    uint64_t *dec_full = drain + 2;           // [FSTAGES], both CTAs: this CTA's decoders
+    float *lut = reinterpret_cast<float *>(smem + FSTAGES * PSTAGE_BYTES + 256);
     uint8_t *raw = smem + RAW_OFFSET;
 
     const int warp = threadIdx.x >> 5;
@@ -871,9 +885,9 @@ gemm_if4_fused_2sm(const uint8_t *__restrict__ a_codes, const uint8_t *__restric
     const int k_blocks = K / BK;
 
     if (threadIdx.x == 0) {
-        for (int st = 0; st < PSTAGES; ++st) {
+        for (int st = 0; st < FSTAGES; ++st) {
             mbar_init(smem_u32(&full[st]), 2);           // one forwarder per CTA
-            mbar_init(smem_u32(&dec_full[st]), DEC_WARPS);
+            mbar_init(smem_u32(&dec_full[st]), DEC_WARPS / NPAR);
             mbar_init(smem_u32(&empty[st]), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -901,10 +915,12 @@ gemm_if4_fused_2sm(const uint8_t *__restrict__ a_codes, const uint8_t *__restric
 
     if (warp >= DEC_WARP0) {
         // ------------------------------------------------------- decoders
-        // thread td owns part h = td / 256 (GPT of the 4 groups) of slab row
-        // td % 256 (rows 0-127 A, 128-255 B) in every K step
+        // thread td: set p = td / SET_THREADS takes the K steps i = p, p +
+        // NPAR, ...; within the set, part h (GPT of the 4 groups) of slab row
+        // srow (rows 0-127 A, 128-255 B)
         const int td = threadIdx.x - DEC_WARP0 * 32;
-        const int srow = td & 255, h = td >> 8;
+        const int par = td / SET_THREADS, tp = td % SET_THREADS;
+        const int srow = tp & 255, h = tp >> 8;
         const bool is_a = srow < PBM;
         const int rloc = is_a ? srow : srow - PBM;              // row in this CTA's slab
         const uint8_t *codes = is_a ? a_codes : b_codes;
@@ -913,23 +929,25 @@ gemm_if4_fused_2sm(const uint8_t *__restrict__ a_codes, const uint8_t *__restric
         const uint32_t slab0 = smem_u32(is_a ? smem_a : smem_b) + (uint32_t)rloc * 128u;
         const uint32_t sw = (uint32_t)(rloc & 7);
         const uint32_t lut_addr = smem_u32(lut);
-        const uint32_t raw0 = smem_u32(raw);
+        const uint32_t raw0 = smem_u32(raw) + (uint32_t)(par * RAW_STAGES * RAW_STAGE_BYTES);
         // this thread's 16-byte code chunks c = h * (2 / TPR) + j (plane c, row
         // srow) and its scale word
         const uint32_t chunk0 = (uint32_t)h * (2u / TPR);
         const uint32_t code_off = chunk0 * 4096u + (uint32_t)srow * 16u;
-        const uint32_t scale_off = RAW_SCALE_OFF + (uint32_t)td * 4u;
+        const uint32_t scale_off = RAW_SCALE_OFF + (uint32_t)tp * 4u;
         const int64_t code_stride = K / 2, scale_stride = K / 16;
         const int my_tiles = pair_id < tiles ? (tiles - pair_id + num_pairs - 1) / num_pairs : 0;
         const int64_t steps = (int64_t)my_tiles * k_blocks;
-        // Fetch side of the raw ring: copies step fi's code bytes of this
-        // thread's part and the row's 4 scale bytes (zero-filled past the
-        // matrix) into slot fslot, one commit group per step (an empty group
-        // past the end).
-        int ft = pair_id, fkb = 0, fslot = 0;
+        const int64_t my_steps = steps > par ? (steps - par + NPAR - 1) / NPAR : 0;
+        // Fetch side of the raw ring: copies the code bytes of this thread's
+        // part of the set's fi-th step, and the row's 4 scale bytes
+        // (zero-filled past the matrix), into slot fslot, one commit group per
+        // step (an empty group past the end).  (ft, fkb): tile and K step.
+        int ft = pair_id, fkb = par, fslot = 0;
+        while (fkb >= k_blocks) { fkb -= k_blocks; ft += num_pairs; }
         int64_t fi = 0;
         auto fetch_next = [&]() {
-            if (fi < steps) {
+            if (fi < my_steps) {
                 const int row = (is_a ? (ft % m_tiles) * 2 * PBM + (int)rank * PBM
                                       : (ft / m_tiles) * PBN + (int)rank * PBNH) + rloc;
                 const bool in = row < rows_total;
@@ -942,7 +960,8 @@ gemm_if4_fused_2sm(const uint8_t *__restrict__ a_codes, const uint8_t *__restric
                     cp_async16(slot + code_off + (uint32_t)j * 4096u, src + 16 * j, in ? 16u : 0u);
                 cp_async4(slot + scale_off,
                           scales + (int64_t)rr * scale_stride + (int64_t)fkb * 4, in ? 4u : 0u);
-                if (++fkb == k_blocks) { fkb = 0; ft += num_pairs; }
+                fkb += NPAR;
+                while (fkb >= k_blocks) { fkb -= k_blocks; ft += num_pairs; }
                 ++fi;
                 if (++fslot == RAW_STAGES) fslot = 0;
             }
@@ -950,17 +969,19 @@ gemm_if4_fused_2sm(const uint8_t *__restrict__ a_codes, const uint8_t *__restric
         };
 #pragma unroll 1
         for (int s = 0; s < RAW_STAGES - 1; ++s) fetch_next();
-        int stage = 0, rslot = 0;
+        // operand stage and phase of step i = par + NPAR * j: stage i % FSTAGES,
+        // phase (i / FSTAGES) & 1
+        int stage = par, rslot = 0;
         uint32_t phase = 0;
 #pragma unroll 1
-        for (int64_t i = 0; i < steps; ++i) {
+        for (int64_t j = 0; j < my_steps; ++j) {
             fetch_next();
-            cp_async_wait<RAW_STAGES - 1>();             // this thread's step i bytes landed
+            cp_async_wait<RAW_STAGES - 1>();             // this thread's bytes of the step landed
             const uint32_t slot = raw0 + (uint32_t)rslot * RAW_STAGE_BYTES;
             if (++rslot == RAW_STAGES) rslot = 0;
             uint32_t w[2 * GPT];
 #pragma unroll
-            for (int j = 0; j < 2 / TPR; ++j) lds_v4(slot + code_off + (uint32_t)j * 4096u, w + 4 * j);
+            for (int c = 0; c < 2 / TPR; ++c) lds_v4(slot + code_off + (uint32_t)c * 4096u, w + 4 * c);
             const uint32_t sc = lds_u32(slot + scale_off);
             // the stage is free once the MMAs that read it have completed
             bool freed = true;
@@ -968,16 +989,16 @@ gemm_if4_fused_2sm(const uint8_t *__restrict__ a_codes, const uint8_t *__restric
             if (!__shfl_sync(0xFFFFFFFFu, freed ? 1 : 0, 0)) break;
             const uint32_t dst = slab0 + (uint32_t)stage * (uint32_t)PA_BYTES;
 #pragma unroll
-            for (uint32_t j = 0; j < (uint32_t)GPT; ++j) {
-                const uint32_t g = (uint32_t)h * GPT + j;      // group in the 64-wide step
+            for (uint32_t q = 0; q < (uint32_t)GPT; ++q) {
+                const uint32_t g = (uint32_t)h * GPT + q;      // group in the 64-wide step
                 uint32_t o[8];
                 const uint32_t sb = (sc >> (8 * g)) & 0xFFu;
                 const float e4 = f32_from_e4m3(sb);
                 const uint32_t im = 0u - (sb >> 7);
                 const BytePlanes P = group_planes<false>(lut_addr + ((sb >> 1) & 0x40u), e4);
-                const uint32_t bad = decode_word16(w[2 * j], im, P, o) |
-                                     decode_word16(w[2 * j + 1], im, P, o + 4);
-                if (bad != 0u) decode_group_f16(w[2 * j], w[2 * j + 1], sb, lut_addr, o);
+                const uint32_t bad = decode_word16(w[2 * q], im, P, o) |
+                                     decode_word16(w[2 * q + 1], im, P, o + 4);
+                if (bad != 0u) decode_group_f16(w[2 * q], w[2 * q + 1], sb, lut_addr, o);
                 sts_v4(dst + (((2u * g) ^ sw) << 4), o);
                 sts_v4(dst + (((2u * g + 1u) ^ sw) << 4), o + 4);
             }
@@ -985,7 +1006,8 @@ gemm_if4_fused_2sm(const uint8_t *__restrict__ a_codes, const uint8_t *__restric
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&dec_full[stage]));
-            if (++stage == PSTAGES) { stage = 0; phase ^= 1u; }
+            stage += NPAR;
+            if (stage >= FSTAGES) { stage -= FSTAGES; phase ^= 1u; }
         }
         cp_async_wait<0>();                              // no copy in flight at exit
     } else if (warp == 0 && lane == 0) {
@@ -1001,7 +1023,7 @@ gemm_if4_fused_2sm(const uint8_t *__restrict__ a_codes, const uint8_t *__restric
         for (int64_t i = 0; i < steps; ++i) {
             if (!mbar_wait(smem_u32(&dec_full[stage]), phase, abort_flag)) break;
             arrive_remote(full_leader0 + (uint32_t)stage * 8u);
-            if (++stage == PSTAGES) { stage = 0; phase ^= 1u; }
+            if (++stage == FSTAGES) { stage = 0; phase ^= 1u; }
         }
     } else if (warp == 1 && lane == 0 && leader) {
         // ------------------------------------------- MMA issuer (leader)
@@ -1025,7 +1047,7 @@ gemm_if4_fused_2sm(const uint8_t *__restrict__ a_codes, const uint8_t *__restric
                     umma_f16_pair(d_tmem, smem_desc_sw128(a0 + kk * UMMA_K * 2),
                                   smem_desc_sw128(b0 + kk * UMMA_K * 2), (kb | kk) != 0 ? 1u : 0u);
                 umma_commit_both(smem_u32(&empty[stage]));
-                if (++stage == PSTAGES) { stage = 0; phase ^= 1u; }
+                if (++stage == FSTAGES) { stage = 0; phase ^= 1u; }
             }
             if (!ok) break;
             umma_commit_both(smem_u32(&acc_full[acc]));

@@ -1,8 +1,8 @@
 """A CPU model of the byte-permute group decode, checked against the
 per-element table decode on every scale byte and every code in every position.
 
-The 16-bit decoders (if4_decode_f16, if4_dequantize to bf16 / fp16 and the
-fused-decode linear) decode a group without a table load per element.  They
+The fp16 operand decoders (if4_decode_f16, the fused-decode linear) and the
+round trip's bf16 output decode a group without a table load per element.  They
 round the group's eight magnitudes once, t[m] = out(fl32(base[m] * eff)) for
 m = 0..7 (base: the FP4 magnitudes, or the INT4 magnitudes fl32(k * fl(6/7))),
 and split them into a low-byte and a high-byte plane of 8 bytes each.  Each

@@ -271,10 +271,8 @@ def _arbitrary_codes(seed, rows=64, cols=4096):
                                 float("inf"), float("nan")])
 def test_dequantize_every_scale_byte_arbitrary_codes(ts):
     """Arbitrary code bytes (INT4 code 8 included, which the encoder never
-    emits) under every scale byte and degenerate tensor scales.  The 16-bit
-    outputs take the byte-permute decode, or the per-element table for INT4
-    code 8 and for a scale that is not finite with its sign bit clear; every
-    output equals the oracle's dequantization."""
+    emits) under every scale byte and degenerate tensor scales: every output
+    of the dequantizer (per-element table decode) equals the oracle's."""
     b = B()
     codes, scales = _arbitrary_codes(int(abs(ts) * 10) % 97 if np.isfinite(ts) else 5)
     ts32 = np.float32(ts)
@@ -287,8 +285,10 @@ def test_dequantize_every_scale_byte_arbitrary_codes(ts):
 
 
 def test_decode_f16_arbitrary_codes():
-    """As above for the linear's fp16 operand decode (scale bytes 0x7F and
-    0xFF are E4M3 NaN: their groups decode to NaN on both sides)."""
+    """As above for the linear's fp16 operand decode, which takes the
+    byte-permute decode, and the per-element table for groups holding INT4
+    code 8 (scale bytes 0x7F and 0xFF are E4M3 NaN: their groups decode to
+    NaN on both sides)."""
     b = B()
     codes, scales = _arbitrary_codes(9)
     d = b.decode_f16(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda()).cpu()
