@@ -16,14 +16,13 @@
 // and element i's code sits at bits [w*i, w*i + w) of the group's
 // little-endian code bytes (12 per group for IF6, 6 for IF3).
 //
-// Design: one thread per group of 16 (a grid-stride loop with the next
-// group's load in flight), the FP rounding done with exact power-of-two
-// scalings and one round-to-nearest-even, the INT integer with one fused
-// multiply-add (a single rounding of the exact product), the INT values from
-// a shared table of correctly rounded quotients, and the decision from the
-// two binary64 error sums in element order, the rule itself.  These formats
-// are not on the bench's step, so the kernels favour plainness over the IF4
-// fast path's binary32 decision.
+// Design: one thread per group of 16 in a grid-stride loop.  FP6 codes come
+// from the hardware E2M3 conversion (round to nearest even, saturating), FP3
+// codes from compares; the INT integer from one fused multiply-add (a single
+// rounding of the exact product).  The decision takes IF4's fast path: the
+// two error sums in binary32, and the binary64 rule itself (its INT values
+// the correctly rounded quotients, from a shared table) only for a group
+// whose binary32 margin is within the band.
 
 #include <cuda_runtime.h>
 
@@ -129,9 +128,11 @@ __device__ __forceinline__ void fill_int_table(float *tab)
     }
 }
 
-// 16 inputs of group g as floats.
+// 16 inputs of group g as floats; amax = max |x| and nonfinite (Inf or NaN
+// present, after which the outputs are unspecified).  16-bit inputs take the
+// maximum on the packed words, two elements per instruction.
 template <int DT>
-__device__ __forceinline__ void load16(const char *p, float (&x)[16])
+__device__ __forceinline__ void load16(const char *p, float (&x)[16], float &amax, bool &nonfinite)
 {
     if constexpr (DT == IF4_F32) {
 #pragma unroll
@@ -143,21 +144,48 @@ __device__ __forceinline__ void load16(const char *p, float (&x)[16])
             x[4 * q + 2] = __uint_as_float(c);
             x[4 * q + 3] = __uint_as_float(d);
         }
+        amax = 0.0f;
+        nonfinite = false;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float a = fabsf(x[i]);
+            nonfinite |= !(a <= 3.4028235e38f);
+            amax = a > amax ? a : amax;
+        }
     } else {
         uint32_t w[8];
         ld_nc_v4(p, w[0], w[1], w[2], w[3]);
         ld_nc_v4(p + 16, w[4], w[5], w[6], w[7]);
+        uint32_t m = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             if constexpr (DT == IF4_BF16) {
+                m = absmax_bf16x2(m, w[j]);
                 x[2 * j] = __uint_as_float(w[j] << 16);
                 x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
             } else {
+                m = absmax_f16x2(m, w[j]);
                 x[2 * j] = f16lo_to_f32(w[j]);
                 x[2 * j + 1] = f16hi_to_f32(w[j]);
             }
         }
+        const uint32_t m16 = max(m & 0x7FFFu, (m >> 16) & 0x7FFFu);
+        if constexpr (DT == IF4_BF16) {
+            nonfinite = m16 >= 0x7F80u;
+            amax = __uint_as_float(m16 << 16);
+        } else {
+            nonfinite = m16 >= 0x7C00u;
+            amax = f16lo_to_f32(m16);
+        }
     }
+}
+
+template <int DT>
+__device__ __forceinline__ void load16(const char *p, float (&x)[16])
+{
+    float amax;
+    bool nonfinite;
+    load16<DT>(p, x, amax, nonfinite);
 }
 
 template <int DT>
@@ -170,33 +198,28 @@ __device__ __forceinline__ const char *row_addr(const char *base, uint32_t g, ui
     return base + (int64_t)row * ld_bytes + (int64_t)(g - row * gpr) * gbytes;
 }
 
-// Store the 16 codes of a group, element i at bits [BITS*i, BITS*i + BITS).
+// Store the 16 codes of a group, element i at bits [BITS*i, BITS*i + BITS):
+// codes joined in pairs, then quads (each code below 2^BITS, so the sums do
+// not carry), then the quads cut into the stored words.
 template <int BITS>
 __device__ __forceinline__ void store_codes(uint8_t *p, const uint32_t (&c)[16])
 {
-    uint64_t lo = 0, hi = 0;
+    uint32_t q[4];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int pos = BITS * i;
-        if (pos + BITS <= 64) {
-            lo |= (uint64_t)c[i] << pos;
-        } else if (pos >= 64) {
-            hi |= (uint64_t)c[i] << (pos - 64);
-        } else {
-            lo |= (uint64_t)c[i] << pos;
-            hi |= (uint64_t)c[i] >> (64 - pos);
-        }
-    }
+    for (int k = 0; k < 4; ++k)
+        q[k] = c[4 * k] + (c[4 * k + 1] << BITS) + (c[4 * k + 2] << (2 * BITS)) +
+               (c[4 * k + 3] << (3 * BITS));
     if constexpr (BITS == 6) {          // 12 bytes at a 4-byte aligned address
-        uint32_t *q = reinterpret_cast<uint32_t *>(p);
-        q[0] = (uint32_t)lo;
-        q[1] = (uint32_t)(lo >> 32);
-        q[2] = (uint32_t)hi;
+        uint32_t *w = reinterpret_cast<uint32_t *>(p);
+        w[0] = q[0] | (q[1] << 24);
+        w[1] = (q[1] >> 8) | (q[2] << 16);
+        w[2] = (q[2] >> 16) | (q[3] << 8);
     } else {                            // 6 bytes at a 2-byte aligned address
-        uint16_t *q = reinterpret_cast<uint16_t *>(p);
-        q[0] = (uint16_t)lo;
-        q[1] = (uint16_t)(lo >> 16);
-        q[2] = (uint16_t)(lo >> 32);
+        uint16_t *w = reinterpret_cast<uint16_t *>(p);
+        const uint32_t lo = q[0] | (q[1] << 12) | (q[2] << 24);
+        w[0] = (uint16_t)lo;
+        w[1] = (uint16_t)(lo >> 16);
+        w[2] = (uint16_t)((q[2] >> 8) | (q[3] << 4));
     }
 }
 
@@ -224,9 +247,132 @@ __device__ __forceinline__ void load_codes(const uint8_t *p, uint32_t (&c)[16])
 
 __device__ __forceinline__ bool ts_ok(float ts) { return ts >= 0x1p-117f && ts <= 0x1p117f; }
 
-// Quantizer: one group per thread per round of a grid-stride loop.
+// Block scale sb_f = fl(fl(amax / fpmax) / ts).  The first quotient is an
+// IEEE division for IF6 and the exact amax * 1/4 for IF3 (amax >= 2^-124);
+// the second is Markstein's: with y = fl(1/ts), s = fl(a y), fl(s + fl(a - s
+// ts) y) is the correctly rounded a / ts when neither quotient over- nor
+// underflows.  Below a = 2^-100 the IEEE division is used; from s = 2^100 the
+// unrefined s is returned (any such value saturates to 448, as the exact one
+// does).
+template <int BITS>
+__device__ __forceinline__ float block_scale_w(float amax, float ts, float rts)
+{
+    float a;
+    if constexpr (BITS == 3)
+        a = amax >= 0x1p-124f ? __fmul_rn(amax, 0.25f) : __fdiv_rn(amax, 4.0f);
+    else
+        a = __fdiv_rn(amax, Width<BITS>::fpmax);
+    const float s = __fmul_rn(a, rts);
+    if (!(a >= 0x1p-100f && s < 0x1p100f)) return a >= 0x1p-100f ? s : __fdiv_rn(a, ts);
+    return __fmaf_rn(__fmaf_rn(-s, ts, a), rts, s);
+}
+
+// E2M3 codes of an element pair (code of v0 in bits 0-5, of v1 in bits 8-13,
+// sign in the code's bit 5) by the hardware conversion (round to nearest
+// even, saturating at 7.5), and the differences qf - v, each exact (qf is v
+// rounded to the grid, within a factor of two of it, or 0): one
+// mixed-precision subtract of the code's f16 value.
+__device__ __forceinline__ uint32_t e2m3_pair(float v0, float v1, float &d0, float &d1)
+{
+    uint32_t c;
+    asm("{\n\t.reg .b16 b, l, u;\n\t.reg .b32 h;\n\t"
+        "cvt.rn.satfinite.e2m3x2.f32 b, %4, %3;\n\t"
+        "cvt.rn.f16x2.e2m3x2 h, b;\n\t"
+        "mov.b32 {l, u}, h;\n\t"
+        "sub.rn.f32.f16 %1, l, %3;\n\t"
+        "sub.rn.f32.f16 %2, u, %4;\n\t"
+        "cvt.u32.u16 %0, b;\n\t}"
+        : "=r"(c), "=f"(d0), "=f"(d1) : "f"(v0), "f"(v1));
+    return c;
+}
+
+// The decision rule itself, for a group whose binary32 margin is within its
+// band: the two binary64 error sums in element order, from the group's
+// inputs reloaded at p.  Returns true when INT wins.
 template <int DT, int BITS>
-__global__ void __launch_bounds__(256)
+__device__ __noinline__ bool ifw_int_wins_exact(const char *p, float inv, float c_int,
+                                                const float *int_tab)
+{
+    float xv[16];
+    load16<DT>(p, xv);
+    double e_fp = 0.0, e_int = 0.0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float v = __fmul_rn(xv[i], inv);
+        const double df = __dsub_rn((double)v, (double)fp_value<BITS>(fp_code<BITS>(v)));
+        const double di =
+            __dsub_rn((double)v, (double)int_tab[int_code<BITS>(int_k<BITS>(v, c_int))]);
+        e_fp = __dadd_rn(e_fp, __dmul_rn(df, df));
+        e_int = __dadd_rn(e_int, __dmul_rn(di, di));
+    }
+    return e_int < e_fp;
+}
+
+// FP and INT candidates of one group and their binary32 error sums (two
+// lanes each).  CLAMP: |v| held below 2^19 and the INT integer clamped to
+// [-kmax, kmax], as a subnormal or the largest block scale needs.  Under any
+// other block scale |v| <= fpmax (1 + 2^-4) (1 + 4u): IF3's |v * 3/4| stays
+// below 3.5 and needs no clamp; IF6's v * 62/15 reaches 32.9, so its integer
+// is still clamped.  IF3 also takes max |df + di| (the tie test).
+template <int BITS, bool CLAMP>
+__device__ __forceinline__ void ifw_candidates(const float (&xv)[16], float inv, float c_int,
+                                               float nc_q, uint32_t (&cf)[16], uint32_t (&ci)[16],
+                                               float (&ef)[2], float (&ei)[2], float &tie)
+{
+    constexpr int KM = Width<BITS>::kmax;
+    constexpr uint32_t MASK = (1u << BITS) - 1u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float v[2], df[2];
+        v[0] = __fmul_rn(xv[2 * j], inv);
+        v[1] = __fmul_rn(xv[2 * j + 1], inv);
+        if constexpr (BITS == 6) {
+            const uint32_t c2 = e2m3_pair(v[0], v[1], df[0], df[1]);
+            cf[2 * j] = c2 & 0x3Fu;
+            cf[2 * j + 1] = (c2 >> 8) & 0x3Fu;
+        } else {
+#pragma unroll
+            for (int l = 0; l < 2; ++l) {
+                // E2M0 by selects (as fp_code<3>: ties to the even
+                // code, above 3 and NaN to 4), the code from the
+                // value's exponent, the sign of v kept
+                const float a = fabsf(v[l]);
+                const float q = !(a <= 3.0f) ? 4.0f
+                              : (a >= 1.5f ? 2.0f : (a > 0.5f ? 1.0f : 0.0f));
+                const uint32_t qb = __float_as_uint(q);
+                const uint32_t sgn = (__float_as_uint(v[l]) >> 29) & 4u;
+                cf[2 * j + l] = (qb != 0u ? (qb >> 23) - 126u : 0u) | sgn;
+                df[l] = __fsub_rn(__uint_as_float(qb | (sgn << 29)), v[l]);   // exact
+            }
+        }
+#pragma unroll
+        for (int l = 0; l < 2; ++l) {
+            // k = clamp(RNE(v * c), -KM, KM): |v| is held below 2^19 first,
+            // where one fused multiply-add rounds the exact product once
+            const float vc = CLAMP ? fminf(fmaxf(v[l], -0x1p19f), 0x1p19f) : v[l];
+            float r = __fmaf_rn(vc, c_int, kMagic);
+            if (CLAMP || BITS == 6)
+                r = fminf(fmaxf(r, kMagic - (float)KM), kMagic + (float)KM);
+            ci[2 * j + l] = __float_as_uint(r) & MASK;     // two's complement
+            const float di = __fmaf_rn(__fsub_rn(r, kMagic), nc_q, v[l]);
+            ef[l] = __fmaf_rn(df[l], df[l], ef[l]);
+            ei[l] = __fmaf_rn(di, di, ei[l]);
+            if constexpr (BITS == 3) tie = fmaxf(tie, fabsf(__fadd_rn(df[l], di)));
+        }
+    }
+}
+
+// Quantizer: one group per thread per round of a grid-stride loop.
+//
+// Decision, fast path (as IF4's): the two squared-error sums in binary32,
+// two lanes of 8 fused multiply-adds each, then one add.  The FP differences
+// are exact; an INT difference is one fused multiply-add v - k * fl(c) (c =
+// 15/62 or 4/3), off from the rule's v - fl(num k / den) by at most 2^-20
+// plus one rounding.  Outside the band 2^-16 (S + 1) (S = the sum of both
+// errors) the binary32 sign is the rule's; inside it the group is decided by
+// the binary64 rule itself (ifw_int_wins_exact).
+template <int DT, int BITS>
+__global__ void __launch_bounds__(256, 4)     // four blocks per SM: IF3 3 % faster than three
 ifw_quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, uint32_t ngroups,
                     int mode, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
                     const float *__restrict__ ts_ptr, int *err, int check_ts)
@@ -240,21 +386,18 @@ ifw_quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, 
     if (check_ts && blockIdx.x == 0 && threadIdx.x == 0 && !ts_ok(ts) && err)
         atomicOr(err, IF4_DEV_BAD_SCALE);
     const float c_int = BITS == 6 ? __fdiv_rn(62.0f, 15.0f) : 0.75f;
+    const float nc_q = BITS == 6 ? -__fdiv_rn(15.0f, 62.0f) : -__fdiv_rn(4.0f, 3.0f);
+    const float rts = __frcp_rn(ts);
     __syncthreads();
     bool nonfinite = false;
     const uint32_t stride = gridDim.x * blockDim.x;
     for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < ngroups; g += stride) {
-        float xv[16];
-        load16<DT>(row_addr(x, g, gpr, ld_bytes, GB), xv);
-        float amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float a = fabsf(xv[i]);
-            nonfinite |= !(a <= 3.4028235e38f);
-            amax = a > amax ? a : amax;
-        }
-        const uint32_t sb =
-            e4m3_from_f32(__fdiv_rn(__fdiv_rn(amax, Width<BITS>::fpmax), ts)) & 0x7Fu;
+        const char *p = row_addr(x, g, gpr, ld_bytes, GB);
+        float xv[16], amax;
+        bool nf;
+        load16<DT>(p, xv, amax, nf);
+        nonfinite |= nf;
+        const uint32_t sb = e4m3_from_f32(block_scale_w<BITS>(amax, ts, rts)) & 0x7Fu;
         uint32_t out[16];
         uint32_t scale = 0;
         if (sb == 0) {
@@ -264,18 +407,33 @@ ifw_quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, 
             const float eff = __fmul_rn(f32_from_e4m3(sb), ts);
             const float inv = __frcp_rn(eff);
             uint32_t cf[16], ci[16];
-            double e_fp = 0.0, e_int = 0.0;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float v = __fmul_rn(xv[i], inv);
-                cf[i] = fp_code<BITS>(v);
-                ci[i] = int_code<BITS>(int_k<BITS>(v, c_int));
-                const double df = __dsub_rn((double)v, (double)fp_value<BITS>(cf[i]));
-                const double di = __dsub_rn((double)v, (double)int_tab[ci[i]]);
-                e_fp = __dadd_rn(e_fp, __dmul_rn(df, df));
-                e_int = __dadd_rn(e_int, __dmul_rn(di, di));
+            float ef[2] = {0.0f, 0.0f}, ei[2] = {0.0f, 0.0f};
+            float tie = 0.0f;        // IF3: max |df + di| (see below)
+            // a subnormal or the largest block scale: v may leave the range
+            // the unclamped path relies on
+            if ((sb - 1u) < 7u || sb == 0x7Eu)
+                ifw_candidates<BITS, true>(xv, inv, c_int, nc_q, cf, ci, ef, ei, tie);
+            else
+                ifw_candidates<BITS, false>(xv, inv, c_int, nc_q, cf, ci, ef, ei, tie);
+            bool use_int = mode == W_INT;
+            if (mode == W_IF) {
+                const float e_fp = __fadd_rn(ef[0], ef[1]), e_int = __fadd_rn(ei[0], ei[1]);
+                const float d = __fsub_rn(e_fp, e_int);
+                const float S = __fadd_rn(e_fp, e_int);
+                const float band = __fmul_rn(__fadd_rn(S, 1.0f), 0x1p-16f);
+                use_int = d > band;
+                // S == 0: every error is zero or below 2^-75 where both
+                // candidates are 0; the sums tie and FP stays
+                // IF3: a group whose FP and INT values coincide element by
+                // element (0 or +-4 on both grids: about one group in 17 of
+                // the activations) ties exactly and keeps FP.  Then df + di
+                // = qf - k fl(4/3) plus one rounding, below 2^-19; where the
+                // values differ it is at least 1/3 - 2^-19.
+                if (!(fabsf(d) > band) && S != 0.0f)
+                    use_int = (BITS == 3 && tie <= 0x1p-18f)
+                                  ? false
+                                  : ifw_int_wins_exact<DT, BITS>(p, inv, c_int, int_tab);
             }
-            const bool use_int = mode == W_INT || (mode == W_IF && e_int < e_fp);
 #pragma unroll
             for (int i = 0; i < 16; ++i) out[i] = use_int ? ci[i] : cf[i];
             scale = sb | (use_int ? 0x80u : 0u);

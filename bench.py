@@ -71,7 +71,8 @@ def parse():
                             "linear_fused",
                             "nvint4_quantize", "nvfp4_4over6_quantize", "if4_quantize_rht",
                             "if4_decode_f16", "fused_quantize", "fused_quantize_rht",
-                            "fused_quantize_dequant"],
+                            "fused_quantize_dequant", "if6_quantize", "if3_quantize",
+                            "if6_dequantize", "if3_dequantize"],
                    help="launch only this kernel, warmup+steps times (for ncu captures)")
     return p.parse_args()
 
@@ -990,6 +991,8 @@ def run_kernel_only(args):
         return
     x_cpu = make_input(args.workload)
     step = Step(x_cpu, sets=1)
+    if args.kernel_only.startswith(("if6", "if3")):
+        step.init_widths()
     s = step.sets[0]
     b.if4_tensor_amax(s["x"], s["amax"], step.err)
     b.if4_tensor_scale(s["amax"], s["ts"])
