@@ -223,17 +223,33 @@ __device__ __forceinline__ void store_codes(uint8_t *p, const uint32_t (&c)[16])
     }
 }
 
+// The code bytes of a group as three words (IF6: 12 bytes as three 32-bit
+// loads; IF3: 6 bytes as three 16-bit loads), then the 16 codes from them.
 template <int BITS>
-__device__ __forceinline__ void load_codes(const uint8_t *p, uint32_t (&c)[16])
+__device__ __forceinline__ void load_code_words(const uint8_t *p, uint32_t (&w)[3])
+{
+    if constexpr (BITS == 6) {
+        const uint32_t *q = reinterpret_cast<const uint32_t *>(p);
+        w[0] = __ldg(q);
+        w[1] = __ldg(q + 1);
+        w[2] = __ldg(q + 2);
+    } else {
+        const uint16_t *q = reinterpret_cast<const uint16_t *>(p);
+        w[0] = __ldg(q);
+        w[1] = __ldg(q + 1);
+        w[2] = __ldg(q + 2);
+    }
+}
+
+template <int BITS>
+__device__ __forceinline__ void unpack_code_words(const uint32_t (&w)[3], uint32_t (&c)[16])
 {
     uint64_t lo, hi = 0;
     if constexpr (BITS == 6) {
-        const uint32_t *q = reinterpret_cast<const uint32_t *>(p);
-        lo = (uint64_t)__ldg(q) | ((uint64_t)__ldg(q + 1) << 32);
-        hi = __ldg(q + 2);
+        lo = (uint64_t)w[0] | ((uint64_t)w[1] << 32);
+        hi = w[2];
     } else {
-        const uint16_t *q = reinterpret_cast<const uint16_t *>(p);
-        lo = (uint64_t)__ldg(q) | ((uint64_t)__ldg(q + 1) << 16) | ((uint64_t)__ldg(q + 2) << 32);
+        lo = (uint64_t)w[0] | ((uint64_t)w[1] << 16) | ((uint64_t)w[2] << 32);
     }
     constexpr uint64_t M = (1u << BITS) - 1u;
 #pragma unroll
@@ -390,9 +406,11 @@ ifw_quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, 
     const float rts = __frcp_rn(ts);
     __syncthreads();
     bool nonfinite = false;
+    const bool contig = ld_bytes == (int64_t)gpr * GB;
     const uint32_t stride = gridDim.x * blockDim.x;
     for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < ngroups; g += stride) {
-        const char *p = row_addr(x, g, gpr, ld_bytes, GB);
+        // a contiguous tensor needs no division for the group's address
+        const char *p = contig ? x + (int64_t)g * GB : row_addr(x, g, gpr, ld_bytes, GB);
         float xv[16], amax;
         bool nf;
         load16<DT>(p, xv, amax, nf);
@@ -460,30 +478,51 @@ ifw_dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restri
     for (int c = threadIdx.x; c < (1 << BITS); c += blockDim.x) fp_tab[c] = fp_value<BITS>(c);
     const float ts = *ts_ptr;
     __syncthreads();
+    const bool contig = ld_bytes == (int64_t)gpr * (16 * OB);
+    // a dense, 32-byte aligned output: every group's outputs start on a
+    // 32-byte sector, so 256-bit stores write whole sectors (two 128-bit
+    // stores would each write half of every sector they touch)
+    const bool v8 = contig && (reinterpret_cast<uintptr_t>(y) & 31u) == 0u;
     const uint32_t stride = gridDim.x * blockDim.x;
     for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < ngroups; g += stride) {
-        uint32_t c[16];
-        load_codes<BITS>(codes + (int64_t)g * CB, c);
+        uint32_t w[3], c[16];
+        load_code_words<BITS>(codes + (int64_t)g * CB, w);
+        unpack_code_words<BITS>(w, c);
         const uint32_t sb = __ldg(scales + g);
         const float eff = __fmul_rn(f32_from_e4m3(sb & 0x7Fu), ts);
         const float *tab = (sb & 0x80u) ? int_tab : fp_tab;
         float yv[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) yv[i] = __fmul_rn(tab[c[i]], eff);
-        char *p = const_cast<char *>(row_addr(y, g, gpr, ld_bytes, 16 * OB));
+        char *p = contig ? y + (int64_t)g * (16 * OB)
+                         : const_cast<char *>(row_addr(y, g, gpr, ld_bytes, 16 * OB));
         if constexpr (ODT == IF4_F32) {
+            if (v8) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                st_v4(p + 16 * q, __float_as_uint(yv[4 * q]), __float_as_uint(yv[4 * q + 1]),
-                      __float_as_uint(yv[4 * q + 2]), __float_as_uint(yv[4 * q + 3]));
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t o[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) o[j] = __float_as_uint(yv[8 * h + j]);
+                    st_v8(p + 32 * h, o);
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    st_v4(p + 16 * q, __float_as_uint(yv[4 * q]), __float_as_uint(yv[4 * q + 1]),
+                          __float_as_uint(yv[4 * q + 2]), __float_as_uint(yv[4 * q + 3]));
+            }
         } else {
             uint32_t o[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 o[j] = ODT == IF4_BF16 ? bf16x2_from_f32(yv[2 * j], yv[2 * j + 1])
                                        : f16x2_from_f32(yv[2 * j], yv[2 * j + 1]);
-            st_v4(p, o[0], o[1], o[2], o[3]);
-            st_v4(p + 16, o[4], o[5], o[6], o[7]);
+            if (v8) {
+                st_v8(p, o);
+            } else {
+                st_v4(p, o[0], o[1], o[2], o[3]);
+                st_v4(p + 16, o[4], o[5], o[6], o[7]);
+            }
         }
     }
 }
