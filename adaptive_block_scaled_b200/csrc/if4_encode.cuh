@@ -349,6 +349,13 @@ struct If4Fast {
     bool int4, general, near;
 };
 
+// XQ: xv holds 4 times the group's values (the transform's H x, whose y is
+// H x / 4); v = xv * fl(inv / 4), equal to fl(y * inv) whenever y and inv / 4
+// are exact.  A block scale whose inverse is below 2^-122 (inv / 4 would be
+// subnormal) takes the general path.  An element whose y is subnormal has
+// |v| < 6.4 * 2^-24 against the group's amax above 2^-100: both candidates are
+// a zero of v's sign either way, and its squares are far below any margin.
+template <bool XQ = false>
 __device__ __forceinline__ If4Fast if4_fast(const f2_t (&xv)[8], float amax, float ts, float rts,
                                             const float *inv_tab)
 {
@@ -363,8 +370,10 @@ __device__ __forceinline__ If4Fast if4_fast(const f2_t (&xv)[8], float amax, flo
     o.general = !(amax >= 0x1p-100f && s < 0x1p100f) || (sb - 1u) < 7u || sb == 0x7Eu;
     const float inv = inv_tab[sb];
     o.inv = inv;
+    if constexpr (XQ) o.general = o.general || (sb != 0u && !(inv >= 0x1p-122f));
+    const float inv_v = XQ ? __fmul_rn(inv, 0.25f) : inv;
 
-    const f2_t INV = f2_pack(inv, inv);
+    const f2_t INV = f2_pack(inv_v, inv_v);
     f2_t v[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = f2_mul(xv[j], INV);

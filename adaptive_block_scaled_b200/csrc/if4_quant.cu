@@ -164,6 +164,9 @@ struct SignMasks {
 
 // The transform on the 8 element pairs of a group (pair j = elements 2j,
 // 2j+1): stage 1 inside each pair, stages 2, 4, 8 between pairs j and j + h/2.
+// QUARTER: also the final times 1/4; without it x holds H x, for callers
+// that fold the exact 1/4 into a later scaling.
+template <bool QUARTER = true>
 __device__ __forceinline__ void hadamard16(f2_t (&x)[8])
 {
 #pragma unroll
@@ -183,9 +186,11 @@ __device__ __forceinline__ void hadamard16(f2_t (&x)[8])
             }
         }
     }
-    const f2_t Q = f2_pack(0.25f, 0.25f);
+    if constexpr (QUARTER) {
+        const f2_t Q = f2_pack(0.25f, 0.25f);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) x[j] = f2_mul(x[j], Q);
+        for (int j = 0; j < 8; ++j) x[j] = f2_mul(x[j], Q);
+    }
 }
 
 // The same transform on 16 scalars (the rare exact paths).
@@ -210,8 +215,11 @@ __device__ __forceinline__ void hadamard16_scalar(float (&y)[16], uint32_t signs
 }
 
 // Unpack with the transform: sign masks on the raw bits, pairs as in
-// unpack_group, the transform, then max |y| over the transformed group.
-template <int DT>
+// unpack_group, the transform, then max |y| over the transformed group
+// (y = H x / 4).  QUARTER = false leaves x = H x (not y); the returned max is
+// |y|'s either way: max fl(|H x| / 4) = fl(max |H x| / 4), rounding being
+// monotone, subnormals included.
+template <int DT, bool QUARTER = true>
 __device__ __forceinline__ float unpack_group_rht(const Raw<DT> &r, const SignMasks &sm,
                                                   f2_t (&x)[8], bool &nonfinite)
 {
@@ -230,7 +238,7 @@ __device__ __forceinline__ float unpack_group_rht(const Raw<DT> &r, const SignMa
                 x[j] = f2_pack(f16lo_to_f32(w), f16hi_to_f32(w));
         }
     }
-    hadamard16(x);
+    hadamard16<false>(x);
     uint32_t m0 = 0, m1 = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -241,7 +249,12 @@ __device__ __forceinline__ float unpack_group_rht(const Raw<DT> &r, const SignMa
     }
     const uint32_t m = absmax_f32(m0, __uint_as_float(m1)) & 0x7FFFFFFFu;
     nonfinite = m >= 0x7F800000u;
-    return __uint_as_float(m);
+    if constexpr (QUARTER) {
+        const f2_t Q = f2_pack(0.25f, 0.25f);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] = f2_mul(x[k], Q);
+    }
+    return __fmul_rn(__uint_as_float(m), 0.25f);
 }
 
 // The 16 (transformed, when RHT) inputs of a group, re-read from memory.
@@ -464,7 +477,7 @@ __device__ __forceinline__ GroupCode encode_if4(const f2_t (&xv)[8], float amax,
                                               uint32_t signs)
 {
     constexpr int GB = 16 * elem_bytes<DT>();
-    const If4Fast f = if4_fast(xv, amax, ts, rts, inv_tab);
+    const If4Fast f = if4_fast<RHT>(xv, amax, ts, rts, inv_tab);
     return if4_finish(f, amax, ts, rts, inv_tab, [&](float (&y)[16]) {
         reload_group<DT, RHT>(group_addr<GB>(x, g, gpr, ld_bytes), signs, y);
     });
@@ -592,8 +605,10 @@ __device__ __forceinline__ bool quantize_one(const Raw<DT> &r, uint32_t g, const
     f2_t xv[8];
     bool nonfinite;
     float amax;
+    // IF4 with the transform keeps x = H x and folds the exact 1/4 into the
+    // inverse block scale (if4_fast<true>); the other modes take y = H x / 4
     if constexpr (RHT)
-        amax = unpack_group_rht<DT>(r, sm, xv, nonfinite);
+        amax = unpack_group_rht<DT, MODE != Q_IF4>(r, sm, xv, nonfinite);
     else
         amax = unpack_group<DT>(r, xv, nonfinite);
     GroupCode out;
@@ -763,7 +778,7 @@ amax_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, uint32_t
                 if constexpr (RHT) {
                     f2_t xv[8];
                     bool nf;
-                    m = max(m, __float_as_uint(unpack_group_rht<DT>(r[u], sm, xv, nf)));
+                    m = max(m, __float_as_uint(unpack_group_rht<DT, false>(r[u], sm, xv, nf)));
                 } else {
                     m = max(m, group_absmax_bits<DT>(r[u]));
                 }
@@ -920,7 +935,7 @@ quantize_fused_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr
                 if constexpr (RHT) {
                     f2_t xv[8];
                     bool nf;
-                    m = max(m, __float_as_uint(unpack_group_rht<DT>(r[u], sm, xv, nf)));
+                    m = max(m, __float_as_uint(unpack_group_rht<DT, false>(r[u], sm, xv, nf)));
                 } else {
                     m = max(m, group_absmax_bits<DT>(r[u]));
                 }

@@ -490,6 +490,23 @@ def test_rht_quantize_on_gradient_like_data(signs):
     check_rht(torch.from_numpy(t).to(torch.bfloat16), signs, f"student-t {signs:#06x}")
 
 
+def test_rht_quantize_extreme_magnitudes():
+    """The IF4 path with the transform scales v by fl(inv / 4) on H x: groups
+    from 2^-110 to 2^121 in magnitude (the largest group's inverse scale
+    below 2^-122, where the kernels leave that path; tiny groups whose H x
+    elements are subnormal beside a normal amax), and a given tensor scale
+    that puts most groups there; codes and scales equal the oracle's."""
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((64, 1024)).astype(np.float64)
+    x *= np.exp2(rng.integers(-110, 122, (64, 64))).repeat(16, axis=1)
+    x[0, :16] = np.ldexp(1.0, 123)          # no sign flips: H x = 2^127 (finite), y = 2^125
+    x[1, :16] = np.where(np.arange(16) == 3, np.ldexp(1.0, 20), np.ldexp(1.0, -130))
+    x = x.astype(np.float32)
+    check_rht(torch.from_numpy(x), 0x0000, "extreme magnitudes")
+    check_rht(torch.from_numpy(x), 0x0001, "extreme magnitudes, given ts",
+              ts=np.float32(np.ldexp(1.0, 116)))
+
+
 def test_rht_quantize_dtypes_shapes_and_given_scale():
     rng = np.random.default_rng(32)
     for shape in [(1, 16), (7, 80), (33, 272)]:
