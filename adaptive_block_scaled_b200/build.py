@@ -29,7 +29,7 @@ SOURCES = [
     ("if4_linear_noalloc.cu", []),
     ("ifw_quant.cu", ["-fmad=false"]),    # IF6 / IF3: the same arithmetic contract
 ]
-HEADERS = ["if4_device.cuh", "if4_encode.cuh", "if4_decode.cuh", "exports.map"]
+HEADERS = ["if4_device.cuh", "if4_encode.cuh", "if4_decode.cuh", "if4_internal.h", "exports.map"]
 
 
 def _nvcc():

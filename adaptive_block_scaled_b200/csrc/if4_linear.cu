@@ -36,6 +36,7 @@
 #include "../../include/if4.h"
 #include "if4_decode.cuh"
 #include "if4_encode.cuh"
+#include "if4_internal.h"
 
 namespace {
 
@@ -1351,9 +1352,7 @@ int if4_linear(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_t
     if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return IF4_ERR_ALIGN;
     uint8_t *wa = static_cast<uint8_t *>(workspace);
     uint8_t *wb = wa + align_up((size_t)M * (size_t)K * 2, 256);
-    rc = if4_decode_f16(a_codes, a_scales, M, K, wa, stream);
-    if (rc != IF4_OK) return rc;
-    rc = if4_decode_f16(b_codes, b_scales, N, K, wb, stream);
+    rc = internal_decode_f16_pair(a_codes, a_scales, M, wa, b_codes, b_scales, N, wb, K, stream);
     if (rc != IF4_OK) return rc;
     return launch_gemm(wa, wb, a_ts, b_ts, M, N, K, c, err_flag, static_cast<cudaStream_t>(stream));
 }
@@ -1392,9 +1391,7 @@ int if4_linear_quantized(const uint8_t *a_codes, const uint8_t *a_scales, const 
     if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return IF4_ERR_ALIGN;
     uint8_t *wa = static_cast<uint8_t *>(workspace);
     uint8_t *wb = wa + align_up((size_t)M * (size_t)K * 2, 256);
-    rc = if4_decode_f16(a_codes, a_scales, M, K, wa, stream);
-    if (rc != IF4_OK) return rc;
-    rc = if4_decode_f16(b_codes, b_scales, N, K, wb, stream);
+    rc = internal_decode_f16_pair(a_codes, a_scales, M, wa, b_codes, b_scales, N, wb, K, stream);
     if (rc != IF4_OK) return rc;
     const GemmOut o{c, c_codes, c_scales, c_ts};
     return launch_gemm_t<true>(wa, wb, a_ts, b_ts, M, N, K, o, err_flag,

@@ -803,6 +803,9 @@ def linear_report(pk, steps=20, warmup=3):
                                                c_codes, c_scales, c_ts, err_flag=err))
     t_sep = timed(lambda: (b.if4_linear(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], ws, c, err),
                            b.if4_quantize(c, c_codes, c_scales, c_ts, b.TS_GIVEN, err)))
+    # the public entry point as one call: both operands' decode in one
+    # launch, then the GEMM
+    t_call = timed(lambda: b.if4_linear(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], ws, c, err))
     # the decoders inside the GEMM (no workspace): the same C
     t_fused = timed(lambda: b.if4_linear_fused(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], c, err))
     flops = 2.0 * M * N * K
@@ -812,6 +815,7 @@ def linear_report(pk, steps=20, warmup=3):
             "decode_a_ms": t[0], "decode_b_ms": t[1], "gemm_ms": t[2], "linear_ms": total,
             "gemm_tflops": gemm_tf, "linear_tflops": flops / (total * 1e-3) / 1e12,
             "cublas_f16_ms": t_cublas, "cublas_f16_tflops": flops / (t_cublas * 1e-3) / 1e12,
+            "linear_call_ms": t_call, "linear_call_tflops": flops / (t_call * 1e-3) / 1e12,
             "linear_if4_out_ms": t_q, "linear_then_quantize_ms": t_sep,
             "linear_fused_decode_ms": t_fused,
             "linear_fused_decode_tflops": flops / (t_fused * 1e-3) / 1e12,
