@@ -329,47 +329,6 @@ __device__ __forceinline__ float block_scale4(float amax, float ts, float rts)
     return t;
 }
 
-// FP4 code word of four element pairs and their decoded values as floats.
-__device__ __forceinline__ uint32_t fp4_word_values(const f2_t (&v)[4], f2_t (&q)[4])
-{
-    uint32_t word;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 h0, h1, h2, h3;\n\t"
-        ".reg .b16 l0, l1, l2, l3, u0, u1, u2, u3;\n\t"
-        ".reg .f32 x<8>, e<8>;\n\t"
-        "mov.b64 {x0, x1}, %5;\n\t"
-        "mov.b64 {x2, x3}, %6;\n\t"
-        "mov.b64 {x4, x5}, %7;\n\t"
-        "mov.b64 {x6, x7}, %8;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, x1, x0;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, x3, x2;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, x5, x4;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, x7, x6;\n\t"
-        "mov.b32 %0, {b0, b1, b2, b3};\n\t"
-        "cvt.rn.f16x2.e2m1x2 h0, b0;\n\t"
-        "cvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 h2, b2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
-        "mov.b32 {l0, u0}, h0;\n\t"
-        "mov.b32 {l1, u1}, h1;\n\t"
-        "mov.b32 {l2, u2}, h2;\n\t"
-        "mov.b32 {l3, u3}, h3;\n\t"
-        "cvt.f32.f16 e0, l0;\n\t"
-        "cvt.f32.f16 e1, u0;\n\t"
-        "cvt.f32.f16 e2, l1;\n\t"
-        "cvt.f32.f16 e3, u1;\n\t"
-        "cvt.f32.f16 e4, l2;\n\t"
-        "cvt.f32.f16 e5, u2;\n\t"
-        "cvt.f32.f16 e6, l3;\n\t"
-        "cvt.f32.f16 e7, u3;\n\t"
-        "mov.b64 %1, {e0, e1};\n\t"
-        "mov.b64 %2, {e2, e3};\n\t"
-        "mov.b64 %3, {e4, e5};\n\t"
-        "mov.b64 %4, {e6, e7};\n\t}"
-        : "=r"(word), "=l"(q[0]), "=l"(q[1]), "=l"(q[2]), "=l"(q[3])
-        : "l"(v[0]), "l"(v[1]), "l"(v[2]), "l"(v[3]));
-    return word;
-}
-
 // Binary64 reconstruction errors of the two 4/6 candidates in element order
 // (the rule itself), for groups whose binary32 margin is within rounding.
 // The 16 inputs are all loaded before the sums start (one round trip).
@@ -403,11 +362,15 @@ __device__ __noinline__ bool four_wins_exact(const char *p, float inv6, float ef
 
 // 4/6 encode of one group: FP4 under the block scale of amax/6 and under that
 // of amax/4, reconstruction errors sum (x - fl(q * eff))^2 compared, equal
-// errors keep /6.  Fast path: each difference is one explicit fma(q, -eff,
-// x), which differs from the rule's x - fl(q * eff) by at most 2^-24 * 6 eff,
-// and each sum by at most 9 roundings; the binary32 difference of the sums is
-// then within 2^-20 S + 2^-21 X^2 of the rule (X = 6 max(eff6, eff4)), so
-// outside the band 2^-18 S + 2^-19 X^2 + 2^-126 its sign is the rule's.
+// errors keep /6.  Fast path: each candidate's squared differences q - v in
+// the scaled domain (exact mixed-precision subtracts), summed in two lanes
+// and scaled by fl(eff^2).  eff (v - q) differs from the rule's x - fl(q *
+// eff) by at most about 3.1 u X per element (v = fl(x fl(1/eff))), and with
+// the sums' roundings the binary32 difference stays within 2^-19.3 S +
+// 2^-20.4 X^2 of the rule (X = 6 max(eff6, eff4)), so outside the band 2^-18
+// S + 2^-19 X^2 + 2^-126 its sign is the rule's.  Above X = 2^60 (where
+// eff^2 may overflow), and when exactly one block scale is zero, the rule
+// decides.
 template <int DT>
 __device__ __forceinline__ GroupCode encode_group_46(const f2_t (&x)[8], float amax, float ts,
                                                    float rts, const float *inv_tab,
@@ -421,29 +384,29 @@ __device__ __forceinline__ GroupCode encode_group_46(const f2_t (&x)[8], float a
     uint32_t w6[2], w4[2];
     f2_t e6 = f2_pack(0.0f, 0.0f), e4 = f2_pack(0.0f, 0.0f);
     const f2_t INV6 = f2_pack(inv6, inv6), INV4 = f2_pack(inv4, inv4);
-    const f2_t NEFF6 = f2_pack(-eff6, -eff6), NEFF4 = f2_pack(-eff4, -eff4);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        f2_t v6[4], v4[4], q6[4], q4[4];
+        f2_t v6[4], v4[4], d6[4], d4[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             v6[j] = f2_mul(x[4 * h + j], INV6);
             v4[j] = f2_mul(x[4 * h + j], INV4);
         }
-        w6[h] = fp4_word_values(v6, q6);
-        w4[h] = fp4_word_values(v4, q4);
+        w6[h] = fp4_word<true>(v6, d6);          // d = qf - v, exact
+        w4[h] = fp4_word<true>(v4, d4);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const f2_t d6 = f2_fma(q6[j], NEFF6, x[4 * h + j]);
-            const f2_t d4 = f2_fma(q4[j], NEFF4, x[4 * h + j]);
-            e6 = f2_fma(d6, d6, e6);
-            e4 = f2_fma(d4, d4, e4);
+            e6 = f2_fma(d6[j], d6[j], e6);
+            e4 = f2_fma(d4[j], d4[j], e4);
         }
     }
     float a0, a1, b0, b1;
     f2_unpack(e6, a0, a1);
     f2_unpack(e4, b0, b1);
-    const float s6 = __fadd_rn(a0, a1), s4 = __fadd_rn(b0, b1);
+    // the scaled-domain sums times fl(eff^2): the x-domain sums, to within
+    // the band below
+    const float s6 = __fmul_rn(__fadd_rn(a0, a1), __fmul_rn(eff6, eff6));
+    const float s4 = __fmul_rn(__fadd_rn(b0, b1), __fmul_rn(eff4, eff4));
     const float d = __fsub_rn(s6, s4);
     const float X = __fmul_rn(6.0f, fmaxf(eff6, eff4));
     const float band = __fmaf_rn(__fadd_rn(s6, s4), 0x1p-18f,
@@ -451,7 +414,11 @@ __device__ __forceinline__ GroupCode encode_group_46(const f2_t (&x)[8], float a
     bool four = d > 0.0f;
     if (sb4 == sb6)
         four = false;                 // identical candidates: a tie, keep /6
-    else if (!(fabsf(d) > band))
+    // the rule decides within the band; above X = 2^60, where eff^2 may
+    // overflow; and when one block scale is zero (its v is 0, so the
+    // scaled-domain sum is 0, while every output of that candidate is 0 and
+    // its x-domain error the sum of x^2)
+    else if (!(fabsf(d) > band) || X > 0x1p60f || sb6 == 0u || sb4 == 0u)
         four = four_wins_exact<DT>(group_addr<16 * elem_bytes<DT>()>(xbase, g, gpr, ld_bytes), inv6,
                                    eff6, inv4, eff4);
     GroupCode out;
