@@ -198,29 +198,19 @@ __device__ __forceinline__ const char *row_addr(const char *base, uint32_t g, ui
     return base + (int64_t)row * ld_bytes + (int64_t)(g - row * gpr) * gbytes;
 }
 
-// Store the 16 codes of a group, element i at bits [BITS*i, BITS*i + BITS):
-// codes joined in pairs, then quads (each code below 2^BITS, so the sums do
-// not carry), then the quads cut into the stored words.
-template <int BITS>
-__device__ __forceinline__ void store_codes(uint8_t *p, const uint32_t (&c)[16])
+// Store the 16 codes of an IF6 group, element i at bits [6i, 6i + 6): codes
+// joined in quads (each code below 2^6, so the sums do not carry), the quads
+// cut into three 32-bit words at a 4-byte aligned address.
+__device__ __forceinline__ void store_codes6(uint8_t *p, const uint32_t (&c)[16])
 {
     uint32_t q[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k)
-        q[k] = c[4 * k] + (c[4 * k + 1] << BITS) + (c[4 * k + 2] << (2 * BITS)) +
-               (c[4 * k + 3] << (3 * BITS));
-    if constexpr (BITS == 6) {          // 12 bytes at a 4-byte aligned address
-        uint32_t *w = reinterpret_cast<uint32_t *>(p);
-        w[0] = q[0] | (q[1] << 24);
-        w[1] = (q[1] >> 8) | (q[2] << 16);
-        w[2] = (q[2] >> 16) | (q[3] << 8);
-    } else {                            // 6 bytes at a 2-byte aligned address
-        uint16_t *w = reinterpret_cast<uint16_t *>(p);
-        const uint32_t lo = q[0] | (q[1] << 12) | (q[2] << 24);
-        w[0] = (uint16_t)lo;
-        w[1] = (uint16_t)(lo >> 16);
-        w[2] = (uint16_t)((q[2] >> 8) | (q[3] << 4));
-    }
+        q[k] = c[4 * k] + (c[4 * k + 1] << 6) + (c[4 * k + 2] << 12) + (c[4 * k + 3] << 18);
+    uint32_t *w = reinterpret_cast<uint32_t *>(p);
+    w[0] = q[0] | (q[1] << 24);
+    w[1] = (q[1] >> 8) | (q[2] << 16);
+    w[2] = (q[2] >> 16) | (q[3] << 8);
 }
 
 // The code bytes of a group as three words (IF6: 12 bytes as three 32-bit
@@ -324,100 +314,164 @@ __device__ __noinline__ bool ifw_int_wins_exact(const char *p, float inv, float 
     return e_int < e_fp;
 }
 
-// FP and INT candidates of one group and their binary32 error sums (two
-// lanes each).  CLAMP: |v| held below 2^19 and the INT integer clamped to
-// [-kmax, kmax], as a subnormal or the largest block scale needs.  Under any
-// other block scale |v| <= fpmax (1 + 2^-4) (1 + 4u): IF3's |v * 3/4| stays
-// below 3.5 and needs no clamp; IF6's v * 62/15 reaches 32.9, so its integer
-// is still clamped.  IF3 also takes max |df + di| (the tie test).
-template <int BITS, bool CLAMP>
-__device__ __forceinline__ void ifw_candidates(const float (&xv)[16], float inv, float c_int,
+// IF6: FP and INT candidates of one group and their binary32 error sums (two
+// lanes: lane 0 sums the even elements, lane 1 the odd ones).  CLAMP: |v|
+// held below 2^19, as a subnormal or the largest block scale needs; the
+// integer is clamped to [-31, 31] on every path (under the other block
+// scales |v| <= 7.5 (1 + 2^-4) (1 + 4u), and v * 62/15 reaches 32.9).  Element
+// pairs (2j, 2j + 1) go through paired binary32 instructions, each lane
+// rounded as its scalar form (57.4 against 62.7 us for the scalar loop on the
+// 8192 x 8192 activation).
+template <bool CLAMP>
+__device__ __forceinline__ void if6_candidates(const float (&xv)[16], float inv, float c_int,
                                                float nc_q, uint32_t (&cf)[16], uint32_t (&ci)[16],
-                                               float (&ef)[2], float (&ei)[2], float &tie)
+                                               float (&ef)[2], float (&ei)[2])
 {
-    constexpr int KM = Width<BITS>::kmax;
-    constexpr uint32_t MASK = (1u << BITS) - 1u;
-    // element pairs (2j, 2j + 1); IF6 takes them in paired binary32
-    // instructions, each lane rounded as its scalar counterpart (IF6: 57.4
-    // against 62.7 us scalar on the 8192 x 8192 activation; IF3 measured
-    // 0.8% slower paired and stays scalar); either way lane 0 sums the even
-    // elements, lane 1 the odd ones
+    constexpr int KM = Width<6>::kmax;
     const f2_t INV = f2_pack(inv, inv), C = f2_pack(c_int, c_int);
     const f2_t M = f2_pack(kMagic, kMagic), NM = f2_pack(-kMagic, -kMagic);
     const f2_t NCQ = f2_pack(nc_q, nc_q);
     f2_t EF = f2_pack(ef[0], ef[1]), EI = f2_pack(ei[0], ei[1]);
-    float e3f[2] = {ef[0], ef[1]}, e3i[2] = {ei[0], ei[1]};
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
+        const f2_t V = f2_mul(f2_pack(xv[2 * j], xv[2 * j + 1]), INV);
         float v[2], df[2];
-        f2_t V = 0;
-        if constexpr (BITS == 6) {
-            V = f2_mul(f2_pack(xv[2 * j], xv[2 * j + 1]), INV);
-            f2_unpack(V, v[0], v[1]);
-        } else {
-            v[0] = __fmul_rn(xv[2 * j], inv);
-            v[1] = __fmul_rn(xv[2 * j + 1], inv);
-        }
-        if constexpr (BITS == 6) {
-            const uint32_t c2 = e2m3_pair(v[0], v[1], df[0], df[1]);
-            cf[2 * j] = c2 & 0x3Fu;
-            cf[2 * j + 1] = (c2 >> 8) & 0x3Fu;
-        } else {
+        f2_unpack(V, v[0], v[1]);
+        const uint32_t c2 = e2m3_pair(v[0], v[1], df[0], df[1]);
+        cf[2 * j] = c2 & 0x3Fu;
+        cf[2 * j + 1] = (c2 >> 8) & 0x3Fu;
+        // k = clamp(RNE(v * c), -31, 31): one fused multiply-add rounds the
+        // exact product once while |v| < 2^19
+        f2_t VC = V;
+        if constexpr (CLAMP)
+            VC = f2_pack(fminf(fmaxf(v[0], -0x1p19f), 0x1p19f),
+                         fminf(fmaxf(v[1], -0x1p19f), 0x1p19f));
+        f2_t R = f2_fma(VC, C, M);
+        float r[2];
+        f2_unpack(R, r[0], r[1]);
 #pragma unroll
-            for (int l = 0; l < 2; ++l) {
-                // E2M0 by selects (as fp_code<3>: ties to the even
-                // code, above 3 and NaN to 4), the code from the
-                // value's exponent, the sign of v kept
-                const float a = fabsf(v[l]);
-                const float q = !(a <= 3.0f) ? 4.0f
-                              : (a >= 1.5f ? 2.0f : (a > 0.5f ? 1.0f : 0.0f));
-                const uint32_t qb = __float_as_uint(q);
-                const uint32_t sgn = (__float_as_uint(v[l]) >> 29) & 4u;
-                cf[2 * j + l] = (qb != 0u ? (qb >> 23) - 126u : 0u) | sgn;
-                df[l] = __fsub_rn(__uint_as_float(qb | (sgn << 29)), v[l]);   // exact
-            }
-        }
-        // k = clamp(RNE(v * c), -KM, KM): |v| is held below 2^19 first,
-        // where one fused multiply-add rounds the exact product once
-        if constexpr (BITS == 6) {
-            f2_t VC = V;
-            if constexpr (CLAMP)
-                VC = f2_pack(fminf(fmaxf(v[0], -0x1p19f), 0x1p19f),
-                             fminf(fmaxf(v[1], -0x1p19f), 0x1p19f));
-            f2_t R = f2_fma(VC, C, M);
-            float r[2];
-            f2_unpack(R, r[0], r[1]);
-#pragma unroll
-            for (int l = 0; l < 2; ++l)
-                r[l] = fminf(fmaxf(r[l], kMagic - (float)KM), kMagic + (float)KM);
-            R = f2_pack(r[0], r[1]);
-            ci[2 * j] = __float_as_uint(r[0]) & MASK;      // two's complement
-            ci[2 * j + 1] = __float_as_uint(r[1]) & MASK;
-            const f2_t DI = f2_fma(f2_add(R, NM), NCQ, V);  // v - k fl(c), one rounding
-            const f2_t DF = f2_pack(df[0], df[1]);
-            EF = f2_fma(DF, DF, EF);
-            EI = f2_fma(DI, DI, EI);
-        } else {
-#pragma unroll
-            for (int l = 0; l < 2; ++l) {
-                const float vc = CLAMP ? fminf(fmaxf(v[l], -0x1p19f), 0x1p19f) : v[l];
-                float r = __fmaf_rn(vc, c_int, kMagic);
-                if (CLAMP) r = fminf(fmaxf(r, kMagic - (float)KM), kMagic + (float)KM);
-                ci[2 * j + l] = __float_as_uint(r) & MASK;
-                const float di = __fmaf_rn(__fsub_rn(r, kMagic), nc_q, v[l]);
-                e3f[l] = __fmaf_rn(df[l], df[l], e3f[l]);
-                e3i[l] = __fmaf_rn(di, di, e3i[l]);
-                tie = fmaxf(tie, fabsf(__fadd_rn(df[l], di)));
-            }
-        }
+        for (int l = 0; l < 2; ++l)
+            r[l] = fminf(fmaxf(r[l], kMagic - (float)KM), kMagic + (float)KM);
+        R = f2_pack(r[0], r[1]);
+        ci[2 * j] = __float_as_uint(r[0]) & 0x3Fu;         // two's complement
+        ci[2 * j + 1] = __float_as_uint(r[1]) & 0x3Fu;
+        const f2_t DI = f2_fma(f2_add(R, NM), NCQ, V);      // v - k fl(c), one rounding
+        const f2_t DF = f2_pack(df[0], df[1]);
+        EF = f2_fma(DF, DF, EF);
+        EI = f2_fma(DI, DI, EI);
     }
-    if constexpr (BITS == 6) {
-        f2_unpack(EF, ef[0], ef[1]);
-        f2_unpack(EI, ei[0], ei[1]);
-    } else {
-        ef[0] = e3f[0]; ef[1] = e3f[1];
-        ei[0] = e3i[0]; ei[1] = e3i[1];
+    f2_unpack(EF, ef[0], ef[1]);
+    f2_unpack(EI, ei[0], ei[1]);
+}
+
+// 1.0f where the comparison holds, else 0.0f; the unordered forms (gtu, geu)
+// hold for a NaN operand.
+__device__ __forceinline__ float set_gtu(float a, float b)
+{
+    float d;
+    asm("set.gtu.f32.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+
+__device__ __forceinline__ float set_geu(float a, float b)
+{
+    float d;
+    asm("set.geu.f32.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+
+// 1.0f when the sign bit of v is set (a negative zero too), else 0.0f.
+__device__ __forceinline__ float sign_bit_f(float v)
+{
+    float d;
+    asm("set.lt.f32.s32 %0, %1, 0;" : "=f"(d) : "r"(__float_as_uint(v)));
+    return d;
+}
+
+// IF3: both candidates of one group as four 12-bit quads of codes (element
+// 4k + i at bits [3i, 3i + 3) of quad k), and the binary32 error sums in two
+// lanes (even and odd elements, each in element order).
+//
+// E2M0 from three comparisons of a = |v| that give 1.0 or 0.0: s1 = [a > 1/2],
+// s2 = [a >= 3/2], s3 = [a > 3].  The value is s1 + s2 + 2 s3 (0, 1, 2, 4),
+// the magnitude code s1 + s2 + s3 (0 to 3): ties go to the even code (1/2 ->
+// 0, 3/2 -> 2, 3 -> 2) and a NaN, every comparison holding, to 4.  The FP
+// quad is accumulated as the exact float 2^23 + sum (code_i 8^i) and read from
+// its low 12 bits; code_i = magnitude + 4 [sign bit of v].  |qf - v| = fl(q -
+// a) (exact under the unclamped scales; otherwise the same rounding of the
+// same difference) enters the sum squared.  The INT integer k = RNE(3v/4) from
+// one fused multiply-add as in IF6 (CLAMP: |v| held below 2^19 and k clamped
+// to [-3, 3]; under any other block scale |3v/4| < 3.5 needs neither).
+template <bool CLAMP>
+__device__ __forceinline__ void if3_candidates(const float (&xv)[16], float inv, float nc_q,
+                                               uint32_t (&fq)[4], uint32_t (&iq)[4],
+                                               float (&ef)[2], float (&ei)[2])
+{
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        float acc = 0x1p23f;
+        uint32_t iw = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e = 4 * k + i;
+            const float w = (float)(1 << (3 * i));          // 8^i
+            const float v = __fmul_rn(xv[e], inv);
+            const float a = fabsf(v);
+            const float s1 = set_gtu(a, 0.5f), s2 = set_geu(a, 1.5f), s3 = set_gtu(a, 3.0f);
+            const float A = __fadd_rn(s1, s2);
+            const float df = __fsub_rn(__fmaf_rn(s3, 2.0f, A), a);
+            acc = __fmaf_rn(A, w, acc);
+            acc = __fmaf_rn(__fmaf_rn(sign_bit_f(v), 4.0f, s3), w, acc);
+            const float vc = CLAMP ? fminf(fmaxf(v, -0x1p19f), 0x1p19f) : v;
+            float r = __fmaf_rn(vc, 0.75f, kMagic);
+            if (CLAMP) r = fminf(fmaxf(r, kMagic - 3.0f), kMagic + 3.0f);
+            iw |= (__float_as_uint(r) & 7u) << (3 * i);      // two's complement
+            const float di = __fmaf_rn(__fsub_rn(r, kMagic), nc_q, v);
+            ef[i & 1] = __fmaf_rn(df, df, ef[i & 1]);
+            ei[i & 1] = __fmaf_rn(di, di, ei[i & 1]);
+        }
+        fq[k] = __float_as_uint(acc) & 0xFFFu;
+        iq[k] = iw;
     }
+}
+
+// IF3: true when the FP and INT values of every element coincide (both 0, or
+// both +4 or both -4), found on the codes: a slot coincides exactly when its
+// FP magnitude code is 0 or 3 (bits 0 and 1 equal) and bit 0 of the FP and
+// INT codes agree.  Where the FP value is 0 (|v| <= 1/2) k is 0; where it is
+// 4 (|v| > 3) |k| is 2 or 3 with the sign of v; so the codes pair as (000 or
+// 100, 000), (011, 011 or 010), (111, 101 or 110), and the test keeps the
+// first of each pair.
+__device__ __forceinline__ bool if3_values_coincide(const uint32_t (&fq)[4], const uint32_t (&iq)[4])
+{
+    uint32_t t = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) t |= (fq[k] ^ (fq[k] >> 1)) | (fq[k] ^ iq[k]);
+    return (t & 0x249u) == 0u;                 // bit 0 of each of the 4 slots
+}
+
+// The 6 code bytes of an IF3 group from its four quads.
+__device__ __forceinline__ void store_quads3(uint8_t *p, const uint32_t (&q)[4])
+{
+    uint16_t *w = reinterpret_cast<uint16_t *>(p);
+    const uint32_t lo = q[0] | (q[1] << 12) | (q[2] << 24);
+    w[0] = (uint16_t)lo;
+    w[1] = (uint16_t)(lo >> 16);
+    w[2] = (uint16_t)((q[2] >> 8) | (q[3] << 4));
+}
+
+// The fast decision from the two binary32 sums: INT when e_fp - e_int
+// exceeds the band 2^-16 (S + 1); near when the margin is within it and S !=
+// 0 (S == 0: every error is zero or below 2^-75 where both candidates are 0,
+// the sums tie and FP stays).
+__device__ __forceinline__ bool fast_int(const float (&ef)[2], const float (&ei)[2], bool &near)
+{
+    const float e_fp = __fadd_rn(ef[0], ef[1]), e_int = __fadd_rn(ei[0], ei[1]);
+    const float d = __fsub_rn(e_fp, e_int);
+    const float S = __fadd_rn(e_fp, e_int);
+    const float band = __fmul_rn(__fadd_rn(S, 1.0f), 0x1p-16f);
+    near = !(fabsf(d) > band) && S != 0.0f;
+    return d > band;
 }
 
 // Quantizer: one group per thread per round of a grid-stride loop.
@@ -458,47 +512,61 @@ ifw_quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, 
         load16<DT>(p, xv, amax, nf);
         nonfinite |= nf;
         const uint32_t sb = e4m3_from_f32(block_scale_w<BITS>(amax, ts, rts)) & 0x7Fu;
-        uint32_t out[16];
         uint32_t scale = 0;
-        if (sb == 0) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) out[i] = 0;
-        } else {
-            const float eff = __fmul_rn(f32_from_e4m3(sb), ts);
-            const float inv = __frcp_rn(eff);
-            uint32_t cf[16], ci[16];
-            float ef[2] = {0.0f, 0.0f}, ei[2] = {0.0f, 0.0f};
-            float tie = 0.0f;        // IF3: max |df + di| (see below)
-            // a subnormal or the largest block scale: v may leave the range
-            // the unclamped path relies on
-            if ((sb - 1u) < 7u || sb == 0x7Eu)
-                ifw_candidates<BITS, true>(xv, inv, c_int, nc_q, cf, ci, ef, ei, tie);
-            else
-                ifw_candidates<BITS, false>(xv, inv, c_int, nc_q, cf, ci, ef, ei, tie);
-            bool use_int = mode == W_INT;
-            if (mode == W_IF) {
-                const float e_fp = __fadd_rn(ef[0], ef[1]), e_int = __fadd_rn(ei[0], ei[1]);
-                const float d = __fsub_rn(e_fp, e_int);
-                const float S = __fadd_rn(e_fp, e_int);
-                const float band = __fmul_rn(__fadd_rn(S, 1.0f), 0x1p-16f);
-                use_int = d > band;
-                // S == 0: every error is zero or below 2^-75 where both
-                // candidates are 0; the sums tie and FP stays
-                // IF3: a group whose FP and INT values coincide element by
-                // element (0 or +-4 on both grids: about one group in 17 of
-                // the activations) ties exactly and keeps FP.  Then df + di
-                // = qf - k fl(4/3) plus one rounding, below 2^-19; where the
-                // values differ it is at least 1/3 - 2^-19.
-                if (!(fabsf(d) > band) && S != 0.0f)
-                    use_int = (BITS == 3 && tie <= 0x1p-18f)
-                                  ? false
-                                  : ifw_int_wins_exact<DT, BITS>(p, inv, c_int, int_tab);
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) out[i] = use_int ? ci[i] : cf[i];
-            scale = sb | (use_int ? 0x80u : 0u);
+        // a subnormal or the largest block scale: v may leave the range the
+        // unclamped path relies on
+        const bool clamp = (sb - 1u) < 7u || sb == 0x7Eu;
+        float eff = 0.0f, inv = 0.0f;
+        float ef[2] = {0.0f, 0.0f}, ei[2] = {0.0f, 0.0f};
+        if (sb != 0) {
+            eff = __fmul_rn(f32_from_e4m3(sb), ts);
+            inv = __frcp_rn(eff);
         }
-        store_codes<BITS>(codes + (int64_t)g * CB, out);
+        if constexpr (BITS == 6) {
+            uint32_t out[16];
+            if (sb == 0) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) out[i] = 0;
+            } else {
+                uint32_t cf[16], ci[16];
+                if (clamp) if6_candidates<true>(xv, inv, c_int, nc_q, cf, ci, ef, ei);
+                else if6_candidates<false>(xv, inv, c_int, nc_q, cf, ci, ef, ei);
+                bool use_int = mode == W_INT;
+                if (mode == W_IF) {
+                    bool near;
+                    use_int = fast_int(ef, ei, near);
+                    if (near) use_int = ifw_int_wins_exact<DT, 6>(p, inv, c_int, int_tab);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) out[i] = use_int ? ci[i] : cf[i];
+                scale = sb | (use_int ? 0x80u : 0u);
+            }
+            store_codes6(codes + (int64_t)g * CB, out);
+        } else {
+            uint32_t out[4] = {0u, 0u, 0u, 0u};
+            if (sb != 0) {
+                uint32_t fq[4], iq[4];
+                if (clamp) if3_candidates<true>(xv, inv, nc_q, fq, iq, ef, ei);
+                else if3_candidates<false>(xv, inv, nc_q, fq, iq, ef, ei);
+                bool use_int = mode == W_INT;
+                if (mode == W_IF) {
+                    bool near;
+                    use_int = fast_int(ef, ei, near);
+                    // a group whose FP and INT values coincide element by
+                    // element (0 or +-4 on both grids: about one group in 17
+                    // of the activations) ties exactly and keeps FP, without
+                    // the binary64 rule
+                    if (near)
+                        use_int = if3_values_coincide(fq, iq)
+                                      ? false
+                                      : ifw_int_wins_exact<DT, 3>(p, inv, c_int, int_tab);
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) out[k] = use_int ? iq[k] : fq[k];
+                scale = sb | (use_int ? 0x80u : 0u);
+            }
+            store_quads3(codes + (int64_t)g * CB, out);
+        }
         scales[g] = (uint8_t)scale;
     }
     if (nonfinite && err) atomicOr(err, IF4_DEV_NONFINITE);

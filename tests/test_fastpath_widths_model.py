@@ -166,24 +166,104 @@ def test_fp_grids():
     assert np.signbit(fp_value(-0.01, 6)) and np.signbit(fp_value(-0.2, 3))
 
 
-def test_coinciding_values_tie_and_the_tie_test_finds_exactly_them():
-    """IF3 groups whose FP and INT values coincide element by element tie
-    under the rule (FP kept), and the kernels' test max |df + di| <= 2^-18
-    holds for exactly those groups: where the values coincide df + di is the
-    INT offset plus one rounding; where they differ it is at least 1/3."""
+def _e2m0_sets(v):
+    """The IF3 kernel's E2M0: three comparisons of a = |v| giving 1 or 0,
+    the unordered forms holding for NaN: (value, magnitude code)."""
+    a = abs(v)
+    s1 = 0.0 if a <= 0.5 else 1.0
+    s2 = 0.0 if a < 1.5 else 1.0
+    s3 = 0.0 if a <= 3.0 else 1.0
+    return s1 + s2 + 2.0 * s3, int(s1 + s2 + s3)
+
+
+def _codes3(v, clamp=False):
+    """(FP code, INT code) of one element as the IF3 kernel forms them."""
+    _, mag = _e2m0_sets(v)
+    fcode = mag | (4 if np.signbit(v) else 0)
+    vc = min(max(v, -2.0 ** 19), 2.0 ** 19) if clamp else v
+    k = int(np.rint(vc * 0.75))
+    if clamp:
+        k = min(max(k, -3), 3)
+    return fcode, k & 7
+
+
+def _coincide_codes(fcodes, icodes):
+    """The kernel's test, on 12-bit quads of 3-bit codes."""
+    t = 0
+    for q in range(4):
+        fq = sum(c << (3 * i) for i, c in enumerate(fcodes[4 * q:4 * q + 4]))
+        iq = sum(c << (3 * i) for i, c in enumerate(icodes[4 * q:4 * q + 4]))
+        t |= (fq ^ (fq >> 1)) | (fq ^ iq)
+    return (t & 0x249) == 0
+
+
+def _v_sweep():
+    """Every binary32 value near the comparison and rounding boundaries of
+    both grids (1/2, 2/3, 3/2, 2, 3, 10/3), a dense grid over the range,
+    zeros of both signs, both infinities and large values."""
+    vals = set()
+    for b in (0.5, 2 / 3, 1.5, 2.0, 3.0, 10 / 3, 4.0):
+        c = np.float32(b)
+        for d in range(-40, 41):
+            vals.add(float(np.nextafter(c, np.float32(np.inf)) if d > 0 else c) if abs(d) <= 1
+                     else float(c + np.float32(d) * np.spacing(c)))
+    vals.update(float(t) for t in np.linspace(0, 4.5, 9001, dtype=np.float32))
+    vals.update([0.0, 2.0 ** -140, 1e30, 2.0 ** 19, 2.0 ** 25, float("inf")])
+    return sorted(vals | {-t for t in vals})
+
+
+def test_e2m0_by_comparisons_is_the_grid_rounding():
+    """The comparisons give the E2M0 rounding with ties to the even code
+    (the oracle's grid and tie rule, restated by fp_value), NaN to 4."""
+    for v in _v_sweep():
+        q, mag = _e2m0_sets(v)
+        assert q == abs(fp_value(v, 3)), v
+        assert [0.0, 1.0, 2.0, 4.0][mag] == q
+    assert _e2m0_sets(float("nan")) == (4.0, 3)
+
+
+def test_float_packing_of_fp_codes_is_exact():
+    """The FP quad as the float 2^23 + sum(code_i 8^i), accumulated as
+    2^23 + A w + (4 sign + s3) w per element, reads back the packed codes."""
+    rng = np.random.default_rng(41)
+    for _ in range(2000):
+        codes = rng.integers(0, 8, 4)
+        acc = F32(2.0 ** 23)
+        for i, c in enumerate(codes):
+            mag, sign = int(c) & 3, int(c) >> 2
+            s3 = float(mag == 3)
+            A = F32(mag - s3)
+            w = F32(8 ** i)
+            acc = F32(acc + A * w)
+            acc = F32(acc + F32(F32(sign * 4.0) + F32(s3)) * w)
+        bits = int(np.array([acc], dtype=np.float32).view(np.uint32)[0]) & 0xFFF
+        assert bits == sum(int(c) << (3 * i) for i, c in enumerate(codes))
+
+
+@pytest.mark.parametrize("clamp", [False, True])
+def test_code_test_finds_exactly_the_coinciding_elements(clamp):
+    """Per element over the sweep, and per group on random groups: the
+    kernels' code test holds exactly where the FP value and the rule's INT
+    value coincide (both 0, or both +-4), under both the unclamped and the
+    clamped integer."""
+    sweep = [v for v in _v_sweep() if clamp or abs(v) < 2.0 ** 19]
+    for v in sweep:
+        f, i = _codes3(v, clamp)
+        same = fp_value(v, 3) == int_value(float(np.clip(np.rint(
+            (min(max(v, -2.0 ** 19), 2.0 ** 19) if clamp else v) * 0.75), -3, 3)), 3)
+        assert _coincide_codes([f] * 16, [i] * 16) == same, v
     rng = np.random.default_rng(23)
-    cq = WIDTHS[3]["cq"]
     hits = 0
     for _ in range(3000):
         # mostly small elements (both grids 0), the maximum at +-4 (both 4)
         v16 = [r32(t) for t in rng.normal(0, 0.3, 16)]
         v16[rng.integers(16)] = float(rng.choice([-1.0, 1.0]) * 4.0)
         same = all(fp_value(v, 3) == int_value(int_k(v, 3), 3) for v in v16)
-        tie = max(abs(r32(r32(fp_value(v, 3) - v) + fma32(int_k(v, 3), -cq, v))) for v in v16)
-        assert (tie <= 2.0 ** -18) == same
+        f, i = zip(*(_codes3(v, clamp) for v in v16))
+        assert _coincide_codes(list(f), list(i)) == same
         if same:
             hits += 1
-            assert not exact_decision(v16, 3)
+            assert not exact_decision(v16, 3)          # a tie keeps FP
     assert 0 < hits < 3000
 
 

@@ -113,6 +113,21 @@ def test_tiny_zero_and_saturated_groups(bits):
 
 
 @pytest.mark.parametrize("bits", [6, 3])
+def test_scaled_values_overflow(bits):
+    """A given tensor scale (2^-117) far below the data's: every block scale
+    saturates and v = x * fl(1/fl(448 ts)) overflows binary32 to +-Inf for
+    all but the zero elements.  FP saturates, INT clamps to +-kmax, both
+    error sums are infinite, and the rule keeps FP."""
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((8, 64)) * 1e37).astype(np.float32)
+    x[0, :4] = [3e38, -3e38, 0.0, -0.0]
+    for mode in ("adaptive", "fp", "int"):
+        ref = check_w(torch.from_numpy(x), bits, "overflowing v", mode, ts=np.float32(2.0 ** -117),
+                      dequant=mode == "adaptive")
+        assert ((ref["scales"] & 0x7F) == 0x7E).all()
+
+
+@pytest.mark.parametrize("bits", [6, 3])
 def test_strided_rows(bits):
     base = workloads.llm_weight(5, rows=128, cols=1024 + 64)
     x_dev = base.cuda()[:, 8:8 + 1024]
