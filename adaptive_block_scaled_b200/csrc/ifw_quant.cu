@@ -407,32 +407,58 @@ __device__ __forceinline__ void if3_candidates(const float (&xv)[16], float inv,
                                                uint32_t (&fq)[4], uint32_t (&iq)[4],
                                                float (&ef)[2], float (&ei)[2])
 {
+    // element pairs (4k + 2p, 4k + 2p + 1) in paired binary32 instructions,
+    // each lane rounded as its scalar form (60.8 against 65.6 us scalar on
+    // the 8192 x 8192 activation); the FP quad in two lanes (even elements
+    // from 2^23, odd ones from 0) added at the end, exactly
+    const f2_t INV = f2_pack(inv, inv), C = f2_pack(0.75f, 0.75f);
+    const f2_t M = f2_pack(kMagic, kMagic), NM = f2_pack(-kMagic, -kMagic);
+    const f2_t NCQ = f2_pack(nc_q, nc_q), TWO = f2_pack(2.0f, 2.0f), FOUR = f2_pack(4.0f, 4.0f);
+    f2_t EF = f2_pack(ef[0], ef[1]), EI = f2_pack(ei[0], ei[1]);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        float acc = 0x1p23f;
+        f2_t ACC = f2_pack(0x1p23f, 0.0f);
         uint32_t iw = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int e = 4 * k + i;
-            const float w = (float)(1 << (3 * i));          // 8^i
-            const float v = __fmul_rn(xv[e], inv);
-            const float a = fabsf(v);
-            const float s1 = set_gtu(a, 0.5f), s2 = set_geu(a, 1.5f), s3 = set_gtu(a, 3.0f);
-            const float A = __fadd_rn(s1, s2);
-            const float df = __fsub_rn(__fmaf_rn(s3, 2.0f, A), a);
-            acc = __fmaf_rn(A, w, acc);
-            acc = __fmaf_rn(__fmaf_rn(sign_bit_f(v), 4.0f, s3), w, acc);
-            const float vc = CLAMP ? fminf(fmaxf(v, -0x1p19f), 0x1p19f) : v;
-            float r = __fmaf_rn(vc, 0.75f, kMagic);
-            if (CLAMP) r = fminf(fmaxf(r, kMagic - 3.0f), kMagic + 3.0f);
-            iw |= (__float_as_uint(r) & 7u) << (3 * i);      // two's complement
-            const float di = __fmaf_rn(__fsub_rn(r, kMagic), nc_q, v);
-            ef[i & 1] = __fmaf_rn(df, df, ef[i & 1]);
-            ei[i & 1] = __fmaf_rn(di, di, ei[i & 1]);
+        for (int p = 0; p < 2; ++p) {
+            const int e = 4 * k + 2 * p;
+            const f2_t W = f2_pack((float)(1 << (6 * p)), (float)(1 << (6 * p + 3)));   // 8^i
+            const f2_t V = f2_mul(f2_pack(xv[e], xv[e + 1]), INV);
+            float v0, v1;
+            f2_unpack(V, v0, v1);
+            const float a0 = fabsf(v0), a1 = fabsf(v1);
+            const f2_t S1 = f2_pack(set_gtu(a0, 0.5f), set_gtu(a1, 0.5f));
+            const f2_t S2 = f2_pack(set_geu(a0, 1.5f), set_geu(a1, 1.5f));
+            const f2_t S3 = f2_pack(set_gtu(a0, 3.0f), set_gtu(a1, 3.0f));
+            const f2_t SG = f2_pack(sign_bit_f(v0), sign_bit_f(v1));
+            const f2_t A = f2_add(S1, S2);
+            const f2_t DF = f2_sub(f2_fma(S3, TWO, A), f2_pack(a0, a1));
+            ACC = f2_fma(A, W, ACC);
+            ACC = f2_fma(f2_fma(SG, FOUR, S3), W, ACC);
+            f2_t VC = V;
+            if constexpr (CLAMP)
+                VC = f2_pack(fminf(fmaxf(v0, -0x1p19f), 0x1p19f), fminf(fmaxf(v1, -0x1p19f), 0x1p19f));
+            f2_t R = f2_fma(VC, C, M);
+            float r0, r1;
+            f2_unpack(R, r0, r1);
+            if constexpr (CLAMP) {
+                r0 = fminf(fmaxf(r0, kMagic - 3.0f), kMagic + 3.0f);
+                r1 = fminf(fmaxf(r1, kMagic - 3.0f), kMagic + 3.0f);
+                R = f2_pack(r0, r1);
+            }
+            iw |= ((__float_as_uint(r0) & 7u) << (6 * p)) |           // two's complement
+                  ((__float_as_uint(r1) & 7u) << (6 * p + 3));
+            const f2_t DI = f2_fma(f2_add(R, NM), NCQ, V);
+            EF = f2_fma(DF, DF, EF);
+            EI = f2_fma(DI, DI, EI);
         }
-        fq[k] = __float_as_uint(acc) & 0xFFFu;
+        float acc0, acc1;
+        f2_unpack(ACC, acc0, acc1);
+        fq[k] = __float_as_uint(__fadd_rn(acc0, acc1)) & 0xFFFu;
         iq[k] = iw;
     }
+    f2_unpack(EF, ef[0], ef[1]);
+    f2_unpack(EI, ei[0], ei[1]);
 }
 
 // IF3: true when the FP and INT values of every element coincide (both 0, or
