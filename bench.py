@@ -68,7 +68,7 @@ def parse():
                    help="skip the per-workload parity and quality block")
     p.add_argument("--kernel-only", default=None,
                    choices=["amax", "if4_quantize", "if4_dequantize", "nvfp4_quantize", "gemm",
-                            "linear_fused",
+                            "linear_fused", "linear_quantized",
                             "nvint4_quantize", "nvfp4_4over6_quantize", "if4_quantize_rht",
                             "if4_decode_f16", "fused_quantize", "fused_quantize_rht",
                             "fused_quantize_dequant", "if6_quantize", "if3_quantize",
@@ -995,7 +995,7 @@ def run_ours(args):
 def run_kernel_only(args):
     """Only the chosen kernel, on the chosen workload: the command ncu wraps."""
     from adaptive_block_scaled_b200 import binding as b
-    if args.kernel_only in ("gemm", "linear_fused"):
+    if args.kernel_only in ("gemm", "linear_fused", "linear_quantized"):
         M, N, K = 8192, 4096, 4096
         a, bw = make_input("linear_8192x4096x4096")
         dev = torch.device("cuda")
@@ -1003,9 +1003,21 @@ def run_kernel_only(args):
         wa, wb = b.decode_f16(aq[0], aq[1]), b.decode_f16(bq[0], bq[1])
         c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         err = torch.zeros(1, dtype=torch.int32, device=dev)
+        if args.kernel_only == "linear_quantized":
+            # the output's tensor scale from one plain linear first
+            ws = torch.empty(b.if4_linear_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+            b.if4_linear(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], ws, c, err)
+            c_ts = torch.ones(1, dtype=torch.float32, device=dev)
+            b.if4_tensor_amax(c, c_ts)
+            b.if4_tensor_scale(c_ts, c_ts)
+            c_codes = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
+            c_scales = torch.empty((M, N // 16), dtype=torch.uint8, device=dev)
         for _ in range(args.warmup + args.steps):
             if args.kernel_only == "gemm":
                 b.if4_gemm_f16(wa, wb, aq[2], bq[2], c, err)
+            elif args.kernel_only == "linear_quantized":
+                b.if4_linear_quantized(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], ws, c_codes,
+                                       c_scales, c_ts, err_flag=err)
             else:
                 b.if4_linear_fused(aq[0], aq[1], aq[2], bq[0], bq[1], bq[2], c, err)
         torch.cuda.synchronize()
