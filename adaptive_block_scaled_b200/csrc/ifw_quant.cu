@@ -265,9 +265,12 @@ __device__ __forceinline__ void unpack_code_words(const uint32_t (&w)[3], uint32
 
 __device__ __forceinline__ bool ts_ok(float ts) { return ts >= 0x1p-117f && ts <= 0x1p117f; }
 
-// Block scale sb_f = fl(fl(amax / fpmax) / ts).  The first quotient is an
-// IEEE division for IF6 and the exact amax * 1/4 for IF3 (amax >= 2^-124);
-// the second is Markstein's: with y = fl(1/ts), s = fl(a y), fl(s + fl(a - s
+// Block scale sb_f = fl(fl(amax / fpmax) / ts).  The first quotient is the
+// exact amax * 1/4 for IF3 (amax >= 2^-124); for IF6 it is q = fl(amax y)
+// with y = fl(1/7.5), corrected once to q + fl(amax - 7.5 q) y, which equals
+// the IEEE division for every finite amax >= 2^-100 (checked on the CPU for
+// every mantissa); below, and for Inf or NaN, the IEEE division.  The second
+// quotient is Markstein's: with y = fl(1/ts), s = fl(a y), fl(s + fl(a - s
 // ts) y) is the correctly rounded a / ts when neither quotient over- nor
 // underflows.  Below a = 2^-100 the IEEE division is used; from s = 2^100 the
 // unrefined s is returned (any such value saturates to 448, as the exact one
@@ -276,10 +279,15 @@ template <int BITS>
 __device__ __forceinline__ float block_scale_w(float amax, float ts, float rts)
 {
     float a;
-    if constexpr (BITS == 3)
+    if constexpr (BITS == 3) {
         a = amax >= 0x1p-124f ? __fmul_rn(amax, 0.25f) : __fdiv_rn(amax, 4.0f);
-    else
+    } else if (amax >= 0x1p-100f && amax <= 3.4028235e38f) {
+        const float y = __uint_as_float(0x3E088889u);       // fl(1/7.5)
+        const float q = __fmul_rn(amax, y);
+        a = __fmaf_rn(__fmaf_rn(-q, 7.5f, amax), y, q);
+    } else {
         a = __fdiv_rn(amax, Width<BITS>::fpmax);
+    }
     const float s = __fmul_rn(a, rts);
     if (!(a >= 0x1p-100f && s < 0x1p100f)) return a >= 0x1p-100f ? s : __fdiv_rn(a, ts);
     return __fmaf_rn(__fmaf_rn(-s, ts, a), rts, s);

@@ -295,3 +295,38 @@ def test_block_scale_second_quotient_equals_the_ieee_division(bits):
     assert valid.sum() > n // 2
     bad = valid & (got != want)
     assert not bad.any(), (amax[bad][:5], ts[bad][:5])
+
+
+def _markstein_div75(amax):
+    """The IF6 kernel's fl(amax / 7.5): q = fl(amax * fl(1/7.5)), then q +
+    fl(amax - 7.5 q) * fl(1/7.5) in one fused multiply-add."""
+    a = amax.astype(np.float64)
+    r = float(np.float32(1.0) / np.float32(7.5))
+    q = (a * r).astype(np.float32).astype(np.float64)
+    n = a.size
+    return _fma32_vec(_fma32_vec(-q, np.full(n, 7.5), a), np.full(n, r), q)
+
+
+def test_amax_over_7_5_quotient_every_mantissa_and_exponent():
+    """IF6's first block-scale quotient by the two-step form equals the IEEE
+    division for every one of the 2^23 binary32 values in [1, 2), and for
+    4096 mantissas (the 2048 smallest and largest, random ones filling the
+    rest) of every binade from 2^-100 (below it the kernel divides) to the
+    largest finite float.  Away from under- and overflow both sides scale
+    exactly with a power of two, so the first binade covers every mantissa
+    of every binade; the sampled binades check the ends."""
+    one_binade = (np.arange(1 << 23, dtype=np.uint32) | np.uint32(127 << 23)).view(np.float32)
+    got = _markstein_div75(one_binade)
+    want = (one_binade / np.float32(7.5)).astype(np.float64)
+    assert np.array_equal(got, want)
+    rng = np.random.default_rng(37)
+    mant = np.concatenate([np.arange(1024), (1 << 23) - 1 - np.arange(1024),
+                           rng.integers(0, 1 << 23, 2048)]).astype(np.uint32)
+    exps = np.arange(27, 255, dtype=np.uint32)          # 2^-100 .. 2^127
+    bits = (exps[:, None] << np.uint32(23)) | mant[None, :]
+    amax = bits.ravel().view(np.float32)
+    with np.errstate(over="ignore"):
+        got = _markstein_div75(amax)
+        want = (amax / np.float32(7.5)).astype(np.float64)
+    bad = got != want
+    assert not bad.any(), amax[bad][:5]

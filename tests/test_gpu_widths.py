@@ -97,23 +97,26 @@ def test_every_bf16_value_both_candidates(bits):
 
 
 @pytest.mark.parametrize("bits", [6, 3])
-def test_tiny_zero_and_saturated_groups(bits):
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_tiny_zero_and_saturated_groups(bits, dtype):
     rng = np.random.default_rng(31)
     x = rng.standard_normal((64, 256)).astype(np.float32)
     x *= np.exp2(-rng.integers(0, 30, (64, 16))).repeat(16, axis=1).astype(np.float32)
     x[0, 0] = 1000.0
     x[1, :16] = -0.0
     x[2, 16:32] = -1e-7
-    ref = check_w(torch.from_numpy(x), bits, "tiny groups")
+    xt = torch.from_numpy(x).to(dtype)
+    ref = check_w(xt, bits, "tiny groups")
     sb = ref["scales"] & 0x7F
     assert (sb == 0).any() and ((sb > 0) & (sb < 8)).any()
-    amax = float(np.abs(x).max())
+    amax = float(xt.float().abs().max())
     fpmax = 7.5 if bits == 6 else 4.0
-    check_w(torch.from_numpy(x), bits, "saturating ts", ts=np.float32(amax / (fpmax * 448) / 64))
+    check_w(xt, bits, "saturating ts", ts=np.float32(amax / (fpmax * 448) / 64))
 
 
 @pytest.mark.parametrize("bits", [6, 3])
-def test_scaled_values_overflow(bits):
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_scaled_values_overflow(bits, dtype):
     """A given tensor scale (2^-117) far below the data's: every block scale
     saturates and v = x * fl(1/fl(448 ts)) overflows binary32 to +-Inf for
     all but the zero elements.  FP saturates, INT clamps to +-kmax, both
@@ -122,8 +125,8 @@ def test_scaled_values_overflow(bits):
     x = (rng.standard_normal((8, 64)) * 1e37).astype(np.float32)
     x[0, :4] = [3e38, -3e38, 0.0, -0.0]
     for mode in ("adaptive", "fp", "int"):
-        ref = check_w(torch.from_numpy(x), bits, "overflowing v", mode, ts=np.float32(2.0 ** -117),
-                      dequant=mode == "adaptive")
+        ref = check_w(torch.from_numpy(x).to(dtype), bits, "overflowing v", mode,
+                      ts=np.float32(2.0 ** -117), dequant=mode == "adaptive")
         assert ((ref["scales"] & 0x7F) == 0x7E).all()
 
 
