@@ -546,6 +546,13 @@ ifw_quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, 
     const float c_int = BITS == 6 ? __fdiv_rn(62.0f, 15.0f) : 0.75f;
     const float nc_q = BITS == 6 ? -__fdiv_rn(15.0f, 62.0f) : -__fdiv_rn(4.0f, 3.0f);
     const float rts = __frcp_rn(ts);
+    // IF3: inv = fl(1/fl(E4M3 * ts)) of every block scale byte, once per
+    // block (58.6 against 59.2 us on the 8192 x 8192 activation; IF6 measured
+    // 56.8 against 56.5 us with it and computes it per group)
+    __shared__ float inv_tab[BITS == 3 ? 128 : 1];
+    if (BITS == 3 && threadIdx.x < 128)
+        inv_tab[threadIdx.x] =
+            threadIdx.x == 0 ? 0.0f : __frcp_rn(__fmul_rn(f32_from_e4m3(threadIdx.x), ts));
     __syncthreads();
     bool nonfinite = false;
     const bool contig = ld_bytes == (int64_t)gpr * GB;
@@ -591,12 +598,9 @@ ifw_quantize_kernel(const char *__restrict__ x, int64_t ld_bytes, uint32_t gpr, 
         // a subnormal or the largest block scale: v may leave the range the
         // unclamped path relies on
         const bool clamp = (sb - 1u) < 7u || sb == 0x7Eu;
-        float eff = 0.0f, inv = 0.0f;
+        const float inv = BITS == 3 ? inv_tab[sb]
+                          : (sb != 0 ? __frcp_rn(__fmul_rn(f32_from_e4m3(sb), ts)) : 0.0f);
         float ef[2] = {0.0f, 0.0f}, ei[2] = {0.0f, 0.0f};
-        if (sb != 0) {
-            eff = __fmul_rn(f32_from_e4m3(sb), ts);
-            inv = __frcp_rn(eff);
-        }
         if constexpr (BITS == 6) {
             uint32_t out[16];
             if (sb == 0) {
