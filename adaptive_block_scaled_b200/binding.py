@@ -58,6 +58,8 @@ def _load():
                                    _vp, _vp, _vp, _vp, _vp],
         "if4_quantize_fused_dequant": [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp,
                                        _vp, _vp, _vp, _vp],
+        "if4_quantize_fused_dequant_shared": [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp,
+                                              _vp, _vp, _vp, _int, _vp, _vp],
         "if4_decode_f16": [_vp, _vp, _i64, _i64, _vp, _vp],
         "if4_gemm_f16": [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
         "if4_linear_workspace_bytes": [_i64, _i64, _i64],
@@ -410,6 +412,29 @@ def if4_quantize_fused_dequant(x, codes, scales, nv_codes, nv_scales, ts, sync_w
                                err_flag=None, stream=None):
     """The single launch that also writes y, the bf16 decode of its IF4 codes
     (dense, 32-byte aligned)."""
+    rows, cols, ld = _fused_dequant_args(x, codes, scales, nv_codes, nv_scales, sync_words, y)
+    _check(lib.if4_quantize_fused_dequant(_ptr(x), _dtype(x, "x"), rows, cols, ld, _ptr(codes),
+                                          _ptr(scales), _ptr(nv_codes), _ptr(nv_scales),
+                                          _ptr(ts), _ptr(sync_words), _ptr(y), _ptr(err_flag),
+                                          _stream(stream)),
+           "if4_quantize_fused_dequant")
+
+
+def if4_quantize_fused_dequant_shared(x, codes, scales, nv_codes, nv_scales, ts, sync_words, y,
+                                      share, err_flag=None, stream=None):
+    """The same launch on 1/share of the device's resident blocks, for
+    `share` calls at once on different streams (each with its own
+    sync_words); outputs byte-identical to if4_quantize_fused_dequant."""
+    rows, cols, ld = _fused_dequant_args(x, codes, scales, nv_codes, nv_scales, sync_words, y)
+    _check(lib.if4_quantize_fused_dequant_shared(_ptr(x), _dtype(x, "x"), rows, cols, ld,
+                                                 _ptr(codes), _ptr(scales), _ptr(nv_codes),
+                                                 _ptr(nv_scales), _ptr(ts), _ptr(sync_words),
+                                                 _ptr(y), int(share), _ptr(err_flag),
+                                                 _stream(stream)),
+           "if4_quantize_fused_dequant_shared")
+
+
+def _fused_dequant_args(x, codes, scales, nv_codes, nv_scales, sync_words, y):
     rows, cols, ld = _matrix(x, "x")
     _u8(codes, "codes", (rows, cols // 2))
     _u8(scales, "scales", (rows, cols // 16))
@@ -423,11 +448,7 @@ def if4_quantize_fused_dequant(x, codes, scales, nv_codes, nv_scales, ts, sync_w
                          f"{FUSED_SYNC_WORDS} elements")
     if y.dtype != torch.bfloat16 or tuple(y.shape) != (rows, cols) or not y.is_contiguous():
         raise ValueError("y must be a dense bf16 tensor of the shape of x")
-    _check(lib.if4_quantize_fused_dequant(_ptr(x), _dtype(x, "x"), rows, cols, ld, _ptr(codes),
-                                          _ptr(scales), _ptr(nv_codes), _ptr(nv_scales),
-                                          _ptr(ts), _ptr(sync_words), _ptr(y), _ptr(err_flag),
-                                          _stream(stream)),
-           "if4_quantize_fused_dequant")
+    return rows, cols, ld
 
 
 def quantize_fused_dequant(x, with_nvfp4=True, sync_words=None, err_flag=None, stream=None):

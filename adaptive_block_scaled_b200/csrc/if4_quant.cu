@@ -1332,11 +1332,13 @@ template <int DT, bool V8, bool RHT, bool NV, bool DQ = false>
 int launch_fused(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
                  uint8_t *nv_codes, uint8_t *nv_scales, float *ts, uint32_t *sync, int *err,
                  cudaStream_t st, const DeviceInfo &d, const SignMasks &sm, uint32_t signs,
-                 void *y = nullptr)
+                 void *y = nullptr, int share = 1)
 {
     auto k = quantize_fused_kernel<DT, V8, RHT, NV, DQ>;
     static const int occ = resident_blocks(k, 256);
-    const uint32_t grid = grid_for(occ, d, s.ngroups, 256);
+    // a share of the device: floor(occ / share) blocks per SM, so that
+    // `share` launches on other streams are resident at the same time
+    const uint32_t grid = grid_for(std::max(1, occ / share), d, s.ngroups, 256);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(256, 1, 1);
@@ -1366,7 +1368,7 @@ template <int DT, bool RHT>
 int dispatch_fused_dt(const Shape &s, const void *x, uint8_t *codes, uint8_t *scales,
                       uint8_t *nv_codes, uint8_t *nv_scales, float *ts, uint32_t *sync, int *err,
                       cudaStream_t st, const DeviceInfo &d, const SignMasks &sm, uint32_t signs,
-                      void *y)
+                      void *y, int share)
 {
     const bool nv = nv_codes != nullptr;
     if constexpr (!RHT) {
@@ -1374,27 +1376,29 @@ int dispatch_fused_dt(const Shape &s, const void *x, uint8_t *codes, uint8_t *sc
             if (s.v8)
                 return nv ? launch_fused<DT, true, false, true, true>(
                                 s, x, codes, scales, nv_codes, nv_scales, ts, sync, err, st, d, sm,
-                                signs, y)
+                                signs, y, share)
                           : launch_fused<DT, true, false, false, true>(
                                 s, x, codes, scales, nv_codes, nv_scales, ts, sync, err, st, d, sm,
-                                signs, y);
+                                signs, y, share);
             return nv ? launch_fused<DT, false, false, true, true>(
                             s, x, codes, scales, nv_codes, nv_scales, ts, sync, err, st, d, sm,
-                            signs, y)
+                            signs, y, share)
                       : launch_fused<DT, false, false, false, true>(
                             s, x, codes, scales, nv_codes, nv_scales, ts, sync, err, st, d, sm,
-                            signs, y);
+                            signs, y, share);
         }
     }
     if (s.v8)
         return nv ? launch_fused<DT, true, RHT, true>(s, x, codes, scales, nv_codes, nv_scales, ts,
-                                                      sync, err, st, d, sm, signs)
+                                                      sync, err, st, d, sm, signs, nullptr,
+                                                      share)
                   : launch_fused<DT, true, RHT, false>(s, x, codes, scales, nv_codes, nv_scales,
-                                                       ts, sync, err, st, d, sm, signs);
+                                                       ts, sync, err, st, d, sm, signs, nullptr,
+                                                       share);
     return nv ? launch_fused<DT, false, RHT, true>(s, x, codes, scales, nv_codes, nv_scales, ts,
-                                                   sync, err, st, d, sm, signs)
+                                                   sync, err, st, d, sm, signs, nullptr, share)
               : launch_fused<DT, false, RHT, false>(s, x, codes, scales, nv_codes, nv_scales, ts,
-                                                    sync, err, st, d, sm, signs);
+                                                    sync, err, st, d, sm, signs, nullptr, share);
 }
 
 template <int ODT, bool UNIT_TS>
@@ -1417,11 +1421,12 @@ template <bool RHT>
 int fused_entry(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
                 uint8_t *codes, uint8_t *scales, uint8_t *nv_codes, uint8_t *nv_scales, float *ts,
                 uint32_t *sync_words, int *err_flag, void *stream, uint32_t signs,
-                void *y = nullptr)
+                void *y = nullptr, int share = 1)
 {
     Shape s;
     int rc = check_tensor(x, x_dtype, rows, cols, ld_x, s);
     if (rc != IF4_OK) return rc;
+    if (share < 1 || share > 64) return IF4_ERR_SHAPE;
     if (ts == nullptr || sync_words == nullptr) return IF4_ERR_NULL;
     if ((nv_codes == nullptr) != (nv_scales == nullptr)) return IF4_ERR_NULL;
     if (s.ngroups > 0 && (codes == nullptr || scales == nullptr)) return IF4_ERR_NULL;
@@ -1442,13 +1447,13 @@ int fused_entry(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t 
     switch (x_dtype) {
     case IF4_F32:
         return dispatch_fused_dt<DT_F32, RHT>(s, x, codes, scales, nv_codes, nv_scales, ts,
-                                                sync_words, err_flag, st, d, sm, signs, y);
+                                                sync_words, err_flag, st, d, sm, signs, y, share);
     case IF4_BF16:
         return dispatch_fused_dt<DT_BF16, RHT>(s, x, codes, scales, nv_codes, nv_scales, ts,
-                                                 sync_words, err_flag, st, d, sm, signs, y);
+                                                 sync_words, err_flag, st, d, sm, signs, y, share);
     default:
         return dispatch_fused_dt<DT_F16, RHT>(s, x, codes, scales, nv_codes, nv_scales, ts,
-                                                sync_words, err_flag, st, d, sm, signs, y);
+                                                sync_words, err_flag, st, d, sm, signs, y, share);
     }
 }
 
@@ -1562,6 +1567,18 @@ int if4_quantize_fused_dequant(const void *x, int x_dtype, int64_t rows, int64_t
     if (reinterpret_cast<uintptr_t>(y) % 32 != 0) return IF4_ERR_ALIGN;
     return fused_entry<false>(x, x_dtype, rows, cols, ld_x, codes, scales, nv_codes, nv_scales, ts,
                               sync_words, err_flag, stream, 0u, y);
+}
+
+int if4_quantize_fused_dequant_shared(const void *x, int x_dtype, int64_t rows, int64_t cols,
+                                      int64_t ld_x, uint8_t *codes, uint8_t *scales,
+                                      uint8_t *nv_codes, uint8_t *nv_scales, float *ts,
+                                      uint32_t *sync_words, void *y, int share, int *err_flag,
+                                      void *stream)
+{
+    if (rows > 0 && cols > 0 && y == nullptr) return IF4_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(y) % 32 != 0) return IF4_ERR_ALIGN;
+    return fused_entry<false>(x, x_dtype, rows, cols, ld_x, codes, scales, nv_codes, nv_scales, ts,
+                              sync_words, err_flag, stream, 0u, y, share);
 }
 
 int if4_quantize_fused_rht(const void *x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,

@@ -198,6 +198,27 @@ int if4_quantize_fused_dequant(const void *x, int x_dtype, int64_t rows, int64_t
                                int *err_flag, void *stream);
 
 /*
+ * if4_quantize_fused_dequant on a share of the device.  The launch sizes its
+ * grid to floor(R / share) blocks per SM (at least one), R being the blocks
+ * of this kernel one SM holds, so that `share` such calls on different
+ * streams, each with its own sync_words, are resident together: the amax
+ * pass of one runs beside the encode pass of another.  Independent tensors
+ * (consecutive steps, the layers of a model) quantized this way on two
+ * streams take less time in total than one after another on one stream,
+ * while each call alone takes longer.  share = 1 is
+ * if4_quantize_fused_dequant.  The outputs do not depend on share: they are
+ * byte-identical to if4_quantize_fused_dequant's.  IF4_ERR_SHAPE for share
+ * outside [1, 64]; other arguments and rules as if4_quantize_fused_dequant.
+ * Launches that share the device must not wait for one another (each call
+ * waits only for its own blocks).
+ */
+int if4_quantize_fused_dequant_shared(const void *x, int x_dtype, int64_t rows, int64_t cols,
+                                      int64_t ld_x, uint8_t *codes, uint8_t *scales,
+                                      uint8_t *nv_codes, uint8_t *nv_scales, float *ts,
+                                      uint32_t *sync_words, void *y, int share, int *err_flag,
+                                      void *stream);
+
+/*
  * The same single launch on the random-sign Hadamard transform of x (see
  * if4_quantize_rht): the amax, the tensor scale, the IF4 codes and the
  * NVFP4 comparator are those of the transformed tensor, equal to

@@ -30,6 +30,8 @@ def lib():
                                          vp, vp, vp, vp]
     L.if4_quantize_fused_dequant.argtypes = [vp, i, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp,
                                              vp, vp]
+    L.if4_quantize_fused_dequant_shared.argtypes = [vp, i, i64, i64, i64, vp, vp, vp, vp, vp, vp,
+                                                    vp, i, vp, vp]
     L.if4_linear_quantized.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, ctypes.c_size_t,
                                        vp, vp, vp, vp, vp, vp]
     L.if4_linear_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
@@ -128,6 +130,14 @@ def test_fused_quantize_host_validation(lib):
     assert h(A, 1, 4, 32, 32, A, A, None, None, None, A, A, None, None) == 1
     assert h(A, 1, 4, 24, 24, A, A, None, None, A, A, A, None, None) == 2
     assert h(A, 1, 4, 32, 32, A, A, None, None, A, A + 64, A, None, None) == 4
+    k = lib.if4_quantize_fused_dequant_shared
+    # the share of the device: 1..64; then the rules of the plain call
+    assert k(A, 1, 4, 32, 32, A, A, None, None, A, A, A, 0, None, None) == 2
+    assert k(A, 1, 4, 32, 32, A, A, None, None, A, A, A, 65, None, None) == 2
+    assert k(A, 1, 4, 32, 32, A, A, None, None, A, A, None, 2, None, None) == 1
+    assert k(A, 1, 4, 32, 32, A, A, None, None, A, A, A + 16, 2, None, None) == 4
+    assert k(A, 1, 4, 24, 24, A, A, None, None, A, A, A, 2, None, None) == 2
+    assert k(A, 1, 4, 32, 32, A, A, None, None, A, A + 64, A, 2, None, None) == 4
     g = lib.if4_quantize_fused_rht
     assert g(A, 1, 4, 32, 32, 0x1234, A, A, None, None, None, A, None, None) == 1
     assert g(A, 1, 4, 24, 24, 0x1234, A, A, None, None, A, A, None, None) == 2

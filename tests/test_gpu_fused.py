@@ -282,3 +282,68 @@ def test_fused_round_trip(case):
     assert np.array_equal(codes.cpu().numpy(), ref["codes"])
     want = torch.from_numpy(oracle.dequantize(ref["codes"], ref["scales"], ref["ts"]))
     assert torch.equal(y.cpu().view(torch.int16), want.to(torch.bfloat16).view(torch.int16))
+
+
+def _round_trip_buffers(x):
+    rows, cols = x.shape
+    dev = x.device
+    return dict(codes=torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev),
+                scales=torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev),
+                nc=torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev),
+                ns=torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev),
+                ts=torch.empty(1, dtype=torch.float32, device=dev),
+                y=torch.empty((rows, cols), dtype=torch.bfloat16, device=dev),
+                sync=torch.zeros(B().FUSED_SYNC_WORDS, dtype=torch.int32, device=dev))
+
+
+def _same(o, ref):
+    return (torch.equal(o["codes"], ref[0]) and torch.equal(o["scales"], ref[1])
+            and o["ts"].item() == ref[2].item() and torch.equal(o["nc"], ref[3])
+            and torch.equal(o["ns"], ref[4])
+            and torch.equal(o["y"].view(torch.int16), ref[5].view(torch.int16)))
+
+
+@pytest.mark.parametrize("share", [1, 2, 3, 4, 64])
+def test_shared_round_trip_is_byte_identical(share):
+    """if4_quantize_fused_dequant_shared: the grid shrinks to 1/share of the
+    resident blocks (64: one block per SM), the outputs do not change."""
+    b = B()
+    x = workloads.activation_outliers(1, tokens=2048, hidden=8192).cuda()
+    ref = b.quantize_fused_dequant(x)
+    o = _round_trip_buffers(x)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    b.if4_quantize_fused_dequant_shared(x, o["codes"], o["scales"], o["nc"], o["ns"], o["ts"],
+                                        o["sync"], o["y"], share, err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and o["sync"][0].item() == 0 and o["sync"][1].item() == 0
+    assert _same(o, ref)
+
+
+def test_shared_launches_on_two_streams_at_once():
+    """Two tensors quantized by shared launches (share 2) on two streams, six
+    calls each, each stream with its own buffers and synchronisation words:
+    every result equals the plain single-stream call on the same tensor."""
+    b = B()
+    xs = [workloads.activation_outliers(s, tokens=4096, hidden=8192).cuda() for s in (2, 3)]
+    refs = [b.quantize_fused_dequant(x) for x in xs]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    bufs = [_round_trip_buffers(x) for x in xs]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cur = torch.cuda.current_stream()
+    for s in streams:
+        s.wait_stream(cur)
+    for rep in range(6):
+        for k in (0, 1):
+            o = bufs[k]
+            with torch.cuda.stream(streams[k]):
+                b.if4_quantize_fused_dequant_shared(xs[k], o["codes"], o["scales"], o["nc"],
+                                                    o["ns"], o["ts"], o["sync"], o["y"], 2,
+                                                    err_flag=err)
+    for s in streams:
+        cur.wait_stream(s)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for k in (0, 1):
+        assert bufs[k]["sync"][0].item() == 0 and bufs[k]["sync"][1].item() == 0
+        assert _same(bufs[k], refs[k])
