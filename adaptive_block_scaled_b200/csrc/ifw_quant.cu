@@ -16,13 +16,15 @@
 // and element i's code sits at bits [w*i, w*i + w) of the group's
 // little-endian code bytes (12 per group for IF6, 6 for IF3).
 //
-// Design: one thread per group of 16 in a grid-stride loop.  FP6 codes come
-// from the hardware E2M3 conversion (round to nearest even, saturating), FP3
-// codes from compares; the INT integer from one fused multiply-add (a single
-// rounding of the exact product).  The decision takes IF4's fast path: the
-// two error sums in binary32, and the binary64 rule itself (its INT values
-// the correctly rounded quotients, from a shared table) only for a group
-// whose binary32 margin is within the band.
+// Design: one thread per group of 16 in a grid-stride loop, element pairs in
+// paired binary32 instructions.  FP6 codes come from the hardware E2M3
+// conversion (round to nearest even, saturating), FP3 codes from three
+// comparisons that give 1.0 or 0.0, summed and packed by exact FMAs; the INT
+// integer from one fused multiply-add (a single rounding of the exact
+// product).  The decision takes IF4's fast path: the two error sums in
+// binary32, and the binary64 rule itself (its INT values the correctly
+// rounded quotients, from a shared table) only for a group whose binary32
+// margin is within the band; IF3 first tests its codes for an exact tie.
 
 #include <cuda_runtime.h>
 
@@ -524,9 +526,9 @@ __device__ __forceinline__ bool fast_int(const float (&ef)[2], const float (&ei)
 //
 // Decision, fast path (as IF4's): the two squared-error sums in binary32,
 // two lanes of 8 fused multiply-adds each, then one add.  The FP differences
-// are exact; an INT difference is one fused multiply-add v - k * fl(c) (c =
-// 15/62 or 4/3), off from the rule's v - fl(num k / den) by at most 2^-20
-// plus one rounding.  Outside the band 2^-16 (S + 1) (S = the sum of both
+// are exact under every block scale but the clamped ones; an INT difference
+// is one fused multiply-add v - k * fl(c) (c = 15/62 or 4/3), off from the
+// rule's v - fl(num k / den) by at most 2^-20 plus one rounding.  Outside the band 2^-16 (S + 1) (S = the sum of both
 // errors) the binary32 sign is the rule's; inside it the group is decided by
 // the binary64 rule itself (ifw_int_wins_exact).
 template <int DT, int BITS>
