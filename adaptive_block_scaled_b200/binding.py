@@ -56,6 +56,10 @@ def _load():
                                _vp],
         "if4_quantize_fused_rht": [_vp, _int, _i64, _i64, _i64, ctypes.c_uint32, _vp, _vp, _vp,
                                    _vp, _vp, _vp, _vp, _vp],
+        "if4_quantize_fused_shared": [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
+                                      _int, _vp, _vp],
+        "if4_quantize_fused_rht_shared": [_vp, _int, _i64, _i64, _i64, ctypes.c_uint32, _vp, _vp,
+                                          _vp, _vp, _vp, _vp, _int, _vp, _vp],
         "if4_quantize_fused_dequant": [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp,
                                        _vp, _vp, _vp, _vp],
         "if4_quantize_fused_dequant_shared": [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp,
@@ -171,10 +175,7 @@ def if4_quantize_rht(x, signs, codes, scales, ts, ts_mode=TS_COMPUTE, err_flag=N
                                 _stream(stream)), "if4_quantize_rht")
 
 
-def if4_quantize_fused(x, codes, scales, nv_codes, nv_scales, ts, sync_words, err_flag=None,
-                       stream=None, signs=None):
-    """signs=None: the plain single-launch quantizer; an int: the same on the
-    random-sign Hadamard transform of x (if4_quantize_fused_rht)."""
+def _fused_args(x, codes, scales, nv_codes, nv_scales, sync_words):
     rows, cols, ld = _matrix(x, "x")
     _u8(codes, "codes", (rows, cols // 2))
     _u8(scales, "scales", (rows, cols // 16))
@@ -186,6 +187,36 @@ def if4_quantize_fused(x, codes, scales, nv_codes, nv_scales, ts, sync_words, er
     if sync_words.dtype != torch.int32 or sync_words.numel() < FUSED_SYNC_WORDS:
         raise ValueError(f"sync_words must be an int32 device tensor of at least "
                          f"{FUSED_SYNC_WORDS} elements")
+    return rows, cols, ld
+
+
+def if4_quantize_fused_shared(x, codes, scales, nv_codes, nv_scales, ts, sync_words, share,
+                              err_flag=None, stream=None, signs=None):
+    """The single-launch quantizer (signs=None) or its transform form on
+    1/share of the device's resident blocks (if4_quantize_fused_shared /
+    if4_quantize_fused_rht_shared); outputs byte-identical to the plain
+    call."""
+    rows, cols, ld = _fused_args(x, codes, scales, nv_codes, nv_scales, sync_words)
+    if signs is None:
+        _check(lib.if4_quantize_fused_shared(_ptr(x), _dtype(x, "x"), rows, cols, ld,
+                                             _ptr(codes), _ptr(scales), _ptr(nv_codes),
+                                             _ptr(nv_scales), _ptr(ts), _ptr(sync_words),
+                                             int(share), _ptr(err_flag), _stream(stream)),
+               "if4_quantize_fused_shared")
+    else:
+        _check(lib.if4_quantize_fused_rht_shared(_ptr(x), _dtype(x, "x"), rows, cols, ld,
+                                                 int(signs) & 0xFFFF, _ptr(codes), _ptr(scales),
+                                                 _ptr(nv_codes), _ptr(nv_scales), _ptr(ts),
+                                                 _ptr(sync_words), int(share), _ptr(err_flag),
+                                                 _stream(stream)),
+               "if4_quantize_fused_rht_shared")
+
+
+def if4_quantize_fused(x, codes, scales, nv_codes, nv_scales, ts, sync_words, err_flag=None,
+                       stream=None, signs=None):
+    """signs=None: the plain single-launch quantizer; an int: the same on the
+    random-sign Hadamard transform of x (if4_quantize_fused_rht)."""
+    rows, cols, ld = _fused_args(x, codes, scales, nv_codes, nv_scales, sync_words)
     if signs is None:
         _check(lib.if4_quantize_fused(_ptr(x), _dtype(x, "x"), rows, cols, ld, _ptr(codes),
                                       _ptr(scales), _ptr(nv_codes), _ptr(nv_scales), _ptr(ts),

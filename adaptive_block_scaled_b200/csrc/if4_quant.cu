@@ -1558,6 +1558,15 @@ int if4_quantize_fused(const void *x, int x_dtype, int64_t rows, int64_t cols, i
                               sync_words, err_flag, stream, 0u);
 }
 
+int if4_quantize_fused_shared(const void *x, int x_dtype, int64_t rows, int64_t cols,
+                              int64_t ld_x, uint8_t *codes, uint8_t *scales, uint8_t *nv_codes,
+                              uint8_t *nv_scales, float *ts, uint32_t *sync_words, int share,
+                              int *err_flag, void *stream)
+{
+    return fused_entry<false>(x, x_dtype, rows, cols, ld_x, codes, scales, nv_codes, nv_scales, ts,
+                              sync_words, err_flag, stream, 0u, nullptr, share);
+}
+
 int if4_quantize_fused_dequant(const void *x, int x_dtype, int64_t rows, int64_t cols,
                                int64_t ld_x, uint8_t *codes, uint8_t *scales, uint8_t *nv_codes,
                                uint8_t *nv_scales, float *ts, uint32_t *sync_words, void *y,
@@ -1588,6 +1597,15 @@ int if4_quantize_fused_rht(const void *x, int x_dtype, int64_t rows, int64_t col
 {
     return fused_entry<true>(x, x_dtype, rows, cols, ld_x, codes, scales, nv_codes, nv_scales, ts,
                              sync_words, err_flag, stream, signs & 0xFFFFu);
+}
+
+int if4_quantize_fused_rht_shared(const void *x, int x_dtype, int64_t rows, int64_t cols,
+                                  int64_t ld_x, uint32_t signs, uint8_t *codes, uint8_t *scales,
+                                  uint8_t *nv_codes, uint8_t *nv_scales, float *ts,
+                                  uint32_t *sync_words, int share, int *err_flag, void *stream)
+{
+    return fused_entry<true>(x, x_dtype, rows, cols, ld_x, codes, scales, nv_codes, nv_scales, ts,
+                             sync_words, err_flag, stream, signs & 0xFFFFu, nullptr, share);
 }
 
 int if4_dequantize(const uint8_t *codes, const uint8_t *scales, const float *ts, int64_t rows,

@@ -198,20 +198,24 @@ int if4_quantize_fused_dequant(const void *x, int x_dtype, int64_t rows, int64_t
                                int *err_flag, void *stream);
 
 /*
- * if4_quantize_fused_dequant on a share of the device.  The launch sizes its
- * grid to floor(R / share) blocks per SM (at least one), R being the blocks
- * of this kernel one SM holds, so that `share` such calls on different
- * streams, each with its own sync_words, are resident together: the amax
- * pass of one runs beside the encode pass of another.  Independent tensors
- * (consecutive steps, the layers of a model) quantized this way on two
- * streams take less time in total than one after another on one stream,
- * while each call alone takes longer.  share = 1 is
- * if4_quantize_fused_dequant.  The outputs do not depend on share: they are
- * byte-identical to if4_quantize_fused_dequant's.  IF4_ERR_SHAPE for share
- * outside [1, 64]; other arguments and rules as if4_quantize_fused_dequant.
- * Launches that share the device must not wait for one another (each call
- * waits only for its own blocks).
+ * The single launches on a share of the device: if4_quantize_fused,
+ * if4_quantize_fused_dequant and if4_quantize_fused_rht with one more
+ * argument, share.  The launch sizes its grid to floor(R / share) blocks per
+ * SM (at least one), R being the blocks of its kernel one SM holds, so that
+ * `share` such calls on different streams, each with its own sync_words, are
+ * resident together: the amax pass of one runs beside the encode pass of
+ * another.  Independent tensors (consecutive steps, the layers of a model)
+ * quantized this way on two streams take less time in total than one after
+ * another on one stream, while each call alone takes longer.  share = 1 is
+ * the plain call.  The outputs do not depend on share: they are
+ * byte-identical to the plain call's.  IF4_ERR_SHAPE for share outside
+ * [1, 64]; other arguments and rules as the plain call.  Each call waits
+ * only for its own blocks, never for another launch.
  */
+int if4_quantize_fused_shared(const void *x, int x_dtype, int64_t rows, int64_t cols,
+                              int64_t ld_x, uint8_t *codes, uint8_t *scales, uint8_t *nv_codes,
+                              uint8_t *nv_scales, float *ts, uint32_t *sync_words, int share,
+                              int *err_flag, void *stream);
 int if4_quantize_fused_dequant_shared(const void *x, int x_dtype, int64_t rows, int64_t cols,
                                       int64_t ld_x, uint8_t *codes, uint8_t *scales,
                                       uint8_t *nv_codes, uint8_t *nv_scales, float *ts,
@@ -229,6 +233,12 @@ int if4_quantize_fused_rht(const void *x, int x_dtype, int64_t rows, int64_t col
                            uint32_t signs, uint8_t *codes, uint8_t *scales, uint8_t *nv_codes,
                            uint8_t *nv_scales, float *ts, uint32_t *sync_words, int *err_flag,
                            void *stream);
+/* if4_quantize_fused_rht on a share of the device, as the shared launches
+ * above. */
+int if4_quantize_fused_rht_shared(const void *x, int x_dtype, int64_t rows, int64_t cols,
+                                  int64_t ld_x, uint32_t signs, uint8_t *codes, uint8_t *scales,
+                                  uint8_t *nv_codes, uint8_t *nv_scales, float *ts,
+                                  uint32_t *sync_words, int share, int *err_flag, void *stream);
 
 /*
  * Comparator, all-INT4 ("NVINT4"): the 7/6-scaled INT4 candidate of

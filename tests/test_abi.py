@@ -32,6 +32,10 @@ def lib():
                                              vp, vp]
     L.if4_quantize_fused_dequant_shared.argtypes = [vp, i, i64, i64, i64, vp, vp, vp, vp, vp, vp,
                                                     vp, i, vp, vp]
+    L.if4_quantize_fused_shared.argtypes = [vp, i, i64, i64, i64, vp, vp, vp, vp, vp, vp, i, vp,
+                                            vp]
+    L.if4_quantize_fused_rht_shared.argtypes = [vp, i, i64, i64, i64, ctypes.c_uint32, vp, vp,
+                                                vp, vp, vp, vp, i, vp, vp]
     L.if4_linear_quantized.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, ctypes.c_size_t,
                                        vp, vp, vp, vp, vp, vp]
     L.if4_linear_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
@@ -138,6 +142,13 @@ def test_fused_quantize_host_validation(lib):
     assert k(A, 1, 4, 32, 32, A, A, None, None, A, A, A + 16, 2, None, None) == 4
     assert k(A, 1, 4, 24, 24, A, A, None, None, A, A, A, 2, None, None) == 2
     assert k(A, 1, 4, 32, 32, A, A, None, None, A, A + 64, A, 2, None, None) == 4
+    m = lib.if4_quantize_fused_shared
+    assert m(A, 1, 4, 32, 32, A, A, None, None, A, A, 0, None, None) == 2
+    assert m(A, 1, 4, 32, 32, A, A, None, None, None, A, 2, None, None) == 1
+    assert m(A, 1, 4, 32, 32, A, A, None, None, A, A + 64, 2, None, None) == 4
+    n = lib.if4_quantize_fused_rht_shared
+    assert n(A, 1, 4, 32, 32, 0x1234, A, A, None, None, A, A, 65, None, None) == 2
+    assert n(A, 1, 4, 32, 32, 0x1234, A, A, None, None, None, A, 2, None, None) == 1
     g = lib.if4_quantize_fused_rht
     assert g(A, 1, 4, 32, 32, 0x1234, A, A, None, None, None, A, None, None) == 1
     assert g(A, 1, 4, 24, 24, 0x1234, A, A, None, None, A, A, None, None) == 2

@@ -347,3 +347,30 @@ def test_shared_launches_on_two_streams_at_once():
     for k in (0, 1):
         assert bufs[k]["sync"][0].item() == 0 and bufs[k]["sync"][1].item() == 0
         assert _same(bufs[k], refs[k])
+
+
+@pytest.mark.parametrize("signs", [None, 0xA5C3])
+@pytest.mark.parametrize("share", [2, 64])
+def test_shared_single_launch_is_byte_identical(signs, share):
+    """if4_quantize_fused_shared and if4_quantize_fused_rht_shared: the same
+    codes, scales, ts and NVFP4 output as the plain single launch."""
+    b = B()
+    x = workloads.hadamard_gradient(1, rows=2048, cols=4096).cuda()
+    rows, cols = x.shape
+    ref = [torch.empty((rows, cols // 2), dtype=torch.uint8, device="cuda"),
+           torch.empty((rows, cols // 16), dtype=torch.uint8, device="cuda"),
+           torch.empty((rows, cols // 2), dtype=torch.uint8, device="cuda"),
+           torch.empty((rows, cols // 16), dtype=torch.uint8, device="cuda"),
+           torch.empty(1, dtype=torch.float32, device="cuda")]
+    got = [torch.empty_like(t) for t in ref]
+    s0 = torch.zeros(b.FUSED_SYNC_WORDS, dtype=torch.int32, device="cuda")
+    s1 = torch.zeros(b.FUSED_SYNC_WORDS, dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    b.if4_quantize_fused(x, ref[0], ref[1], ref[2], ref[3], ref[4], s0, err_flag=err, signs=signs)
+    b.if4_quantize_fused_shared(x, got[0], got[1], got[2], got[3], got[4], s1, share,
+                                err_flag=err, signs=signs)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and s1[0].item() == 0 and s1[1].item() == 0
+    for a, c in zip(ref, got):
+        assert torch.equal(a, c)
+
