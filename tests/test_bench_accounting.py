@@ -14,7 +14,9 @@ import bench  # noqa: E402
 def test_algorithmic_bytes_per_element(elem_bytes):
     n = 4096 * 4096
     names = ["fused_quantize_dequant", "fused_quantize", "amax", "if4_quantize",
-             "if4_dequantize", "nvfp4_quantize", "if4_decode_f16"]
+             "if4_dequantize", "nvfp4_quantize", "if4_decode_f16", "nvint4_quantize",
+             "nvfp4_4over6_quantize", "if4_quantize_rht", "fused_quantize_rht", "if6_quantize",
+             "if3_quantize", "if6_dequantize", "if3_dequantize"]
     t = bench.kernel_table({k: 1.0 for k in names}, n, n * elem_bytes, {"hbm_gbs": 6552.0})
     codes = 0.5 + 1 / 16                        # 4-bit codes + one scale byte per 16
     want = {
@@ -25,6 +27,14 @@ def test_algorithmic_bytes_per_element(elem_bytes):
         "fused_quantize_dequant": elem_bytes + 2 * codes + 2,   # ... and the bf16 y
         "if4_dequantize": codes + 2,                        # codes in, bf16 out
         "if4_decode_f16": codes + 2,                        # codes in, fp16 out
+        "nvint4_quantize": elem_bytes + codes,
+        "nvfp4_4over6_quantize": elem_bytes + codes,
+        "if4_quantize_rht": elem_bytes + codes,             # the transform is in registers
+        "fused_quantize_rht": elem_bytes + 2 * codes,
+        "if6_quantize": elem_bytes + 6 / 8 + 1 / 16,        # 6-bit codes, one scale per 16
+        "if3_quantize": elem_bytes + 3 / 8 + 1 / 16,
+        "if6_dequantize": 6 / 8 + 1 / 16 + 2,               # bf16 out
+        "if3_dequantize": 3 / 8 + 1 / 16 + 2,
     }
     for k, per_elem in want.items():
         assert t[k]["bytes"] == pytest.approx(per_elem * n, rel=0, abs=0.5), k
