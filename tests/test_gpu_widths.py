@@ -147,3 +147,29 @@ def test_nonfinite_input_sets_flag(bits):
     b.quantize_w(x, bits, err_flag=err)
     torch.cuda.synchronize()
     assert int(err.item()) & b.DEV_NONFINITE
+
+
+@pytest.mark.parametrize("bits", [6, 3])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+def test_dequantize_arbitrary_codes(bits, dtype):
+    """Random code and scale bytes, every code value of both types (INT6 k =
+    -32 and INT3 k = -4 included, which the quantizer never writes; FP
+    negative zeros; every magnitude), decoded against the oracle's
+    dequantizer and rounded to the output type.  E4M3 NaN scale bytes
+    (0x7F, 0xFF) give NaN on both sides, compared as NaN."""
+    rng = np.random.default_rng(61 + bits)
+    rows, cols = 96, 512
+    codes = rng.integers(0, 256, (rows, cols * bits // 8), dtype=np.uint8)
+    scales = rng.integers(0, 256, (rows, cols // 16), dtype=np.uint8)
+    ts = np.float32(0.37)
+    want = torch.from_numpy(oracle.dequantize_w(codes, scales, ts, bits)).to(dtype)
+    b = B()
+    y = b.dequantize_w(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(),
+                       torch.tensor([ts], dtype=torch.float32, device="cuda"), bits,
+                       dtype=dtype).cpu()
+    nan = torch.isnan(want)
+    assert torch.equal(torch.isnan(y), nan)
+    iv = torch.int32 if dtype == torch.float32 else torch.int16
+    assert torch.equal(y[~nan].view(iv), want[~nan].view(iv))
+    assert nan.any() and (~nan).any()
+
