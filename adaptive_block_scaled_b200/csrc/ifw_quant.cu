@@ -675,11 +675,22 @@ ifw_dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restri
     // stores would each write half of every sector they touch)
     const bool v8 = contig && (reinterpret_cast<uintptr_t>(y) & 31u) == 0u;
     const uint32_t stride = gridDim.x * blockDim.x;
-    for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < ngroups; g += stride) {
-        uint32_t w[3], c[16];
-        load_code_words<BITS>(codes + (int64_t)g * CB, w);
+    const uint32_t g0 = blockIdx.x * blockDim.x + threadIdx.x;
+    // the next group's code words and scale byte are loaded once this
+    // group's codes are unpacked, into the same registers
+    uint32_t w[3] = {0u, 0u, 0u}, sbn = 0u;
+    if (g0 < ngroups) {
+        load_code_words<BITS>(codes + (int64_t)g0 * CB, w);
+        sbn = __ldg(scales + g0);
+    }
+    for (uint32_t g = g0; g < ngroups; g += stride) {
+        uint32_t c[16];
         unpack_code_words<BITS>(w, c);
-        const uint32_t sb = __ldg(scales + g);
+        const uint32_t sb = sbn;
+        if (g + stride < ngroups) {
+            load_code_words<BITS>(codes + (int64_t)(g + stride) * CB, w);
+            sbn = __ldg(scales + g + stride);
+        }
         const float eff = __fmul_rn(f32_from_e4m3(sb & 0x7Fu), ts);
         const float *tab = (sb & 0x80u) ? int_tab : fp_tab;
         float yv[16];
