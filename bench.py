@@ -998,6 +998,9 @@ def run_ours(args):
             "two_streams_shared": {
                 "ms_per_step": ms_two_streams,
                 "value": world * n_elem / (ms_two_streams * 1e-3) / 1e9, "unit": UNIT,
+                "gbs": kernels["fused_quantize_dequant"]["bytes"] / (ms_two_streams * 1e-3) / 1e9,
+                "frac_of_measured_hbm": kernels["fused_quantize_dequant"]["bytes"]
+                / (ms_two_streams * 1e-3) / 1e9 / pk["hbm_gbs"],
                 "how": "the same K steps as one CUDA graph, consecutive steps alternating "
                        "between two streams, each step one if4_quantize_fused_dequant_shared "
                        "launch with share 2 (half the resident blocks per SM), so one "
